@@ -1,0 +1,387 @@
+/*
+ * tf4_oracle.c -- plain, slow, obviously-correct CPU oracle.
+ *
+ * TEST INFRASTRUCTURE ONLY (see tf4_oracle.h for who may use it and for
+ * the pages each definition follows).  Built with -O2 -ffp-contract=off so
+ * that every float expression below is one IEEE binary32 operation with
+ * round-to-nearest-even, exactly as written.
+ *
+ * Exactness notes used throughout:
+ *  - a bf16 value has at most 8 significant bits, an fp32 scale S at most
+ *    24, and every E2M1 codeword or midpoint is k/4 with k < 32, so a
+ *    product (codeword or midpoint) * S is exact in double (<= 29 bits);
+ *  - every decision below is a comparison between two such exact doubles,
+ *    never a comparison of a rounded quotient; "y = |x| / S" is the real
+ *    quotient, compared through |x| vs c*S.
+ */
+#include "tf4_oracle.h"
+
+#include <math.h>
+#include <string.h>
+
+/* E2M1 magnitudes indexed by m3 = exponent(2 bits)<<1 | mantissa(1 bit).
+ * [FQT] section 3: E2M1 = 2-bit exponent, 1-bit mantissa. */
+static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
+
+float orc_bf16_to_float(uint16_t h) {
+  uint32_t u = (uint32_t)h << 16; /* bf16 is the top half of an fp32 */
+  float f;
+  memcpy(&f, &u, sizeof f);
+  return f;
+}
+
+static int bf16_is_finite(uint16_t h) { return (h & 0x7F80u) != 0x7F80u; }
+static int bf16_sign(uint16_t h) { return (h >> 15) & 1; }
+static double bf16_abs(uint16_t h) { return (double)orc_bf16_to_float((uint16_t)(h & 0x7FFFu)); }
+
+double orc_e2m1_value(int m3) { return kE2M1[m3 & 7]; }
+
+/* E4M3 ("fn" variant: no infinities, 0x7F/0xFF are NaN): bias 7,
+ * subnormals m * 2^-9, largest finite 448 (0x7E).  [FQT] section 3 names
+ * E4M3 as the NVFP4 block-scale format. */
+double orc_e4m3_value(uint8_t code) {
+  int sign = code >> 7, e = (code >> 3) & 0xF, m = code & 7;
+  double v;
+  if (e == 0xF && m == 7) return NAN;
+  if (e == 0)
+    v = ldexp((double)m, -9);
+  else
+    v = ldexp(1.0 + m / 8.0, e - 7);
+  return sign ? -v : v;
+}
+
+/* Round a non-negative finite fp32 to E4M3: the nearest of the 127
+ * non-negative finite codes, ties to the even code (even mantissa),
+ * anything above 448 saturates to 448.  Plain search over all codes. */
+uint8_t orc_e4m3_encode(float r) {
+  double rv = (double)r;
+  int best = 0;
+  for (int c = 1; c <= 0x7E; ++c) {
+    double vb = orc_e4m3_value((uint8_t)best), vc = orc_e4m3_value((uint8_t)c);
+    double db = fabs(rv - vb), dc = fabs(rv - vc); /* exact: both near rv, few bits */
+    if (dc < db || (dc == db && (c & 1) == 0)) best = c;
+  }
+  return (uint8_t)best;
+}
+
+/* MXFP4 shared exponent: floor(log2(bamax)) - 2, clamped to the E8M0
+ * range [-127, 127]; an all-zero block takes -127.  [TETRAJET] section 3
+ * (per-group scale).  floor(log2) is read exactly from frexp. */
+int orc_e8m0_exponent(float bamax) {
+  int ex;
+  if (bamax == 0.0f) return -127;
+  (void)frexp((double)bamax, &ex); /* bamax = f * 2^ex, f in [0.5, 1) */
+  int e = (ex - 1) - 2;
+  if (e < -127) e = -127;
+  if (e > 127) e = 127;
+  return e;
+}
+
+/* NVFP4 per-tensor scale s_t = amax / (6 * 448) in fp32.  A result below
+ * the smallest normal fp32 (including amax == 0) makes the whole segment
+ * quantize to signed zeros with s_t = 0. */
+float orc_nvfp4_tensor_scale(float amax) {
+  float s = amax / 2688.0f;
+  if (!(s >= 0x1p-126f)) s = 0.0f;
+  return s;
+}
+
+/* NVFP4 block scale code: b = E4M3( (bamax / 6) / s_t ), two fp32 divides
+ * in that order; s_t == 0 gives 0. */
+uint8_t orc_nvfp4_block_scale_code(float bamax, float s_t) {
+  if (s_t == 0.0f) return 0;
+  float q = bamax / 6.0f;
+  float r = q / s_t;
+  return orc_e4m3_encode(r);
+}
+
+/* Effective block scale S = s_t * dec(b), one fp32 multiply. */
+float orc_nvfp4_block_scale(uint8_t code, float s_t) {
+  float d = (float)orc_e4m3_value(code);
+  return s_t * d;
+}
+
+float orc_mxfp4_block_scale(uint8_t code) { return (float)ldexp(1.0, (int)code - 127); }
+
+/* Round-to-nearest: the codeword nearest to y = ax / S (real quotient),
+ * ties to the even m3; saturation at 6 is the nearest-codeword rule itself.
+ * [TRACE-JA] mismatch section: plain nearest rounding is what the rollout
+ * does; [FQT] section 3: round-to-nearest in the forward pass.
+ * Scan the sorted grid; codeword j beats the current best b (< j) iff y is
+ * above their midpoint, i.e. 2*ax > (V_b + V_j) * S (both sides exact). */
+int orc_rtn_m3(double ax, double S) {
+  if (S == 0.0) return 0;
+  int best = 0;
+  for (int j = 1; j < 8; ++j) {
+    double lhs = 2.0 * ax, rhs = (kE2M1[best] + kE2M1[j]) * S;
+    if (lhs > rhs || (lhs == rhs && (j % 2) == 0)) best = j;
+  }
+  return best;
+}
+
+/* Neighbours of y = ax / S on the grid (S > 0, y < 6, y not a codeword):
+ * lo = the largest j with V_j * S < ax. */
+static int grid_floor(double ax, double S) {
+  int lo = 0;
+  for (int j = 1; j < 8; ++j)
+    if (kE2M1[j] * S < ax) lo = j;
+  return lo;
+}
+
+/* Index of the codeword equal to y, or -1. */
+static int grid_exact(double ax, double S) {
+  for (int j = 0; j < 8; ++j)
+    if (kE2M1[j] * S == ax) return j;
+  return -1;
+}
+
+/* Stochastic rounding with a 24-bit uniform integer r: between the two
+ * neighbours lo < y < hi round up iff r < 2^24 (y - lo) / (hi - lo), i.e.
+ * r * (V_hi - V_lo) * S < 2^24 * (ax - V_lo * S).  Left side: <= 48 bits;
+ * right side: ax and V_lo*S within a factor 2 (or V_lo = 0), so the
+ * difference is exact (Sterbenz) -- both sides exact in double.
+ * y >= 6 saturates to 6; a codeword keeps itself.  [FQT] section 3. */
+int orc_sr_m3(double ax, double S, uint32_t r24) {
+  if (S == 0.0) return 0;
+  if (ax >= 6.0 * S) return 7;
+  int ex = grid_exact(ax, S);
+  if (ex >= 0) return ex;
+  int lo = grid_floor(ax, S), hi = lo + 1;
+  double lhs = (double)r24 * (kE2M1[hi] - kE2M1[lo]) * S;
+  double rhs = 16777216.0 * (ax - kE2M1[lo] * S);
+  return lhs < rhs ? hi : lo;
+}
+
+/* Rollout-guided rounding: of the two grid neighbours of y, take the one
+ * whose mantissa bit (m3 & 1) equals the recorded bit g.  Adjacent
+ * codewords always differ in that bit, so exactly one qualifies.  A value
+ * that is a codeword keeps it; y >= 6 gives 6 (both neighbours are 6).
+ * [TRACE-JA] mechanism section (the candidates are the two adjacent
+ * codewords, chosen by a light comparison) and quantization-info cache
+ * section (mantissa bit + scale identify the codeword). */
+int orc_guided_m3(double ax, double S, int g) {
+  if (S == 0.0) return 0;
+  if (ax >= 6.0 * S) return 7;
+  int ex = grid_exact(ax, S);
+  if (ex >= 0) return ex;
+  int lo = grid_floor(ax, S), hi = lo + 1;
+  return ((lo & 1) == (g & 1)) ? lo : hi;
+}
+
+/* Philox4x32-10 [PHILOX]: 10 rounds of the 4x32 Philox S-box; between
+ * rounds the 2-word key is bumped by the Weyl constants.  One round:
+ *   (hi0, lo0) = M0 * c0,  (hi1, lo1) = M1 * c2   (full 64-bit products)
+ *   c' = (hi1 ^ c1 ^ k0, lo1, hi0 ^ c3 ^ k1, lo0)                        */
+void orc_philox4x32_10(const uint32_t ctr[4], const uint32_t key[2], uint32_t out[4]) {
+  const uint32_t M0 = 0xD2511F53u, M1 = 0xCD9E8D57u;
+  const uint32_t W0 = 0x9E3779B9u, W1 = 0xBB67AE85u;
+  uint32_t c0 = ctr[0], c1 = ctr[1], c2 = ctr[2], c3 = ctr[3];
+  uint32_t k0 = key[0], k1 = key[1];
+  for (int round = 0; round < 10; ++round) {
+    if (round > 0) {
+      k0 += W0;
+      k1 += W1;
+    }
+    uint64_t p0 = (uint64_t)M0 * c0, p1 = (uint64_t)M1 * c2;
+    uint32_t n0 = (uint32_t)(p1 >> 32) ^ c1 ^ k0;
+    uint32_t n1 = (uint32_t)p1;
+    uint32_t n2 = (uint32_t)(p0 >> 32) ^ c3 ^ k1;
+    uint32_t n3 = (uint32_t)p0;
+    c0 = n0;
+    c1 = n1;
+    c2 = n2;
+    c3 = n3;
+  }
+  out[0] = c0;
+  out[1] = c1;
+  out[2] = c2;
+  out[3] = c3;
+}
+
+/* The uniform used by stochastic rounding of element idx: word 0 of
+ * Philox4x32-10 at counter (idx_lo, idx_hi, 0, 0), key (seed_lo, seed_hi),
+ * top 24 bits. */
+uint32_t orc_sr_uniform24(uint64_t idx, uint64_t seed) {
+  uint32_t ctr[4] = {(uint32_t)idx, (uint32_t)(idx >> 32), 0u, 0u};
+  uint32_t key[2] = {(uint32_t)seed, (uint32_t)(seed >> 32)};
+  uint32_t out[4];
+  orc_philox4x32_10(ctr, key, out);
+  return out[0] >> 8;
+}
+
+/* ---------------------------------------------------------------------- */
+/* tensor level                                                            */
+
+static int64_t seg_begin(const int64_t* off, int32_t s, int64_t rows) {
+  (void)rows;
+  return off ? off[s] : 0;
+}
+static int64_t seg_end(const int64_t* off, int32_t s, int64_t rows) { return off ? off[s + 1] : rows; }
+
+static int32_t segment_of_row(const int64_t* off, int32_t nseg, int64_t row) {
+  if (!off) return 0;
+  for (int32_t s = 0; s < nseg; ++s)
+    if (row >= off[s] && row < off[s + 1]) return s;
+  return nseg - 1;
+}
+
+/* Per-segment max |x|.  Non-finite inputs set ORC_NONFINITE and make that
+ * segment's amax NaN. */
+int orc_segment_amax(const uint16_t* x, int64_t rows, int64_t cols, int32_t nseg,
+                     const int64_t* seg_off, float* amax_out) {
+  int status = 0;
+  for (int32_t s = 0; s < nseg; ++s) {
+    float m = 0.0f;
+    int bad = 0;
+    for (int64_t r = seg_begin(seg_off, s, rows); r < seg_end(seg_off, s, rows); ++r)
+      for (int64_t c = 0; c < cols; ++c) {
+        uint16_t h = x[r * cols + c];
+        if (!bf16_is_finite(h)) {
+          bad = 1;
+          continue;
+        }
+        float a = (float)bf16_abs(h);
+        if (a > m) m = a;
+      }
+    amax_out[s] = bad ? NAN : m;
+    if (bad) status |= ORC_NONFINITE;
+  }
+  return status;
+}
+
+int orc_segment_scales(const uint16_t* x, int64_t rows, int64_t cols, int32_t nseg,
+                       const int64_t* seg_off, float* s_t_out) {
+  int status = orc_segment_amax(x, rows, cols, nseg, seg_off, s_t_out);
+  for (int32_t s = 0; s < nseg; ++s)
+    s_t_out[s] = isnan(s_t_out[s]) ? NAN : orc_nvfp4_tensor_scale(s_t_out[s]);
+  return status;
+}
+
+static void put_code(uint8_t* codes, int64_t i, int nib) {
+  uint8_t* p = &codes[i >> 1];
+  if (i & 1)
+    *p = (uint8_t)((*p & 0x0F) | (nib << 4));
+  else
+    *p = (uint8_t)((*p & 0xF0) | nib);
+}
+static int get_code(const uint8_t* codes, int64_t i) { return (codes[i >> 1] >> ((i & 1) * 4)) & 0xF; }
+static void put_bit(uint8_t* bits, int64_t i, int b) {
+  uint8_t* p = &bits[i >> 3];
+  *p = (uint8_t)((*p & ~(1u << (i & 7))) | ((b & 1u) << (i & 7)));
+}
+static int get_bit(const uint8_t* bits, int64_t i) { return (bits[i >> 3] >> (i & 7)) & 1; }
+
+/* Quantize rows [row_begin, row_end) with RTN (mode 0) or SR (mode 1).
+ * NVFP4 takes the per-segment s_t (from orc_segment_scales); MXFP4 ignores
+ * s_t.  Writes the codes, the scale bytes and, if bits != NULL, the
+ * guidance bits of those rows (arrays are full-tensor sized). */
+int orc_quantize_rows(int fmt, int mode, const uint16_t* x, int64_t rows, int64_t cols,
+                      int32_t nseg, const int64_t* seg_off, const float* s_t, uint64_t seed,
+                      int64_t row_begin, int64_t row_end, uint8_t* codes, uint8_t* scales,
+                      uint8_t* bits) {
+  const int block = fmt == ORC_NVFP4 ? 16 : 32;
+  const int64_t nblk_row = cols / block;
+  int status = 0;
+  (void)rows;
+  for (int64_t r = row_begin; r < row_end; ++r) {
+    float st = fmt == ORC_NVFP4 ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
+    if (fmt == ORC_NVFP4 && isnan(st)) status |= ORC_NONFINITE;
+    for (int64_t b = 0; b < nblk_row; ++b) {
+      const int64_t base = r * cols + b * block;
+      float bamax = 0.0f;
+      int bad = 0;
+      for (int k = 0; k < block; ++k) {
+        uint16_t h = x[base + k];
+        if (!bf16_is_finite(h)) bad = 1;
+        else if ((float)bf16_abs(h) > bamax) bamax = (float)bf16_abs(h);
+      }
+      if (bad) status |= ORC_NONFINITE;
+      uint8_t sc;
+      double S;
+      if (fmt == ORC_NVFP4) {
+        sc = (isnan(st) || bad) ? 0 : orc_nvfp4_block_scale_code(bamax, st);
+        S = (isnan(st) || bad) ? 0.0 : (double)orc_nvfp4_block_scale(sc, st);
+      } else {
+        int e = orc_e8m0_exponent(bamax);
+        sc = (uint8_t)(e + 127);
+        S = (double)orc_mxfp4_block_scale(sc);
+      }
+      scales[r * nblk_row + b] = sc;
+      for (int k = 0; k < block; ++k) {
+        const int64_t i = base + k;
+        uint16_t h = x[i];
+        int m3 = 0;
+        if (!bad) {
+          double ax = bf16_abs(h);
+          m3 = mode == ORC_SR ? orc_sr_m3(ax, S, orc_sr_uniform24((uint64_t)i, seed)) : orc_rtn_m3(ax, S);
+        }
+        put_code(codes, i, (bf16_sign(h) << 3) | m3);
+        if (bits) put_bit(bits, i, m3 & 1);
+      }
+    }
+  }
+  return status;
+}
+
+/* Train-side guided quantization of rows [row_begin, row_end): S comes
+ * from the recorded scale byte (and recorded s_t for NVFP4) exactly as on
+ * the rollout side; the sign is the train value's own. */
+int orc_quantize_guided_rows(int fmt, const uint16_t* x, int64_t rows, int64_t cols,
+                             int32_t nseg, const int64_t* seg_off, const uint8_t* rec_scales,
+                             const float* rec_s_t, const uint8_t* rec_bits, int64_t row_begin,
+                             int64_t row_end, uint8_t* codes) {
+  const int block = fmt == ORC_NVFP4 ? 16 : 32;
+  const int64_t nblk_row = cols / block;
+  int status = 0;
+  (void)rows;
+  for (int64_t r = row_begin; r < row_end; ++r) {
+    float st = fmt == ORC_NVFP4 ? rec_s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
+    for (int64_t b = 0; b < nblk_row; ++b) {
+      const int64_t base = r * cols + b * block;
+      uint8_t sc = rec_scales[r * nblk_row + b];
+      double S = fmt == ORC_NVFP4 ? (double)orc_nvfp4_block_scale(sc, st) : (double)orc_mxfp4_block_scale(sc);
+      int bad = 0;
+      for (int k = 0; k < block; ++k)
+        if (!bf16_is_finite(x[base + k])) bad = 1;
+      if (bad) status |= ORC_NONFINITE;
+      for (int k = 0; k < block; ++k) {
+        const int64_t i = base + k;
+        uint16_t h = x[i];
+        int m3 = bad ? 0 : orc_guided_m3(bf16_abs(h), S, get_bit(rec_bits, i));
+        put_code(codes, i, (bf16_sign(h) << 3) | m3);
+      }
+    }
+  }
+  return status;
+}
+
+/* Dequantize rows: out = (-1)^sign * RN_fp32(V[m3] * S); V*S is exact in
+ * double, so the cast is the single rounding. */
+void orc_dequantize_rows(int fmt, const uint8_t* codes, const uint8_t* scales, const float* s_t,
+                         int64_t rows, int64_t cols, int32_t nseg, const int64_t* seg_off,
+                         int64_t row_begin, int64_t row_end, float* out) {
+  const int block = fmt == ORC_NVFP4 ? 16 : 32;
+  const int64_t nblk_row = cols / block;
+  (void)rows;
+  for (int64_t r = row_begin; r < row_end; ++r) {
+    float st = fmt == ORC_NVFP4 ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
+    for (int64_t c = 0; c < cols; ++c) {
+      const int64_t i = r * cols + c;
+      uint8_t sc = scales[r * nblk_row + c / block];
+      double S = fmt == ORC_NVFP4 ? (double)orc_nvfp4_block_scale(sc, st) : (double)orc_mxfp4_block_scale(sc);
+      int nib = get_code(codes, i);
+      float mag = (float)(kE2M1[nib & 7] * S);
+      out[i] = (nib & 8) ? -mag : mag;
+    }
+  }
+}
+
+/* Guidance extraction from codes ([TRACE-JA] quantization-info cache:
+ * the mantissa bit is what is kept). */
+void orc_pack_guidance(const uint8_t* codes, int64_t n, uint8_t* bits) {
+  for (int64_t i = 0; i < n; ++i) put_bit(bits, i, get_code(codes, i) & 1);
+}
+
+void orc_unpack_guidance(const uint8_t* bits, int64_t n, uint8_t* mant) {
+  for (int64_t i = 0; i < n; ++i) mant[i] = (uint8_t)get_bit(bits, i);
+}
