@@ -1,0 +1,519 @@
+#!/usr/bin/env python
+"""Benchmark of the block-scaled FP4 quantization path on B200.
+
+One step = the whole path over the 40-layer activation stack (65536 x 4096
+bf16 per layer, 0.5 * Student-t(4) times per-channel LogNormal(0,1)):
+  rollout side: NVFP4 amax pass + capture for all 40 layers, with guidance
+                bits kept for the deepest 20 (layers 20..39);
+  train side:   guided quantization of perturbed copies of layers 20..39
+                against their records.
+Metric: algorithmic GB/s (bytes the definition forces per element: two
+reads of x for the tensor-scale pass, the code / scale / guidance writes,
+the guided pass's reads and writes), as a fraction of measured HBM copy
+bandwidth.  Inputs (512 MiB per layer) exceed the 126 MB L2, so no flush.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Multi-GPU (torchrun, one rank per GPU): every rank quantizes its own stack
+(weak scaling, no collective on the data path); the time is the max over
+ranks.  ``--impl reference`` times the CPU oracle on a bounded row sample
+of the same workload instead.
+"""
+import argparse
+import hashlib
+import json
+import os
+import shutil
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "quantize/capture/guided GB/s and % of B200 HBM peak (1 GPU)"
+FALLBACK_HBM_GBS = 6650.0
+DATASHEET_HBM_GBS = 8000.0
+
+# algorithmic bytes per element (see the module docstring)
+B_AMAX = 2.0                       # read x
+B_QUANT = 2.0 + 0.5 + 1.0 / 16     # read x, write codes + scale bytes
+B_BITS = 1.0 / 8                   # guidance bits written by capture
+B_GUIDED = 2.0 + 1.0 / 16 + 1.0 / 8 + 0.5  # read x', scales, bits; write codes
+
+
+def parse():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--layers", type=int, default=40)
+    p.add_argument("--deep", type=int, default=20)
+    p.add_argument("--rows", type=int, default=65536)
+    p.add_argument("--cols", type=int, default=4096)
+    p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--cpu-rows", type=int, default=256, help="rows per layer in the oracle sample")
+    p.add_argument("--ref-rows", type=int, default=48, help="rows per layer per reference step")
+    return p.parse_args()
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+def max_over_ranks(v, world, dev):
+    if world == 1:
+        return v
+    import torch.distributed as dist
+
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------- clocks
+class Clocks:
+    """nvidia-smi samples (every 200 ms) during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        if not shutil.which("nvidia-smi"):
+            return
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        self.f = open(self.path, "w")
+        self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                                      "--format=csv,noheader,nounits", "-lms", "200"],
+                                     stdout=self.f, stderr=subprocess.DEVNULL)
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            p = [s.strip() for s in line.split(",")]
+            if len(p) < 9:
+                continue
+            try:
+                rows.append(dict(sm=float(p[1]), max=float(p[2]), power=float(p[3]), hw=p[5], hwt=p[6],
+                                 swt=p[7], pcap=p[8]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        loaded = [r for r in rows if r["power"] > 200] or rows
+        reasons = set()
+        for r in rows:
+            for k, name in (("hw", "hw_slowdown"), ("hwt", "hw_thermal_slowdown"),
+                            ("swt", "sw_thermal_slowdown"), ("pcap", "sw_power_cap")):
+                if r[k].lower() == "active":
+                    reasons.add(name)
+        return dict(sm_mhz=statistics.median(r["sm"] for r in loaded), sm_max_mhz=max(r["max"] for r in rows),
+                    reasons=sorted(reasons), samples=len(rows), power_w_max=max(r["power"] for r in rows))
+
+
+def hbm_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for rel in ("fp4_block_scaled_quantizer_b200/csrc/tf4_kernels.cuh", "fp4_block_scaled_quantizer_b200/csrc/trace_fp4.cu"):
+        with open(os.path.join(ROOT, rel), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel_key):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(p) as f:
+            t = json.load(f)
+    except Exception:
+        return None
+    e = t.get(kernel_key)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e
+
+
+# ------------------------------------------------------------- workload
+def make_stack(args, dev):
+    from fp4_block_scaled_quantizer_b200 import workloads as W
+
+    xs, xts = [], []
+    for layer in range(args.layers):
+        x = W.layer_stack_layer(layer, dev, rows=args.rows, cols=args.cols)
+        xs.append(x)
+        if layer >= args.layers - args.deep:
+            xts.append(W.perturb(x, 1000 + layer))
+    torch.cuda.synchronize()
+    return xs, xts
+
+
+def step_bytes(args):
+    n = args.rows * args.cols
+    deep = args.deep
+    shallow = args.layers - deep
+    cap = n * (args.layers * (B_AMAX + B_QUANT) + deep * B_BITS)
+    gd = n * deep * B_GUIDED
+    return cap + gd, n * (args.layers + deep)
+
+
+def run_ours(args, world, rank, local):
+    import fp4_block_scaled_quantizer_b200 as tf4
+    from fp4_block_scaled_quantizer_b200 import binding as B
+    from fp4_block_scaled_quantizer_b200 import build as libbuild
+
+    libbuild.build()
+    B.lib()
+    dev = torch.device("cuda", local)
+    stream = torch.cuda.current_stream(dev)
+    xs, xts = make_stack(args, dev)
+    L, D = args.layers, args.deep
+    first_deep = L - D
+    n = args.rows * args.cols
+    recs = [tf4.tf4_quantize_capture(xs[i], guidance=i >= first_deep) for i in range(L)]
+    amax = [torch.empty(1, dtype=torch.float32, device=dev) for _ in range(L)]
+    gcodes = [torch.empty(n // 2, dtype=torch.uint8, device=dev) for _ in range(D)]
+    torch.cuda.synchronize()
+
+    def new_events(count):
+        return [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(count)]
+
+    def step(ev):
+        for i in range(L):
+            if ev:
+                ev["amax"][i][0].record(stream)
+            B.tf4_segment_amax(xs[i], out=amax[i])
+            if ev:
+                ev["amax"][i][1].record(stream)
+                ev["quant"][i][0].record(stream)
+            B.tf4_quantize_capture(xs[i], guidance=i >= first_deep, amax_in=amax[i], out=recs[i])
+            if ev:
+                ev["quant"][i][1].record(stream)
+        for j in range(D):
+            if ev:
+                ev["guided"][j][0].record(stream)
+            B.tf4_quantize_guided(xts[j], recs[first_deep + j], out=gcodes[j])
+            if ev:
+                ev["guided"][j][1].record(stream)
+
+    launches_per_step = 2 * L + D
+    for _ in range(args.warmup):
+        step(None)
+    torch.cuda.synchronize()
+    assert B.read_status(dev) == 0, "non-finite input in the workload"
+    # per-kernel events for every timed step, read after the timed region
+    evs = [dict(amax=new_events(L), quant=new_events(L), guided=new_events(D)) for _ in range(args.steps)]
+
+    clocks = Clocks(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for k in range(args.steps):
+        step(evs[k])
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    ms_total = t0.elapsed_time(t1)
+    ms_step = max_over_ranks(ms_total / args.steps, world, dev)
+    times = {k: [[a.elapsed_time(b) for a, b in e[k]] for e in evs] for k in ("amax", "quant", "guided")}
+
+    bytes_step, elems_step = step_bytes(args)
+    value = world * bytes_step / (ms_step * 1e-3) / 1e9
+    peak, peak_kind = hbm_peak()
+
+    # per-kernel averages
+    def avg(k):
+        return statistics.mean(v for s in times[k] for v in s)
+
+    quant_bytes = [n * (B_QUANT + (B_BITS if i >= first_deep else 0.0)) for i in range(L)]
+    per_kernel = {
+        "amax": dict(ms=avg("amax"), bytes=n * B_AMAX),
+        "quant": dict(ms=avg("quant"), bytes=statistics.mean(quant_bytes)),
+        "guided": dict(ms=avg("guided"), bytes=n * B_GUIDED),
+    }
+    shares = {k: sum(sum(s) for s in times[k]) for k in times}
+    tot = sum(shares.values())
+    calls = {}
+    for k, v in per_kernel.items():
+        gbs = v["bytes"] / (v["ms"] * 1e-3) / 1e9
+        calls[k] = dict(us=round(v["ms"] * 1e3, 2), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
+                        share=round(shares[k] / tot, 4))
+    dom = max(shares, key=shares.get)
+    kname = {"amax": "k_amax", "quant": "k_quant(NVFP4, capture)", "guided": "k_guided(NVFP4)"}[dom]
+    achieved = per_kernel[dom]["bytes"] / (per_kernel[dom]["ms"] * 1e-3) / 1e9
+    tr = ncu_traffic(dom)
+    roofline = dict(bound="hbm", kernel=kname, achieved=round(achieved, 1), peak=peak, unit="GB/s",
+                    frac=round(achieved / peak, 4), peak_kind=f"{peak_kind} copy bandwidth",
+                    traffic=(tr["dram_bytes_per_launch"] if tr else None),
+                    algorithmic_bytes_per_launch=per_kernel[dom]["bytes"])
+
+    out = dict(metric=METRIC, value=round(value, 1), unit="GB/s", n_gpus=world, steps=args.steps,
+               warmup=args.warmup, ms_per_step=round(ms_step, 4), higher_is_better=True, scaling="weak",
+               vs_baseline=None, dtype="f32", data="synthetic",
+               config=dict(workload=f"layer_stack: {L} layers x {args.rows}x{args.cols} bf16 "
+                                    f"(0.5*t4 x LogNormal channel scales), NVFP4 capture with guidance for "
+                                    f"layers {first_deep}-{L - 1}, guided quantization of perturbed copies "
+                                    f"of those layers",
+                           layers=L, deep_layers=D, rows=args.rows, cols=args.cols, format="NVFP4",
+                           parallelism=f"dp{world} (independent stacks)",
+                           l2="inputs 512 MiB per layer > 126 MB L2; no flush"),
+               frac_of_peak=round(value / world / peak, 4),
+               frac_of_datasheet=round(value / world / DATASHEET_HBM_GBS, 4),
+               elements_per_s=round(world * elems_step / (ms_step * 1e-3), 1),
+               calls=calls, roofline=roofline, gpu_launches=launches_per_step * args.steps,
+               clocks=clk)
+
+    if not args.no_e2e:
+        out["e2e"] = run_e2e(args, world, dev, xs, xts, recs, amax, gcodes)
+    for t in (xs, xts, gcodes):
+        t.clear()
+    recs.clear()
+    torch.cuda.empty_cache()
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args, args.cpu_rows)
+    return out
+
+
+def run_e2e(args, world, dev, xs, xts, recs, amax, gcodes):
+    """Same step through the public API with host buffers: every step copies
+    the layers' inputs from pinned host memory (double-buffered on a copy
+    stream) and reads every result back to pinned host memory."""
+    import psutil
+
+    from fp4_block_scaled_quantizer_b200 import binding as B
+
+    L, D = args.layers, args.deep
+    first_deep = L - D
+    n = args.rows * args.cols
+    in_bytes = (L + D) * n * 2
+    out_bytes = L * (n // 2 + n // 16 + 4) + D * (n // 8 + n // 2)
+    if psutil.virtual_memory().available < 1.6 * (in_bytes + out_bytes):
+        return dict(value=None, unit="GB/s", skipped="not enough host memory for pinned buffers")
+    hx = [torch.empty_like(x, device="cpu").pin_memory() for x in xs]
+    hxt = [torch.empty_like(x, device="cpu").pin_memory() for x in xts]
+    for h, x in zip(hx + hxt, xs + xts):
+        h.copy_(x)
+    hc = [torch.empty(n // 2, dtype=torch.uint8).pin_memory() for _ in range(L)]
+    hs = [torch.empty(n // 16, dtype=torch.uint8).pin_memory() for _ in range(L)]
+    hst = torch.empty(L, dtype=torch.float32).pin_memory()
+    hb = [torch.empty(n // 8, dtype=torch.uint8).pin_memory() for _ in range(D)]
+    hg = [torch.empty(n // 2, dtype=torch.uint8).pin_memory() for _ in range(D)]
+    # device staging: two input slots
+    slot = [torch.empty_like(xs[0]) for _ in range(2)]
+    comp = torch.cuda.current_stream(dev)
+    copy = torch.cuda.Stream(dev)
+    ready = [torch.cuda.Event() for _ in range(2)]
+    free = [torch.cuda.Event() for _ in range(2)]
+    out_stream = torch.cuda.Stream(dev)
+    done = [torch.cuda.Event() for _ in range(L + D)]
+
+    def e2e_step():
+        jobs = [("cap", i) for i in range(L)] + [("gd", j) for j in range(D)]
+        # prefetch first (slot 0 may still be read by the previous step)
+        with torch.cuda.stream(copy):
+            copy.wait_event(free[0])
+            slot[0].copy_(hx[0], non_blocking=True)
+            ready[0].record(copy)
+        for t, (kind, i) in enumerate(jobs):
+            s = t % 2
+            if t + 1 < len(jobs):
+                nk, ni = jobs[t + 1]
+                src = hx[ni] if nk == "cap" else hxt[ni]
+                with torch.cuda.stream(copy):
+                    if t >= 1:
+                        copy.wait_event(free[(t + 1) % 2])
+                    slot[(t + 1) % 2].copy_(src, non_blocking=True)
+                    ready[(t + 1) % 2].record(copy)
+            comp.wait_event(ready[s])
+            if kind == "cap":
+                B.tf4_segment_amax(slot[s], out=amax[i])
+                B.tf4_quantize_capture(slot[s], guidance=i >= first_deep, amax_in=amax[i], out=recs[i])
+            else:
+                B.tf4_quantize_guided(slot[s], recs[first_deep + i], out=gcodes[i])
+            free[s].record(comp)
+            done[t].record(comp)
+            with torch.cuda.stream(out_stream):
+                out_stream.wait_event(done[t])
+                if kind == "cap":
+                    hc[i].copy_(recs[i].codes, non_blocking=True)
+                    hs[i].copy_(recs[i].scales.view(-1), non_blocking=True)
+                    hst[i:i + 1].copy_(recs[i].s_t, non_blocking=True)
+                    if i >= first_deep:
+                        hb[i - first_deep].copy_(recs[i].bits, non_blocking=True)
+                else:
+                    hg[i].copy_(gcodes[i], non_blocking=True)
+        comp.wait_stream(out_stream)
+
+    for _ in range(1):
+        e2e_step()
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(comp)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    t1.record(comp)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(t0.elapsed_time(t1) / args.e2e_steps, world, dev)
+    bytes_step, _ = step_bytes(args)
+    return dict(value=round(world * bytes_step / (ms * 1e-3) / 1e9, 2), unit="GB/s", ms_per_step=round(ms, 2),
+                h2d_bytes_per_step=in_bytes, d2h_bytes_per_step=out_bytes, steps=args.e2e_steps,
+                overlap="double-buffered H2D on a copy stream, D2H on a third stream")
+
+
+# ---------------------------------------------------------- CPU oracle arm
+def oracle_sample_step(args, rows, xs_host, xts_host):
+    import oracle as O
+
+    L, D = args.layers, args.deep
+    first_deep = L - D
+    recs = []
+    for i in range(L):
+        recs.append(O.quantize(xs_host[i], O.NVFP4, O.RTN, bits=i >= first_deep))
+    for j in range(D):
+        r = recs[first_deep + j]
+        O.quantize_guided(xts_host[j], r["scales"], r["bits"], O.NVFP4, rec_s_t=r["s_t"])
+
+
+def sample_host(args, rows):
+    """The first `rows` rows of every layer (and of the perturbed copies), as
+    bf16 bit patterns on the host."""
+    from fp4_block_scaled_quantizer_b200 import workloads as W
+
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    xs, xts = [], []
+    for layer in range(args.layers):
+        x = W.layer_stack_layer(layer, dev, rows=args.rows, cols=args.cols)
+        xs.append(W.bf16_bits(x[:rows].contiguous()))
+        if layer >= args.layers - args.deep:
+            xts.append(W.bf16_bits(W.perturb(x, 1000 + layer)[:rows].contiguous()))
+        del x
+    return xs, xts
+
+
+def cpu_baseline(args, rows):
+    import oracle as O
+
+    O.lib()
+    xs, xts = sample_host(args, rows)
+    t = time.perf_counter()
+    oracle_sample_step(args, rows, xs, xts)
+    dt = time.perf_counter() - t
+    sample_args = argparse.Namespace(**{**vars(args), "rows": rows})
+    b, _ = step_bytes(sample_args)
+    return dict(value=round(b / dt / 1e9, 4), unit="GB/s", cores=1, kind="oracle",
+                sample=f"first {rows} of {args.rows} rows of each of the {args.layers} layers "
+                       f"(capture) and of the {args.deep} perturbed deep layers (guided); "
+                       f"{dt:.1f} s single-threaded C oracle")
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return None
+    import oracle as O
+
+    O.lib()
+    rows = args.ref_rows
+    xs, xts = sample_host(args, rows)
+    for _ in range(args.warmup):
+        oracle_sample_step(args, rows, xs, xts)
+    t = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(args, rows, xs, xts)
+    dt = (time.perf_counter() - t) / args.steps
+    sample_args = argparse.Namespace(**{**vars(args), "rows": rows})
+    b, _ = step_bytes(sample_args)
+    v = round(b / dt / 1e9, 4)
+    sample = (f"first {rows} of {args.rows} rows of each of the {args.layers} layers (capture) and of the "
+              f"{args.deep} perturbed deep layers (guided) per step")
+    return dict(impl="reference", metric=METRIC, value=v, unit="GB/s", n_gpus=world, steps=args.steps,
+                warmup=args.warmup, ms_per_step=round(dt * 1e3, 2), higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="f64", data="synthetic",
+                config=dict(workload=f"layer_stack: {args.layers} layers x {args.rows}x{args.cols} bf16, "
+                                     f"NVFP4 capture + guided (row sample)", layers=args.layers,
+                            rows=args.rows, cols=args.cols, format="NVFP4"),
+                cpu_baseline=dict(value=v, unit="GB/s", cores=1, kind="oracle", sample=sample),
+                e2e=dict(value=v, unit="GB/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        out = run_reference(args, world, rank)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return
+    world, rank, local = dist_setup(args)
+    try:
+        out = run_ours(args, world, rank, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

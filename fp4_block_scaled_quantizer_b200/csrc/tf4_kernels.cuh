@@ -1,0 +1,659 @@
+// tf4_kernels.cuh -- sm_100a kernels of the trace_fp4 library.
+//
+// Streaming, elementwise + reduction work: no tensor cores.  Every kernel
+// splits its flat array of quantization blocks into one contiguous range
+// per CTA (grid = SMs x resident CTAs, one wave), and lanes of a warp take
+// consecutive blocks so that each warp instruction moves a contiguous span.
+// NVFP4: one lane owns one 16-element block (32 B of bf16, two 16-B loads);
+// MXFP4: one lane owns one 32-element block (four 16-B loads).
+//
+// Definitions followed are stated in include/trace_fp4.h (and the pages
+// cited there); the notes below only explain how each kernel reaches the
+// exact definition.
+#pragma once
+
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/trace_fp4.h"
+
+namespace tf4 {
+
+constexpr int kThreads = 256;
+
+// ------------------------------------------------------------- segments
+// One per-tensor-scale segment covering everything (the common case).
+struct Seg1 {
+  __device__ __forceinline__ int find(int64_t /*block*/) const { return 0; }
+  __device__ __forceinline__ int64_t start(int /*s*/) const { return 0; }
+  __device__ __forceinline__ int count() const { return 1; }
+};
+
+// Ragged segments (row offsets, passed by value in the kernel parameters).
+struct SegN {
+  int32_t nseg;
+  int64_t bpr;  // quantization blocks per row
+  int32_t off[TF4_MAX_SEGMENTS + 1];
+  // The segment holding `block`: the largest s with off[s] <= row (it is
+  // then non-empty).
+  __device__ __forceinline__ int find(int64_t block) const {
+    const int64_t row = block / bpr;
+    int lo = 0, hi = nseg;  // answer in [lo, hi)
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (off[mid] <= row) lo = mid; else hi = mid;
+    }
+    return lo;
+  }
+  __device__ __forceinline__ int64_t start(int s) const { return (int64_t)off[s] * bpr; }
+  __device__ __forceinline__ int count() const { return nseg; }
+};
+
+__device__ __forceinline__ int64_t cta_begin(int64_t i, int64_t grid, int64_t n) {
+  const int64_t q = n / grid, r = n % grid;
+  return i * q + (i < r ? i : r);
+}
+
+// ---------------------------------------------------------- small helpers
+__device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// bf16 pair -> two fp32 (exact widening)
+__device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Max |x| over words of bf16 pairs, as a bf16 bit pattern (0x7F80 or more
+// means a non-finite input: the magnitude bit order is the value order).
+template <int N>
+__device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&w)[N]) {
+  uint32_t m = w[0] & 0x7FFF7FFFu;
+#pragma unroll
+  for (int i = 1; i < N; ++i) m = vmax_u16x2(m, w[i] & 0x7FFF7FFFu);
+  return max(m & 0xFFFFu, m >> 16);
+}
+
+// Eight fp32 values -> eight E2M1 nibbles (hardware RNE, satfinite),
+// element k in bits [4k, 4k+4).
+__device__ __forceinline__ uint32_t cvt_e2m1x8(float v0, float v1, float v2, float v3, float v4,
+                                               float v5, float v6, float v7) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(r)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+  return r;
+}
+
+// Four packed e2m1 pairs (4 bytes) -> eight halves (hardware conversion).
+__device__ __forceinline__ void e2m1x8_to_half(uint32_t c, uint32_t (&h)[4]) {
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
+      "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(c));
+}
+
+// m3 & 1 of eight nibbles -> eight bits (nibble k -> bit k).
+__device__ __forceinline__ uint32_t nibble_lsbs(uint32_t c) {
+  uint32_t t = c & 0x11111111u;
+  t = (t | (t >> 3)) & 0x03030303u;
+  t = (t | (t >> 6)) & 0x000F000Fu;
+  t = (t | (t >> 12)) & 0xFFu;
+  return t;
+}
+
+// E4M3 (fn) scale byte of a non-negative fp32 (hardware RNE, satfinite).
+__device__ __forceinline__ uint32_t e4m3_encode(float r) {
+  return (uint32_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
+}
+
+// Value of an E4M3 byte in [0, 0x7E].
+__device__ __forceinline__ float e4m3_decode(uint32_t b) {
+  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
+  if (e == 0) return (float)m * 0x1p-9f;
+  return __uint_as_float(((e + 120u) << 23) | (m << 20));
+}
+
+// NVFP4 per-tensor scale from the segment amax; non-finite amax -> NaN.
+__device__ __forceinline__ float tensor_scale(float amax, int32_t* status) {
+  if (!(amax <= 3.4028234663852886e38f)) {  // Inf or NaN
+    if (status) atomicOr(status, TF4_DEV_NONFINITE);
+    return __int_as_float(0x7FC00000);
+  }
+  const float s = __fdiv_rn(amax, 2688.0f);
+  return s >= 0x1p-126f ? s : 0.0f;
+}
+
+// A value within 8 fp32 ulps of a bf16 number (low 16 bits near 0 or 2^16).
+__device__ __forceinline__ bool near_bf16(float v) {
+  return ((__float_as_uint(v) + 8u) & 0xFFFFu) < 16u;
+}
+
+// ------------------------------------------------- exact per-element paths
+// RTN m3 of |x| on scale S > 0 by exact comparisons.  fmaf(-mu, S, ax) is
+// rounded once, so its sign is the sign of ax - mu*S exactly as long as the
+// difference cannot underflow, which holds for S >= 2^-124; smaller S is
+// rescaled by 2^64 first (exact).  Three-level search over the midpoints
+// {.25,.75,1.25,1.75,2.5,3.5,5}; ">=" at odd-index midpoints and ">" at
+// even-index ones give ties to the even m3.
+__device__ __forceinline__ uint32_t rtn_m3_exact(float ax, float S) {
+  if (S < 0x1p-100f) {
+    ax *= 0x1p64f;
+    S *= 0x1p64f;
+  }
+  const bool b2 = fmaf(-1.75f, S, ax) >= 0.0f;
+  const float mu = b2 ? 3.5f : 0.75f;
+  const bool b1 = fmaf(-mu, S, ax) >= 0.0f;
+  const float mu3 = b2 ? (b1 ? 5.0f : 2.5f) : (b1 ? 1.25f : 0.25f);
+  const bool b0 = fmaf(-mu3, S, ax) > 0.0f;
+  return (b2 ? 4u : 0u) | (b1 ? 2u : 0u) | (b0 ? 1u : 0u);
+}
+
+// Guided m3 of |x| on scale S > 0 with recorded bit g (exact comparisons as
+// above): f = number of codewords <= y; y >= 6 -> 7; y a codeword -> f;
+// otherwise the neighbour (f or f+1) whose m3 & 1 == g.
+__device__ __forceinline__ uint32_t guided_m3_exact(float ax, float S, uint32_t g) {
+  if (S < 0x1p-100f) {
+    ax *= 0x1p64f;
+    S *= 0x1p64f;
+  }
+  const float d2 = fmaf(-2.0f, S, ax);
+  const bool p2 = d2 >= 0.0f;
+  const float v1 = p2 ? 4.0f : 1.0f;
+  const float d1 = fmaf(-v1, S, ax);
+  const bool p1 = d1 >= 0.0f;
+  const float v0 = p2 ? (p1 ? 6.0f : 3.0f) : (p1 ? 1.5f : 0.5f);
+  const float d0 = fmaf(-v0, S, ax);
+  const bool p0 = d0 >= 0.0f;
+  const uint32_t f = (p2 ? 4u : 0u) | (p1 ? 2u : 0u) | (p0 ? 1u : 0u);
+  const bool exact = p0 ? (d0 == 0.0f) : p1 ? (d1 == 0.0f) : p2 ? (d2 == 0.0f) : (ax == 0.0f);
+  if (f == 7u || exact) return f;
+  return f + ((f ^ g) & 1u);
+}
+
+// Philox4x32-10 (Salmon et al., SC'11), word 0 only, counter (idx, 0, 0),
+// key = seed.
+__device__ __forceinline__ uint32_t philox_w0(uint64_t idx, uint64_t seed) {
+  uint32_t c0 = (uint32_t)idx, c1 = (uint32_t)(idx >> 32), c2 = 0u, c3 = 0u;
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
+    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
+    c0 = hi1 ^ c1 ^ k0;
+    c1 = lo1;
+    c2 = hi0 ^ c3 ^ k1;
+    c3 = lo0;
+  }
+  return c0;
+}
+
+// Magnitude of E2M1 code m3 (0..7) as fp32.
+__device__ __forceinline__ float e2m1_value(uint32_t m3) {
+  const uint32_t e = m3 >> 1, m = m3 & 1u;
+  return e ? __uint_as_float(((e + 126u) << 23) | (m << 22)) : (m ? 0.5f : 0.0f);
+}
+
+// SR m3 of |x| on scale S > 0 with a 24-bit uniform r.  Every product of a
+// codeword (<= 4 significant bits) and S (24 bits) is exact in double, and
+// so are r * gap * S (<= 48 bits) and ax - V_lo * S (within a factor two of
+// each other, or V_lo = 0), so all comparisons are exact.
+__device__ __forceinline__ uint32_t sr_m3_exact(float axf, float Sf, uint32_t r24) {
+  const double ax = axf, S = Sf;
+  if (ax >= 6.0 * S) return 7u;
+  // f = number of nonzero codewords <= y
+  const uint32_t f = (0.5 * S <= ax) + (1.0 * S <= ax) + (1.5 * S <= ax) + (2.0 * S <= ax) +
+                     (3.0 * S <= ax) + (4.0 * S <= ax) + (6.0 * S <= ax);
+  const double vlo = (double)e2m1_value(f), vhi = (double)e2m1_value(f + 1u);
+  if (vlo * S == ax) return f;
+  const double lhs = (double)r24 * (vhi - vlo) * S;
+  const double rhs = 16777216.0 * (ax - vlo * S);
+  return lhs < rhs ? f + 1u : f;
+}
+
+// -------------------------------------------------------------- amax pass
+// Grid-wide max |x| per segment.  Each CTA reduces its range piece by
+// piece (a piece = the part of the range inside one segment) and
+// atomicMax-es the float bit pattern (order-preserving for values >= 0,
+// hence exact and deterministic) into ws[seg].  The last CTA to finish
+// (ticket counter at ws[nseg]) turns the maxima into the outputs, then
+// resets ws to zero for the next call.
+template <class SEG>
+__global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, int64_t nblocks,
+                                                   SEG seg, uint32_t* ws, float* s_t_out,
+                                                   float* amax_out, int32_t* status) {
+  __shared__ uint32_t red[kThreads / 32];
+  __shared__ int last;
+  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, nblocks);
+  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, nblocks);
+  const int tid = threadIdx.x;
+  int64_t lo = b0;
+  while (lo < b1) {
+    const int s = seg.find(lo);
+    const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
+    // chunks [2lo, 2hi), 8 in flight per thread
+    const int64_t c0 = 2 * lo, c1 = 2 * hi;
+    uint32_t m = 0;
+    int64_t c = c0 + tid;
+    for (; c + 7 * kThreads < c1; c += 8 * kThreads) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(x + c + u * kThreads);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        m = vmax_u16x2(m, v[u].x & 0x7FFF7FFFu);
+        m = vmax_u16x2(m, v[u].y & 0x7FFF7FFFu);
+        m = vmax_u16x2(m, v[u].z & 0x7FFF7FFFu);
+        m = vmax_u16x2(m, v[u].w & 0x7FFF7FFFu);
+      }
+    }
+    for (; c < c1; c += kThreads) {
+      const uint4 v = __ldg(x + c);
+      m = vmax_u16x2(m, v.x & 0x7FFF7FFFu);
+      m = vmax_u16x2(m, v.y & 0x7FFF7FFFu);
+      m = vmax_u16x2(m, v.z & 0x7FFF7FFFu);
+      m = vmax_u16x2(m, v.w & 0x7FFF7FFFu);
+    }
+    uint32_t mb = max(m & 0xFFFFu, m >> 16);
+    mb = __reduce_max_sync(0xFFFFFFFFu, mb);
+    if ((tid & 31) == 0) red[tid >> 5] = mb;
+    __syncthreads();
+    if (tid == 0) {
+      uint32_t t = red[0];
+#pragma unroll
+      for (int w = 1; w < kThreads / 32; ++w) t = max(t, red[w]);
+      atomicMax(ws + s, t << 16);
+    }
+    __syncthreads();
+    lo = hi;
+  }
+  // completion ticket
+  if (tid == 0) {
+    __threadfence();
+    const uint32_t t = atomicAdd(ws + seg.count(), 1u);
+    last = (t == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  for (int k = tid; k < seg.count(); k += kThreads) {
+    const uint32_t bits = atomicExch(ws + k, 0u);
+    const float amax = __uint_as_float(bits);
+    if (amax_out) {
+      amax_out[k] = amax;
+      if (!(amax <= 3.4028234663852886e38f) && status) atomicOr(status, TF4_DEV_NONFINITE);
+    }
+    if (s_t_out) s_t_out[k] = tensor_scale(amax, status);
+  }
+  if (tid == 0) ws[seg.count()] = 0u;
+}
+
+// --------------------------------------------------------- quantize pass
+enum { kRTN = 0, kSR = 1, kCAPTURE = 2 };
+
+struct QuantArgs {
+  const uint4* x;
+  int64_t nblocks;
+  const float* st_src;  // s_t per segment, or amax per segment (st_from_amax)
+  int st_from_amax;
+  float* s_t_out;       // written by CTA 0 when st_from_amax
+  uint8_t* codes;
+  uint8_t* scales;
+  uint8_t* bits;        // capture only; may be NULL
+  uint64_t seed;
+  int32_t* status;
+};
+
+// One NVFP4 block (16 bf16 in w[0..7]) -> code words, scale byte, flags.
+template <int MODE>
+__device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, int64_t blk,
+                                            uint64_t seed, uint32_t& c0, uint32_t& c1,
+                                            uint32_t& sc, bool& bad) {
+  const uint32_t mb = block_absmax_bits(w);
+  bad = mb >= 0x7F80u;
+  float S = 0.0f;
+  sc = 0;
+  if (st > 0.0f) {  // st == 0: zero segment; NaN: non-finite segment
+    const float bamax = __uint_as_float(mb << 16);
+    const float q = __fdiv_rn(bamax, 6.0f);
+    const float r = __fdiv_rn(q, st);
+    sc = e4m3_encode(r);
+    S = __fmul_rn(st, e4m3_decode(sc));
+  }
+  if (MODE != kSR && S > 0.0f &&
+      !(S < 0x1p-100f || near_bf16(S) || near_bf16(__fmul_rn(3.0f, S)) ||
+        near_bf16(__fmul_rn(5.0f, S)) || near_bf16(__fmul_rn(7.0f, S)))) {
+    // Fast path: no bf16 value lies within 2^-21 (relative) of any
+    // midpoint * S, so the rounded quotient x * RN(1/S) (relative error
+    // < 2^-22.9) falls on the same side of every midpoint as the exact one
+    // and never on a midpoint: hardware RNE of it is the exact answer.
+    const float rS = __frcp_rn(S);
+    c0 = cvt_e2m1x8(bf_lo(w[0]) * rS, bf_hi(w[0]) * rS, bf_lo(w[1]) * rS, bf_hi(w[1]) * rS,
+                    bf_lo(w[2]) * rS, bf_hi(w[2]) * rS, bf_lo(w[3]) * rS, bf_hi(w[3]) * rS);
+    c1 = cvt_e2m1x8(bf_lo(w[4]) * rS, bf_hi(w[4]) * rS, bf_lo(w[5]) * rS, bf_hi(w[5]) * rS,
+                    bf_lo(w[6]) * rS, bf_hi(w[6]) * rS, bf_lo(w[7]) * rS, bf_hi(w[7]) * rS);
+    return;
+  }
+  // Exact path (near-tie scales, tiny or zero scales, stochastic rounding).
+  uint32_t out[2] = {0u, 0u};
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
+    const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+    uint32_t m3 = 0;
+    if (S > 0.0f) {
+      if (MODE == kSR)
+        m3 = sr_m3_exact(ax, S, philox_w0((uint64_t)blk * 16u + k, seed) >> 8);
+      else
+        m3 = rtn_m3_exact(ax, S);
+    }
+    out[k >> 3] |= (((h >> 15) << 3) | m3) << (4 * (k & 7));
+  }
+  c0 = out[0];
+  c1 = out[1];
+}
+
+// One MXFP4 block (32 bf16 in w[0..15]) -> code words, scale byte, flags.
+template <int MODE>
+__device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk, uint64_t seed,
+                                            uint32_t (&c)[4], uint32_t& sc, bool& bad) {
+  const uint32_t mb = block_absmax_bits(w);
+  bad = mb >= 0x7F80u;
+  const uint32_t E = (mb >> 7) & 0xFFu;  // bf16 exponent field of bamax
+  // e = floor(log2 bamax) - 2 clamped at -127; bamax subnormal or 0 -> -127
+  const int e = (E == 0) ? -127 : max((int)E - 129, -127);
+  sc = (uint32_t)(e + 127);
+  if (MODE != kSR) {
+    // y = x * 2^-e is exact (2^-e is a normal fp32 for e in [-127, 125]),
+    // so hardware RNE of y is the exact answer.
+    const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      c[q] = cvt_e2m1x8(bf_lo(w[4 * q]) * inv, bf_hi(w[4 * q]) * inv, bf_lo(w[4 * q + 1]) * inv,
+                        bf_hi(w[4 * q + 1]) * inv, bf_lo(w[4 * q + 2]) * inv,
+                        bf_hi(w[4 * q + 2]) * inv, bf_lo(w[4 * q + 3]) * inv,
+                        bf_hi(w[4 * q + 3]) * inv);
+    return;
+  }
+  const float S = __uint_as_float(e >= -126 ? (uint32_t)(e + 127) << 23 : 0x00400000u);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) c[q] = 0u;
+#pragma unroll
+  for (int k = 0; k < 32; ++k) {
+    const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
+    const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+    const uint32_t m3 = sr_m3_exact(ax, S, philox_w0((uint64_t)blk * 32u + k, seed) >> 8);
+    c[k >> 3] |= (((h >> 15) << 3) | m3) << (4 * (k & 7));
+  }
+}
+
+__device__ __forceinline__ void report_bad(bool bad, int32_t* status) {
+  if (__any_sync(0xFFFFFFFFu, bad) && (threadIdx.x & 31) == 0 && status)
+    atomicOr(status, TF4_DEV_NONFINITE);
+}
+
+// Quantize pass.  Each CTA walks its block range backwards, so that the
+// first blocks it reads are the ones the amax pass read last (still in L2).
+template <int FMT, int MODE, class SEG>
+__global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
+  constexpr int U = 2;  // blocks per lane per iteration
+  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
+  const int tid = threadIdx.x;
+  if (FMT == TF4_NVFP4 && a.st_from_amax && blockIdx.x == 0 && a.s_t_out)
+    for (int k = tid; k < seg.count(); k += kThreads) a.s_t_out[k] = tensor_scale(a.st_src[k], a.status);
+  int64_t hi = b1;
+  while (hi > b0) {
+    const int s = seg.find(hi - 1);
+    const int64_t lo = max(b0, seg.start(s));
+    float st = 0.0f;
+    if constexpr (FMT == TF4_NVFP4) st = a.st_from_amax ? tensor_scale(a.st_src[s], nullptr) : a.st_src[s];
+    const int64_t n = hi - lo;
+    for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
+      if constexpr (FMT == TF4_NVFP4) {
+        uint32_t w[U][8];
+        int64_t blk[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int64_t k = j + u * kThreads + tid;
+          blk[u] = hi - 1 - k;
+          if (k < n) {
+            const uint4 p = __ldg(a.x + 2 * blk[u]), q = __ldg(a.x + 2 * blk[u] + 1);
+            w[u][0] = p.x; w[u][1] = p.y; w[u][2] = p.z; w[u][3] = p.w;
+            w[u][4] = q.x; w[u][5] = q.y; w[u][6] = q.z; w[u][7] = q.w;
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const bool valid = j + u * kThreads + tid < n;
+          bool bad = false;
+          if (valid) {
+            uint32_t c0, c1, sc;
+            nvfp4_block<MODE>(w[u], st, blk[u], a.seed, c0, c1, sc, bad);
+            reinterpret_cast<uint2*>(a.codes)[blk[u]] = make_uint2(c0, c1);
+            a.scales[blk[u]] = (uint8_t)sc;
+            if (MODE == kCAPTURE && a.bits)
+              reinterpret_cast<uint16_t*>(a.bits)[blk[u]] =
+                  (uint16_t)(nibble_lsbs(c0) | (nibble_lsbs(c1) << 8));
+          }
+          report_bad(bad, a.status);
+        }
+      } else {
+        uint32_t w[U][16];
+        int64_t blk[U];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const int64_t k = j + u * kThreads + tid;
+          blk[u] = hi - 1 - k;
+          if (k < n) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint4 p = __ldg(a.x + 4 * blk[u] + q);
+              w[u][4 * q] = p.x; w[u][4 * q + 1] = p.y; w[u][4 * q + 2] = p.z; w[u][4 * q + 3] = p.w;
+            }
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+          const bool valid = j + u * kThreads + tid < n;
+          bool bad = false;
+          if (valid) {
+            uint32_t c[4], sc;
+            mxfp4_block<MODE>(w[u], blk[u], a.seed, c, sc, bad);
+            reinterpret_cast<uint4*>(a.codes)[blk[u]] = make_uint4(c[0], c[1], c[2], c[3]);
+            a.scales[blk[u]] = (uint8_t)sc;
+            if (MODE == kCAPTURE && a.bits)
+              reinterpret_cast<uint32_t*>(a.bits)[blk[u]] =
+                  nibble_lsbs(c[0]) | (nibble_lsbs(c[1]) << 8) | (nibble_lsbs(c[2]) << 16) |
+                  (nibble_lsbs(c[3]) << 24);
+          }
+          report_bad(bad, a.status);
+        }
+      }
+    }
+    hi = lo;
+  }
+}
+
+// ----------------------------------------------------------- guided pass
+struct GuidedArgs {
+  const uint4* x;
+  int64_t nblocks;
+  const uint8_t* rec_scales;
+  const float* rec_s_t;
+  const uint8_t* rec_bits;
+  uint8_t* codes;
+  int32_t* status;
+};
+
+template <int FMT, class SEG>
+__global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
+  constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;  // elements per block
+  constexpr int NW = BE / 2;                       // bf16 pair words per block
+  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
+  const int tid = threadIdx.x;
+  int64_t lo = b0;
+  while (lo < b1) {
+    const int s = seg.find(lo);
+    const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
+    const float st = FMT == TF4_NVFP4 ? a.rec_s_t[s] : 0.0f;
+    const int64_t n = hi - lo;
+    for (int64_t j = 0; j < n; j += kThreads) {
+      const int64_t k = j + tid;
+      const bool valid = k < n;
+      bool bad = false;
+      if (valid) {
+        const int64_t blk = lo + k;
+        uint32_t w[NW];
+#pragma unroll
+        for (int q = 0; q < NW / 4; ++q) {
+          const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
+          w[4 * q] = p.x; w[4 * q + 1] = p.y; w[4 * q + 2] = p.z; w[4 * q + 3] = p.w;
+        }
+        const uint32_t sc = a.rec_scales[blk];
+        uint32_t g;
+        if constexpr (FMT == TF4_NVFP4) g = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
+        else g = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
+        float S;
+        if constexpr (FMT == TF4_NVFP4) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
+        else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
+        bad = block_absmax_bits(w) >= 0x7F80u;
+        uint32_t c[BE / 8];
+#pragma unroll
+        for (int q = 0; q < BE / 8; ++q) c[q] = 0u;
+#pragma unroll
+        for (int e = 0; e < BE; ++e) {
+          const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+          const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+          const uint32_t m3 = S > 0.0f ? guided_m3_exact(ax, S, (g >> e) & 1u) : 0u;
+          c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
+        }
+        if constexpr (FMT == TF4_NVFP4) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
+        else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);
+      }
+      report_bad(bad, a.status);
+    }
+    lo = hi;
+  }
+}
+
+// ---------------------------------------------------------- dequantize
+struct DequantArgs {
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* s_t;
+  float4* out;
+  int64_t nblocks;
+};
+
+template <int FMT, class SEG>
+__global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
+  constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;
+  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
+  const int tid = threadIdx.x;
+  int64_t lo = b0;
+  while (lo < b1) {
+    const int s = seg.find(lo);
+    const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
+    const float st = FMT == TF4_NVFP4 ? a.s_t[s] : 0.0f;
+    for (int64_t blk = lo + tid; blk < hi; blk += kThreads) {
+      const uint32_t sc = a.scales[blk];
+      float S;
+      if constexpr (FMT == TF4_NVFP4) S = __fmul_rn(st, e4m3_decode(sc));
+      else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
+      uint32_t cw[BE / 8];
+      if constexpr (FMT == TF4_NVFP4) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.codes) + blk);
+        cw[0] = v.x; cw[1] = v.y;
+      } else {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.codes) + blk);
+        cw[0] = v.x; cw[1] = v.y; cw[2] = v.z; cw[3] = v.w;
+      }
+#pragma unroll
+      for (int q = 0; q < BE / 8; ++q) {
+        uint32_t h[4];
+        e2m1x8_to_half(cw[q], h);
+        float f[8];
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&h[p]));
+          f[2 * p] = __fmul_rn(t.x, S);
+          f[2 * p + 1] = __fmul_rn(t.y, S);
+        }
+        float4* o = a.out + (blk * BE + q * 8) / 4;
+        o[0] = make_float4(f[0], f[1], f[2], f[3]);
+        o[1] = make_float4(f[4], f[5], f[6], f[7]);
+      }
+    }
+    lo = hi;
+  }
+}
+
+// ------------------------------------------------------- pack / unpack
+// Units of 32 elements: 16 code bytes -> 4 guidance bytes.  A trailing half
+// unit (16 elements, when rows*cols % 32 == 16) is done by the last thread.
+__global__ void __launch_bounds__(kThreads) k_pack(const uint8_t* __restrict__ codes, uint8_t* bits,
+                                                   int64_t nunits, int tail) {
+  const int64_t u0 = cta_begin(blockIdx.x, gridDim.x, nunits);
+  const int64_t u1 = cta_begin(blockIdx.x + 1, gridDim.x, nunits);
+  for (int64_t u = u0 + threadIdx.x; u < u1; u += kThreads) {
+    const uint4 c = __ldg(reinterpret_cast<const uint4*>(codes) + u);
+    reinterpret_cast<uint32_t*>(bits)[u] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) |
+                                           (nibble_lsbs(c.z) << 16) | (nibble_lsbs(c.w) << 24);
+  }
+  if (tail && blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
+    const uint2 c = *reinterpret_cast<const uint2*>(codes + 16 * nunits);
+    reinterpret_cast<uint16_t*>(bits)[2 * nunits] = (uint16_t)(nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8));
+  }
+}
+
+// bits of one byte -> 8 bytes of 0/1 (bit k -> byte k)
+__device__ __forceinline__ uint2 spread8(uint32_t b) {
+  uint32_t o[2];
+#pragma unroll
+  for (int q = 0; q < 2; ++q) {
+    const uint32_t nib = (b >> (4 * q)) & 0xFu;
+    o[q] = (nib & 1u) | ((nib & 2u) << 7) | ((nib & 4u) << 14) | ((nib & 8u) << 21);
+  }
+  return make_uint2(o[0], o[1]);
+}
+
+// Units of 32 elements: 4 guidance bytes -> 32 bytes of 0/1.
+__global__ void __launch_bounds__(kThreads) k_unpack(const uint8_t* __restrict__ bits, uint8_t* mant,
+                                                     int64_t nunits, int tail) {
+  const int64_t u0 = cta_begin(blockIdx.x, gridDim.x, nunits);
+  const int64_t u1 = cta_begin(blockIdx.x + 1, gridDim.x, nunits);
+  uint4* out = reinterpret_cast<uint4*>(mant);
+  for (int64_t u = u0 + threadIdx.x; u < u1; u += kThreads) {
+    const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(bits) + u);
+    const uint2 a0 = spread8(b & 0xFFu), a1 = spread8((b >> 8) & 0xFFu);
+    const uint2 a2 = spread8((b >> 16) & 0xFFu), a3 = spread8(b >> 24);
+    out[2 * u] = make_uint4(a0.x, a0.y, a1.x, a1.y);
+    out[2 * u + 1] = make_uint4(a2.x, a2.y, a3.x, a3.y);
+  }
+  if (tail && blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
+    const uint32_t b = reinterpret_cast<const uint16_t*>(bits)[2 * nunits];
+    const uint2 a0 = spread8(b & 0xFFu), a1 = spread8(b >> 8);
+    out[2 * nunits] = make_uint4(a0.x, a0.y, a1.x, a1.y);
+  }
+}
+
+}  // namespace tf4

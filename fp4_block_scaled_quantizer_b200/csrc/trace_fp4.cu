@@ -1,0 +1,395 @@
+// trace_fp4.cu -- C ABI of the trace_fp4 library (see include/trace_fp4.h):
+// argument validation, launch geometry, and the kernel launches.
+#include <cuda_runtime.h>
+
+#include <climits>
+#include <cstring>
+#include <mutex>
+
+#include "../../include/trace_fp4.h"
+#include "tf4_kernels.cuh"
+
+namespace {
+
+using tf4::kThreads;
+
+struct Shape {
+  int fmt;
+  int be;         // elements per quantization block
+  int64_t rows, cols, n, nblocks;
+  int nseg;
+  const int64_t* off;
+};
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+tf4_status check_desc(const tf4_desc* d, Shape* sh) {
+  if (!d) return TF4_ERR_INVALID_ARG;
+  if (d->fmt != TF4_NVFP4 && d->fmt != TF4_MXFP4) return TF4_ERR_INVALID_ARG;
+  const int be = d->fmt == TF4_NVFP4 ? 16 : 32;
+  if (d->rows < 0 || d->cols <= 0 || d->cols % be != 0) return TF4_ERR_SHAPE;
+  if (d->rows > 0 && d->cols > (int64_t)(LLONG_MAX / 64) / d->rows) return TF4_ERR_SHAPE;
+  const int nseg = d->num_segments;
+  if (nseg < 1 || nseg > TF4_MAX_SEGMENTS) return TF4_ERR_INVALID_ARG;
+  if (d->fmt == TF4_MXFP4 && nseg != 1) return TF4_ERR_INVALID_ARG;
+  if (nseg > 1 && !d->seg_row_offsets) return TF4_ERR_INVALID_ARG;
+  if (d->seg_row_offsets) {
+    const int64_t* o = d->seg_row_offsets;
+    if (o[0] != 0 || o[nseg] != d->rows) return TF4_ERR_INVALID_ARG;
+    for (int s = 0; s < nseg; ++s)
+      if (o[s + 1] < o[s]) return TF4_ERR_INVALID_ARG;
+    if (nseg > 1 && d->rows > INT_MAX) return TF4_ERR_SHAPE;
+  }
+  sh->fmt = d->fmt;
+  sh->be = be;
+  sh->rows = d->rows;
+  sh->cols = d->cols;
+  sh->n = d->rows * d->cols;
+  sh->nblocks = sh->n / be;
+  sh->nseg = nseg;
+  sh->off = d->seg_row_offsets;
+  return TF4_OK;
+}
+
+tf4::SegN make_segn(const Shape& sh) {
+  tf4::SegN s;
+  std::memset(&s, 0, sizeof s);
+  s.nseg = sh.nseg;
+  s.bpr = sh.cols / sh.be;
+  for (int k = 0; k <= sh.nseg; ++k) s.off[k] = (int32_t)sh.off[k];
+  return s;
+}
+
+bool multi(const Shape& sh) { return sh.nseg > 1; }
+
+int sm_count() {
+  static int cache[128] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+// Resident CTAs per SM of `kernel` on the current device (cached).
+int occupancy(const void* kernel) {
+  struct Entry { int dev; const void* k; int occ; };
+  static Entry cache[256];
+  static int used = 0;
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  for (int i = 0; i < used; ++i)
+    if (cache[i].dev == dev && cache[i].k == kernel) return cache[i].occ;
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, 0) != cudaSuccess || occ <= 0) {
+    cudaGetLastError();
+    occ = 1;
+  }
+  if (used < 256) cache[used++] = Entry{dev, kernel, occ};
+  return occ;
+}
+
+// One wave: SMs x resident CTAs of `kernel`, never more CTAs than units.
+template <class K>
+int64_t wave_grid(K kernel, int64_t units) {
+  const int64_t g = (int64_t)sm_count() * occupancy(reinterpret_cast<const void*>(kernel));
+  return units < g ? (units > 0 ? units : 1) : g;
+}
+
+tf4_status launched() {
+  return cudaGetLastError() == cudaSuccess ? TF4_OK : TF4_ERR_CUDA;
+}
+
+size_t ws_bytes_for(const Shape& sh) {
+  if (sh.fmt != TF4_NVFP4) return 0;
+  return ((size_t)(sh.nseg + 1) * sizeof(uint32_t) + 255) & ~(size_t)255;
+}
+
+// NVFP4 quantize grid: shared by the amax pass and the quantize pass so
+// that both cover the same byte range per CTA.
+template <int MODE>
+int64_t nvfp4_grid(const Shape& sh) {
+  return multi(sh) ? wave_grid(tf4::k_quant<TF4_NVFP4, MODE, tf4::SegN>, sh.nblocks)
+                   : wave_grid(tf4::k_quant<TF4_NVFP4, MODE, tf4::Seg1>, sh.nblocks);
+}
+
+tf4_status launch_amax(const Shape& sh, int64_t grid, const void* x, uint32_t* ws, float* s_t_out,
+                       float* amax_out, int32_t* status, cudaStream_t st) {
+  const uint4* x4 = static_cast<const uint4*>(x);
+  // the amax pass works on 16-element blocks whatever the format
+  const int64_t nb16 = sh.n / 16;
+  if (multi(sh)) {
+    tf4::SegN seg = make_segn(sh);
+    seg.bpr = sh.cols / 16;
+    tf4::k_amax<tf4::SegN><<<(unsigned)grid, kThreads, 0, st>>>(x4, nb16, seg, ws, s_t_out, amax_out, status);
+  } else {
+    tf4::k_amax<tf4::Seg1><<<(unsigned)grid, kThreads, 0, st>>>(x4, nb16, tf4::Seg1{}, ws, s_t_out, amax_out,
+                                                                 status);
+  }
+  return launched();
+}
+
+template <int MODE>
+tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const float* amax_in,
+                         uint8_t* codes, uint8_t* scales, float* s_t, uint8_t* bits, void* ws,
+                         size_t ws_bytes, int32_t* status, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(d, &sh);
+  if (e != TF4_OK) return e;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const bool nv = sh.fmt == TF4_NVFP4;
+  if (nv && !s_t) return TF4_ERR_INVALID_ARG;
+  if (nv && (!aligned(s_t, 4) || (amax_in && !aligned(amax_in, 4)))) return TF4_ERR_ALIGN;
+  if (status && !aligned(status, 4)) return TF4_ERR_ALIGN;
+  if (sh.n == 0) {
+    if (nv) return cudaMemsetAsync(s_t, 0, sizeof(float) * sh.nseg, st) == cudaSuccess ? TF4_OK : TF4_ERR_CUDA;
+    return TF4_OK;
+  }
+  if (!x || !codes || !scales) return TF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || (bits && !aligned(bits, 4))) return TF4_ERR_ALIGN;
+  if (nv && !amax_in) {
+    if (!ws) return TF4_ERR_WORKSPACE;
+    if (!aligned(ws, 4)) return TF4_ERR_ALIGN;
+    if (ws_bytes < ws_bytes_for(sh)) return TF4_ERR_WORKSPACE;
+  }
+  tf4::QuantArgs a;
+  a.x = static_cast<const uint4*>(x);
+  a.nblocks = sh.nblocks;
+  a.codes = codes;
+  a.scales = scales;
+  a.bits = bits;
+  a.seed = seed;
+  a.status = status;
+  a.s_t_out = s_t;
+  if (nv) {
+    const int64_t grid = nvfp4_grid<MODE>(sh);
+    if (amax_in) {
+      a.st_src = amax_in;
+      a.st_from_amax = 1;
+    } else {
+      e = launch_amax(sh, grid, x, static_cast<uint32_t*>(ws), s_t, nullptr, status, st);
+      if (e != TF4_OK) return e;
+      a.st_src = s_t;
+      a.st_from_amax = 0;
+    }
+    if (multi(sh))
+      tf4::k_quant<TF4_NVFP4, MODE, tf4::SegN><<<(unsigned)grid, kThreads, 0, st>>>(a, make_segn(sh));
+    else
+      tf4::k_quant<TF4_NVFP4, MODE, tf4::Seg1><<<(unsigned)grid, kThreads, 0, st>>>(a, tf4::Seg1{});
+  } else {
+    a.st_src = nullptr;
+    a.st_from_amax = 0;
+    a.s_t_out = nullptr;
+    const int64_t grid = wave_grid(tf4::k_quant<TF4_MXFP4, MODE, tf4::Seg1>, sh.nblocks);
+    tf4::k_quant<TF4_MXFP4, MODE, tf4::Seg1><<<(unsigned)grid, kThreads, 0, st>>>(a, tf4::Seg1{});
+  }
+  return launched();
+}
+
+}  // namespace
+
+extern "C" {
+
+size_t tf4_workspace_bytes(const tf4_desc* desc) {
+  Shape sh;
+  if (check_desc(desc, &sh) != TF4_OK) return 0;
+  return ws_bytes_for(sh);
+}
+
+size_t tf4_codes_bytes(const tf4_desc* desc) {
+  Shape sh;
+  return check_desc(desc, &sh) == TF4_OK ? (size_t)(sh.n / 2) : 0;
+}
+
+size_t tf4_scales_bytes(const tf4_desc* desc) {
+  Shape sh;
+  return check_desc(desc, &sh) == TF4_OK ? (size_t)sh.nblocks : 0;
+}
+
+size_t tf4_guidance_bytes(const tf4_desc* desc) {
+  Shape sh;
+  return check_desc(desc, &sh) == TF4_OK ? (size_t)(sh.n / 8) : 0;
+}
+
+size_t tf4_record_bytes(const tf4_desc* desc, int with_codes) {
+  Shape sh;
+  if (check_desc(desc, &sh) != TF4_OK) return 0;
+  size_t b = with_codes ? (size_t)(sh.n / 2) : (size_t)(sh.n / 8);
+  b += (size_t)sh.nblocks;
+  if (sh.fmt == TF4_NVFP4) b += sizeof(float) * (size_t)sh.nseg;
+  return b;
+}
+
+tf4_status tf4_segment_amax(const tf4_desc* desc, const void* x, float* amax, void* ws, size_t ws_bytes,
+                            int32_t* status, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.fmt != TF4_NVFP4) return TF4_ERR_INVALID_ARG;
+  if (!amax) return TF4_ERR_INVALID_ARG;
+  if (!aligned(amax, 4) || (status && !aligned(status, 4))) return TF4_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (sh.n == 0)
+    return cudaMemsetAsync(amax, 0, sizeof(float) * sh.nseg, st) == cudaSuccess ? TF4_OK : TF4_ERR_CUDA;
+  if (!x) return TF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16)) return TF4_ERR_ALIGN;
+  if (!ws) return TF4_ERR_WORKSPACE;
+  if (!aligned(ws, 4)) return TF4_ERR_ALIGN;
+  if (ws_bytes < ws_bytes_for(sh)) return TF4_ERR_WORKSPACE;
+  return launch_amax(sh, nvfp4_grid<tf4::kRTN>(sh), x, static_cast<uint32_t*>(ws), nullptr, amax, status, st);
+}
+
+tf4_status tf4_quantize_rtn(const tf4_desc* desc, const void* x, const float* amax_in, uint8_t* codes,
+                            uint8_t* scales, float* s_t, void* ws, size_t ws_bytes, int32_t* status,
+                            tf4_stream_t stream) {
+  return quantize_impl<tf4::kRTN>(desc, x, 0, amax_in, codes, scales, s_t, nullptr, ws, ws_bytes, status,
+                                  stream);
+}
+
+tf4_status tf4_quantize_sr(const tf4_desc* desc, const void* x, uint64_t seed, const float* amax_in,
+                           uint8_t* codes, uint8_t* scales, float* s_t, void* ws, size_t ws_bytes,
+                           int32_t* status, tf4_stream_t stream) {
+  return quantize_impl<tf4::kSR>(desc, x, seed, amax_in, codes, scales, s_t, nullptr, ws, ws_bytes, status,
+                                 stream);
+}
+
+tf4_status tf4_quantize_capture(const tf4_desc* desc, const void* x, const float* amax_in, uint8_t* codes,
+                                uint8_t* scales, float* s_t, uint8_t* bits, void* ws, size_t ws_bytes,
+                                int32_t* status, tf4_stream_t stream) {
+  if (!bits)
+    return quantize_impl<tf4::kRTN>(desc, x, 0, amax_in, codes, scales, s_t, nullptr, ws, ws_bytes, status,
+                                    stream);
+  return quantize_impl<tf4::kCAPTURE>(desc, x, 0, amax_in, codes, scales, s_t, bits, ws, ws_bytes, status,
+                                      stream);
+}
+
+tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_t* rec_scales,
+                               const float* rec_s_t, const uint8_t* rec_bits, uint8_t* codes, int32_t* status,
+                               tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.n == 0) return TF4_OK;
+  const bool nv = sh.fmt == TF4_NVFP4;
+  if (!x || !rec_scales || !rec_bits || !codes || (nv && !rec_s_t)) return TF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(rec_bits, 4) || (nv && !aligned(rec_s_t, 4)) ||
+      (status && !aligned(status, 4)))
+    return TF4_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tf4::GuidedArgs a;
+  a.x = static_cast<const uint4*>(x);
+  a.nblocks = sh.nblocks;
+  a.rec_scales = rec_scales;
+  a.rec_s_t = rec_s_t;
+  a.rec_bits = rec_bits;
+  a.codes = codes;
+  a.status = status;
+  if (nv) {
+    if (multi(sh)) {
+      const int64_t g = wave_grid(tf4::k_guided<TF4_NVFP4, tf4::SegN>, sh.nblocks);
+      tf4::k_guided<TF4_NVFP4, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+    } else {
+      const int64_t g = wave_grid(tf4::k_guided<TF4_NVFP4, tf4::Seg1>, sh.nblocks);
+      tf4::k_guided<TF4_NVFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+    }
+  } else {
+    const int64_t g = wave_grid(tf4::k_guided<TF4_MXFP4, tf4::Seg1>, sh.nblocks);
+    tf4::k_guided<TF4_MXFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  }
+  return launched();
+}
+
+tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint8_t* scales, const float* s_t,
+                          float* out, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.n == 0) return TF4_OK;
+  const bool nv = sh.fmt == TF4_NVFP4;
+  if (!codes || !scales || !out || (nv && !s_t)) return TF4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(out, 16) || (nv && !aligned(s_t, 4))) return TF4_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tf4::DequantArgs a;
+  a.codes = codes;
+  a.scales = scales;
+  a.s_t = s_t;
+  a.out = reinterpret_cast<float4*>(out);
+  a.nblocks = sh.nblocks;
+  if (nv) {
+    if (multi(sh)) {
+      const int64_t g = wave_grid(tf4::k_dequant<TF4_NVFP4, tf4::SegN>, sh.nblocks);
+      tf4::k_dequant<TF4_NVFP4, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+    } else {
+      const int64_t g = wave_grid(tf4::k_dequant<TF4_NVFP4, tf4::Seg1>, sh.nblocks);
+      tf4::k_dequant<TF4_NVFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+    }
+  } else {
+    const int64_t g = wave_grid(tf4::k_dequant<TF4_MXFP4, tf4::Seg1>, sh.nblocks);
+    tf4::k_dequant<TF4_MXFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  }
+  return launched();
+}
+
+tf4_status tf4_pack_guidance(const tf4_desc* desc, const uint8_t* codes, uint8_t* bits, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.n == 0) return TF4_OK;
+  if (!codes || !bits) return TF4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(bits, 4)) return TF4_ERR_ALIGN;
+  const int64_t units = sh.n / 32;
+  const int tail = (sh.n % 32) != 0;
+  const int64_t g = wave_grid(tf4::k_pack, units > 0 ? units : 1);
+  tf4::k_pack<<<(unsigned)g, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(codes, bits, units, tail);
+  return launched();
+}
+
+tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_t* mant, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.n == 0) return TF4_OK;
+  if (!bits || !mant) return TF4_ERR_INVALID_ARG;
+  if (!aligned(bits, 4) || !aligned(mant, 16)) return TF4_ERR_ALIGN;
+  const int64_t units = sh.n / 32;
+  const int tail = (sh.n % 32) != 0;
+  const int64_t g = wave_grid(tf4::k_unpack, units > 0 ? units : 1);
+  tf4::k_unpack<<<(unsigned)g, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(bits, mant, units, tail);
+  return launched();
+}
+
+tf4_status tf4_read_status(int32_t* dev_status, tf4_stream_t stream) {
+  if (!dev_status) return TF4_ERR_INVALID_ARG;
+  if (!aligned(dev_status, 4)) return TF4_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, dev_status, sizeof h, cudaMemcpyDeviceToHost, st) != cudaSuccess) return TF4_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TF4_ERR_CUDA;
+  if (cudaMemsetAsync(dev_status, 0, sizeof h, st) != cudaSuccess) return TF4_ERR_CUDA;
+  if (h & TF4_DEV_NONFINITE) return TF4_ERR_NONFINITE;
+  if (h & TF4_DEV_TIMEOUT) return TF4_ERR_TIMEOUT;
+  return TF4_OK;
+}
+
+const char* tf4_status_string(tf4_status s) {
+  switch (s) {
+    case TF4_OK: return "ok";
+    case TF4_ERR_INVALID_ARG: return "invalid argument";
+    case TF4_ERR_SHAPE: return "invalid shape (rows/cols, or cols not a multiple of the block size)";
+    case TF4_ERR_ALIGN: return "misaligned pointer";
+    case TF4_ERR_WORKSPACE: return "workspace missing or too small";
+    case TF4_ERR_NONFINITE: return "non-finite input";
+    case TF4_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case TF4_ERR_CUDA: return "CUDA error";
+  }
+  return "unknown status";
+}
+
+int tf4_version(void) { return 1; }
+
+}  // extern "C"

@@ -1,0 +1,186 @@
+/*
+ * trace_fp4.h -- C ABI of the block-scaled FP4 quantization library for
+ * rollout-guided FP4 quantization-aware training, NVIDIA B200 (sm_100a).
+ *
+ * Method (web pages, cited by title and section):
+ *   - "TRACE: Rollout-Guided Quantization-Aware Training for FP4
+ *     Reinforcement Learning of MoE Language Models", summary at
+ *     ai-papers.net: sections "学習とロールアウトの不一致" (nearest rounding
+ *     sends nearby values to different codewords), "TRACEの仕組み" (the
+ *     train side rounds each value to whichever of its two adjacent
+ *     codewords the rollout chose; straight-through backward) and
+ *     "量子化情報キャッシュ" (keep only the mantissa bit and the scale, only
+ *     for the deeper layers -- about 1/6 of the full information).
+ *   - Korean explainer of the same paper (sns.style), "작동 원리": the
+ *     rollout engine must export its quantization results and the trainer
+ *     must consume them.
+ *   - aibr.jp/archives/130278, section 3: NVFP4 = blocks of 16 E2M1 values
+ *     sharing one E4M3 scale; round-to-nearest forward, stochastic rounding
+ *     for backward / weight updates.
+ *   - aibr.jp/archives/132665 (TetraJet), section 3: MXFP4 per-group scale.
+ *
+ * Formats.  E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} indexed by
+ * m3 = exponent<<1 | mantissa; a code nibble is sign<<3 | m3.
+ *   NVFP4: 16-element blocks along the last dimension; per-segment fp32
+ *          tensor scale s_t = amax / (6*448) (below the smallest normal fp32
+ *          it is 0 and the segment quantizes to signed zeros); block scale
+ *          byte b = E4M3_rne_satfinite( fl32(fl32(bamax/6) / s_t) ); the
+ *          block's scale is S = fl32(s_t * E4M3(b)).
+ *   MXFP4: 32-element blocks; scale byte = e + 127 with
+ *          e = clamp(floor(log2 bamax) - 2, -127, 127) (-127 for an
+ *          all-zero block); S = 2^e.  No tensor scale.
+ *   Rounding of y = |x| / S (the exact real quotient):
+ *     RTN     nearest codeword, ties to even m3, saturating at 6;
+ *     SR      between the two neighbours lo < y < hi, round up iff
+ *             r < 2^24 (y-lo)/(hi-lo), r = (word 0 of Philox4x32-10 at
+ *             counter (i mod 2^32, i >> 32, 0, 0), key (seed mod 2^32,
+ *             seed >> 32)) >> 8, i = flat row-major element index within
+ *             the call; y >= 6 gives 6, a codeword keeps itself
+ *             (Salmon et al., "Parallel random numbers: as easy as 1, 2, 3",
+ *             SC'11, defines Philox4x32-10);
+ *     guided  of the two neighbours of y, the one whose m3 & 1 equals the
+ *             recorded bit; y >= 6 gives 6; a codeword keeps itself;
+ *             S == 0 gives signed zero.  The sign is always x's own.
+ *
+ * Layouts (all contiguous, row-major, flat element index i = r*cols + c):
+ *   x         bf16 [rows, cols], cols % 16 == 0 (NVFP4) / % 32 (MXFP4)
+ *   codes     uint8 [rows*cols/2]; element 2j in the low nibble of byte j
+ *   scales    uint8 [rows, cols/block] (linear, not swizzled)
+ *   s_t       float [num_segments] (NVFP4 only)
+ *   guidance  uint8 [rows*cols/8]; bit (i & 7) of byte (i >> 3) = m3_i & 1
+ *
+ * Segments.  NVFP4 may split the rows into num_segments groups (e.g. the
+ * per-expert groups of a mixture-of-experts dispatch), each with its own
+ * s_t.  seg_row_offsets is a HOST array of num_segments + 1 non-decreasing
+ * row offsets, first 0, last rows; empty segments are allowed (their s_t is
+ * 0).  NULL means one segment.  MXFP4 requires num_segments == 1.
+ *
+ * Ownership, streams, errors.  The caller owns every buffer (device memory
+ * unless stated).  The library never allocates, frees or synchronizes,
+ * except tf4_read_status, which synchronizes its stream.  Every call is
+ * asynchronous on `stream` and launches on the current CUDA device.
+ * Argument, shape and alignment problems are returned before anything is
+ * launched.  Device pointers must be 16-byte aligned (x, codes, dequant
+ * output, unpack output), 4-byte aligned (guidance, s_t, amax, workspace,
+ * dev_status); scale arrays have no alignment requirement.
+ * Data-dependent problems (a non-finite input) are OR-ed as
+ * TF4_DEV_NONFINITE into *dev_status (optional, may be NULL); the outputs
+ * of the affected segment (NVFP4 tensor-scale calls) or block are then
+ * unspecified.  A failed launch returns TF4_ERR_CUDA.
+ *
+ * Workspace.  NVFP4 rtn/sr/capture without amax_in, and tf4_segment_amax,
+ * need tf4_workspace_bytes(desc) bytes of device workspace that is
+ * zero-filled before its first use; each call leaves it zero-filled again
+ * when it completes.  Calls that may run concurrently must not share a
+ * workspace.
+ */
+#ifndef TRACE_FP4_H
+#define TRACE_FP4_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same handle type as cudaStream_t; NULL is the legacy default stream. */
+typedef struct CUstream_st* tf4_stream_t;
+
+typedef enum {
+  TF4_OK = 0,
+  TF4_ERR_INVALID_ARG = 1, /* NULL pointer, bad enum, bad segment offsets */
+  TF4_ERR_SHAPE = 2,       /* rows/cols invalid or cols % block != 0       */
+  TF4_ERR_ALIGN = 3,       /* pointer misaligned                            */
+  TF4_ERR_WORKSPACE = 4,   /* workspace missing or too small                */
+  TF4_ERR_NONFINITE = 5,   /* (tf4_read_status) a non-finite input was seen */
+  TF4_ERR_TIMEOUT = 6,     /* (tf4_read_status) a bounded device wait gave up */
+  TF4_ERR_CUDA = 7         /* a CUDA call failed                            */
+} tf4_status;
+
+typedef enum { TF4_NVFP4 = 0, TF4_MXFP4 = 1 } tf4_format;
+
+#define TF4_MAX_SEGMENTS 1024
+#define TF4_DEV_NONFINITE 1 /* bit OR-ed into *dev_status */
+#define TF4_DEV_TIMEOUT 2   /* bit OR-ed into *dev_status */
+
+typedef struct {
+  int32_t fmt;                    /* tf4_format                                */
+  int32_t num_segments;           /* >= 1; MXFP4: 1                           */
+  int64_t rows;                   /* >= 0                                      */
+  int64_t cols;                   /* > 0, multiple of the block size           */
+  const int64_t* seg_row_offsets; /* host, num_segments + 1 entries, or NULL  */
+} tf4_desc;
+
+/* Sizes in bytes.  record_bytes is the per-call quantization record: codes
+ * (with_codes != 0, the full information) or guidance bits (the compact
+ * information), plus scale bytes, plus 4 bytes of s_t per segment (NVFP4). */
+size_t tf4_workspace_bytes(const tf4_desc* desc);
+size_t tf4_codes_bytes(const tf4_desc* desc);
+size_t tf4_scales_bytes(const tf4_desc* desc);
+size_t tf4_guidance_bytes(const tf4_desc* desc);
+size_t tf4_record_bytes(const tf4_desc* desc, int with_codes);
+
+/* NVFP4 segment amax (the grid-wide |x| max pass) on its own: writes
+ * amax[num_segments] (device, float).  With several shards of one tensor
+ * on several GPUs, an all-reduce MAX of these values followed by
+ * quantize calls with amax_in gives every shard the tensor-wide scale. */
+tf4_status tf4_segment_amax(const tf4_desc* desc, const void* x, float* amax, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, tf4_stream_t stream);
+
+/* Round-to-nearest quantization.  NVFP4: s_t (device, [num_segments]) is
+ * written; amax_in (device, [num_segments], may be NULL) supplies the
+ * segment amax and skips the amax pass (no workspace needed).  MXFP4:
+ * amax_in, s_t and the workspace are ignored (pass NULL / 0). */
+tf4_status tf4_quantize_rtn(const tf4_desc* desc, const void* x, const float* amax_in,
+                            uint8_t* codes, uint8_t* scales, float* s_t, void* workspace,
+                            size_t workspace_bytes, int32_t* dev_status, tf4_stream_t stream);
+
+/* Stochastic rounding with the Philox4x32-10 stream keyed by `seed`;
+ * otherwise as tf4_quantize_rtn. */
+tf4_status tf4_quantize_sr(const tf4_desc* desc, const void* x, uint64_t seed,
+                           const float* amax_in, uint8_t* codes, uint8_t* scales, float* s_t,
+                           void* workspace, size_t workspace_bytes, int32_t* dev_status,
+                           tf4_stream_t stream);
+
+/* Rollout-side capture: tf4_quantize_rtn plus the compact guidance
+ * (m3 & 1 of every element) written to guidance_bits.  Pass
+ * guidance_bits = NULL for layers whose guidance is not kept (the caller
+ * picks the deepest L of N layers); the codes, scales and s_t are then
+ * exactly those of tf4_quantize_rtn. */
+tf4_status tf4_quantize_capture(const tf4_desc* desc, const void* x, const float* amax_in,
+                                uint8_t* codes, uint8_t* scales, float* s_t,
+                                uint8_t* guidance_bits, void* workspace, size_t workspace_bytes,
+                                int32_t* dev_status, tf4_stream_t stream);
+
+/* Train-side guided quantization of x (the trainer's value) with the
+ * rollout's recorded scale bytes, recorded s_t (NVFP4; NULL for MXFP4) and
+ * recorded guidance bits.  One pass over x, no workspace. */
+tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_t* rec_scales,
+                               const float* rec_s_t, const uint8_t* rec_bits, uint8_t* codes,
+                               int32_t* dev_status, tf4_stream_t stream);
+
+/* out[i] = (-1)^sign * fl32(V[m3] * S) as fp32 [rows, cols]. */
+tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint8_t* scales,
+                          const float* s_t, float* out, tf4_stream_t stream);
+
+/* Guidance extraction from codes produced elsewhere: bits = m3 & 1. */
+tf4_status tf4_pack_guidance(const tf4_desc* desc, const uint8_t* codes, uint8_t* bits,
+                             tf4_stream_t stream);
+
+/* mant[i] = (bits[i >> 3] >> (i & 7)) & 1, one uint8 per element. */
+tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_t* mant,
+                               tf4_stream_t stream);
+
+/* Synchronizes `stream`, reads *dev_status (device), returns TF4_OK,
+ * TF4_ERR_NONFINITE, TF4_ERR_TIMEOUT or TF4_ERR_CUDA, and clears it. */
+tf4_status tf4_read_status(int32_t* dev_status, tf4_stream_t stream);
+
+const char* tf4_status_string(tf4_status status);
+int tf4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TRACE_FP4_H */

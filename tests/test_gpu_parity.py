@@ -1,0 +1,407 @@
+"""Parity of the CUDA library (through its C ABI) with the CPU oracle.
+
+Bit-exact on codes, scale bytes, s_t bits, guidance bits and dequantized
+fp32 values.  Small cases are compared in full (several CTAs, ragged
+tails, empty segments); the full-size workloads are compared on sampled
+rows that the oracle computes one by one after its own full amax pass.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from fp4_block_scaled_quantizer_b200 import binding as B
+from fp4_block_scaled_quantizer_b200 import build as libbuild
+from fp4_block_scaled_quantizer_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+DEV = "cuda"
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    libbuild.build()
+    B.lib()
+    O.lib()
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+def f32_bits(a):
+    return np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+
+
+def assert_same(name, got, want):
+    got, want = np.asarray(got).reshape(-1), np.asarray(want).reshape(-1)
+    assert got.shape == want.shape, (name, got.shape, want.shape)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, f"{name}: {bad.size} mismatches, first at {bad[:8]}: got {got[bad[:8]]} want {want[bad[:8]]}"
+
+
+def check_quant(xb, fmt, mode=O.RTN, seg=None, seed=0, bits=True):
+    """Run the library on xb (bf16 CUDA tensor) and compare with the oracle."""
+    if mode == O.SR:
+        q = B.tf4_quantize_sr(xb, seed, fmt=fmt, seg_off=seg)
+    else:
+        q = B.tf4_quantize_capture(xb, fmt=fmt, seg_off=seg, guidance=bits)
+    assert B.read_status(xb.device) == 0
+    xs = W.bf16_bits(xb)
+    r = O.quantize(xs, fmt, mode, seg_off=seg, seed=seed, bits=bits and mode != O.SR)
+    assert r["status"] == 0
+    assert_same("codes", host(q.codes), r["codes"])
+    assert_same("scales", host(q.scales), r["scales"])
+    if fmt == O.NVFP4:
+        assert_same("s_t", f32_bits(host(q.s_t)), f32_bits(r["s_t"]))
+    if bits and mode != O.SR:
+        assert_same("bits", host(q.bits), r["bits"])
+    return q, r
+
+
+SHAPES_NV = [(1, 16), (1, 32), (3, 48), (5, 16 * 33), (37, 2048), (129, 4096), (1000, 80), (2, 16 * 3001)]
+SHAPES_MX = [(1, 32), (3, 64), (5, 32 * 33), (37, 2048), (129, 4096), (1000, 96), (2, 32 * 3001)]
+
+
+@pytest.mark.parametrize("shape", SHAPES_NV)
+def test_nvfp4_capture_shapes(shape):
+    xb = W.random_bf16(shape, seed=sum(shape), device=DEV, outlier_frac=0.003)
+    check_quant(xb, O.NVFP4)
+
+
+@pytest.mark.parametrize("shape", SHAPES_MX)
+def test_mxfp4_capture_shapes(shape):
+    xb = W.random_bf16(shape, seed=sum(shape) + 1, device=DEV, outlier_frac=0.003)
+    check_quant(xb, O.MXFP4)
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("seed", [0, 4, 2**40 + 3])
+def test_sr_parity(fmt, seed):
+    xb = W.random_bf16((67, 1024), seed=seed % 1000, device=DEV, outlier_frac=0.01)
+    check_quant(xb, fmt, O.SR, seed=seed)
+
+
+def test_rtn_equals_capture_without_guidance():
+    xb = W.random_bf16((64, 512), seed=3, device=DEV)
+    a = B.tf4_quantize_rtn(xb)
+    b = B.tf4_quantize_capture(xb, guidance=False)
+    assert torch.equal(a.codes, b.codes) and torch.equal(a.scales, b.scales) and torch.equal(a.s_t, b.s_t)
+
+
+def test_e2m1_exhaustive_via_unit_scale():
+    """MXFP4 blocks whose max is 4.0 have S = 1, so y = x: every bf16 value
+    with |x| < 8 (both signs) goes through the device rounding as itself."""
+    b = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    v = ((b.astype(np.uint32) << 16).view(np.float32))
+    sel = b[np.isfinite(v) & (np.abs(v) < 8.0)]
+    per = 31
+    nblk = (len(sel) + per - 1) // per
+    pad = np.zeros(nblk * per, np.uint16)
+    pad[: len(sel)] = sel
+    blocks = np.concatenate([np.full((nblk, 1), 0x4080, np.uint16), pad.reshape(nblk, per)], axis=1)
+    xb = W.from_bits(blocks, DEV)
+    check_quant(xb, O.MXFP4)
+
+
+def test_e4m3_block_scale_sweep():
+    """NVFP4 with s_t = 1 (amax = 2688): every positive bf16 block max up to
+    2688 gives r = bamax/6, sweeping the device E4M3 rounding."""
+    b = np.arange(1, 0x7F80, dtype=np.uint32).astype(np.uint16)
+    v = (b.astype(np.uint32) << 16).view(np.float32)
+    b = b[v <= 2688.0]
+    x = np.zeros((len(b) + 1, 16), np.uint16)
+    x[:-1, 0] = b
+    x[:-1, 1] = 0x8000 | b  # negative copy
+    x[:-1, 2:] = (b[:, None] >> 1) & 0x7F7F
+    x[-1, 0] = 0x4528  # 2688.0
+    check_quant(W.from_bits(x, DEV), O.NVFP4)
+
+
+def _near_tie_tensor(rng, s_mant, rows=256):
+    """Rows whose per-tensor scale is 'nice' (amax = 2688 * s), so that many
+    midpoint * S are bf16 values; elements sit on and around those points."""
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, 0.5, 1, 1.5, 2, 3, 4, 6])
+    out = np.zeros((rows, 16), np.float32)
+    for r in range(rows):
+        S = float(np.float32(rng.choice([0.5, 1.0, 1.25, 0.75, 1.5, 0.875]) * 2.0 ** rng.integers(-3, 3)))
+        pts = rng.choice(mids, 15) * S
+        out[r, 1:] = pts * (1 + rng.choice([-1, 0, 0, 1], 15) * 2.0 ** -8)
+        out[r, 0] = 6 * S
+    out[0, 0] = 2688.0 * s_mant
+    xb = torch.from_numpy(out).to(torch.bfloat16)
+    return xb
+
+
+@pytest.mark.parametrize("s_mant", [1.0, 0.5, 3.0])
+def test_near_tie_blocks(s_mant):
+    rng = np.random.default_rng(int(s_mant * 10))
+    xb = _near_tie_tensor(rng, s_mant).to(DEV)
+    check_quant(xb, O.NVFP4)
+    check_quant(xb, O.NVFP4, O.SR, seed=11)
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+def test_tiny_and_zero_scales(fmt):
+    x = np.zeros((8, 64), np.uint16)
+    x[1, :] = 0x0001          # smallest subnormals
+    x[2, 3] = 0x8000          # -0
+    x[3, :16] = np.arange(16) + 0x0080  # tiny normals
+    x[4, 5] = 0x0C00          # ~1e-35
+    xb = W.from_bits(x, DEV)
+    check_quant(xb, fmt)
+    seg = [0, 2, 2, 4, 8]
+    if fmt == O.NVFP4:
+        check_quant(xb, fmt, seg=seg)
+
+
+def test_segments_ragged_with_empties():
+    xb = W.random_bf16((300, 256), seed=9, device=DEV, outlier_frac=0.01)
+    seg = [0, 0, 1, 1, 50, 51, 51, 299, 300, 300]
+    q, r = check_quant(xb, O.NVFP4, seg=seg)
+    check_quant(xb, O.NVFP4, O.SR, seg=seg, seed=5)
+    xt = W.perturb(xb, 7, rel=0.02)
+    g = B.tf4_quantize_guided(xt, q)
+    want, st = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], O.NVFP4, rec_s_t=r["s_t"], seg_off=seg)
+    assert_same("guided", host(g), want)
+
+
+def test_segment_amax_and_amax_in():
+    xb = W.random_bf16((200, 512), seed=12, device=DEV, outlier_frac=0.01)
+    seg = [0, 20, 20, 150, 200]
+    amax = B.tf4_segment_amax(xb, seg)
+    want, _ = O.segment_amax(W.bf16_bits(xb), seg)
+    assert_same("amax", f32_bits(host(amax)), f32_bits(want))
+    a = B.tf4_quantize_capture(xb, seg_off=seg)
+    b = B.tf4_quantize_capture(xb, seg_off=seg, amax_in=amax)
+    for n in ("codes", "scales", "s_t", "bits"):
+        assert torch.equal(getattr(a, n), getattr(b, n)), n
+
+
+def test_workspace_returns_to_zero():
+    xb = W.random_bf16((64, 1024), seed=13, device=DEV)
+    seg = [0, 10, 64]
+    B.tf4_quantize_rtn(xb, seg_off=seg)
+    torch.cuda.synchronize()
+    for ws in B._ws_cache.values():
+        assert int(ws.count_nonzero()) == 0
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("perturb", [0.0, 1e-3, 0.05])
+def test_guided_parity(fmt, perturb):
+    xb = W.random_bf16((96, 1024), seed=17, device=DEV, outlier_frac=0.005)
+    q, r = check_quant(xb, fmt)
+    xt = W.perturb(xb, 23, rel=perturb) if perturb else xb
+    g = B.tf4_quantize_guided(xt, q)
+    assert B.read_status(xb.device) == 0
+    want, st = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"])
+    assert st == 0
+    assert_same("guided", host(g), want)
+    if perturb == 0.0:
+        assert torch.equal(g, q.codes)
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+def test_guided_reproduces_sr_capture(fmt):
+    xb = W.random_bf16((64, 512), seed=29, device=DEV)
+    q = B.tf4_quantize_sr(xb, 77, fmt=fmt)
+    q.bits = B.tf4_pack_guidance(q.codes, 64, 512, fmt)
+    g = B.tf4_quantize_guided(xb, q)
+    assert torch.equal(g, q.codes)
+
+
+def test_guided_near_ties():
+    rng = np.random.default_rng(5)
+    xb = _near_tie_tensor(rng, 1.0).to(DEV)
+    q, r = check_quant(xb, O.NVFP4)
+    xt = _near_tie_tensor(np.random.default_rng(6), 1.0).to(DEV)
+    g = B.tf4_quantize_guided(xt, q)
+    want, _ = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], O.NVFP4, rec_s_t=r["s_t"])
+    assert_same("guided", host(g), want)
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+def test_dequant_parity(fmt):
+    xb = W.random_bf16((77, 2048), seed=31, device=DEV, outlier_frac=0.01)
+    seg = [0, 30, 77] if fmt == O.NVFP4 else None
+    q, r = check_quant(xb, fmt, seg=seg)
+    d = B.tf4_dequantize(q)
+    want = O.dequantize(r["codes"], r["scales"], 77, 2048, fmt, s_t=r["s_t"], seg_off=seg)
+    assert_same("dequant", f32_bits(host(d)), f32_bits(want))
+
+
+@pytest.mark.parametrize("shape", [(1, 16), (3, 48), (64, 1024), (5, 16 * 33)])
+def test_pack_unpack_parity(shape):
+    rows, cols = shape
+    codes = torch.randint(0, 256, (rows * cols // 2,), dtype=torch.uint8, device=DEV)
+    bits = B.tf4_pack_guidance(codes, rows, cols)
+    want = O.pack_guidance(host(codes), rows * cols)
+    assert_same("pack", host(bits), want)
+    mant = B.tf4_unpack_guidance(bits, rows, cols)
+    assert_same("unpack", host(mant), O.unpack_guidance(want, rows * cols))
+
+
+def test_nonfinite_reported():
+    xb = W.random_bf16((40, 256), seed=37, device=DEV)
+    x = W.bf16_bits(xb)
+    x[25, 7] = 0x7F80
+    seg = [0, 20, 40]
+    xb = W.from_bits(x, DEV)
+    q = B.tf4_quantize_capture(xb, seg_off=seg)
+    assert B.read_status(xb.device) == 5
+    assert B.read_status(xb.device) == 0  # cleared
+    r = O.quantize(x[:20], O.NVFP4, bits=True)
+    assert_same("clean segment", host(q.codes)[: 20 * 128], r["codes"])
+    B.tf4_quantize_rtn(xb, fmt=B.MXFP4)
+    assert B.read_status(xb.device) == 5
+    x2 = W.bf16_bits(W.random_bf16((4, 64), seed=1, device=DEV))
+    q2 = B.tf4_quantize_capture(W.from_bits(x2, DEV))
+    x2[1, 1] = 0x7FC1
+    B.tf4_quantize_guided(W.from_bits(x2, DEV), q2)
+    assert B.read_status(xb.device) == 5
+
+
+def test_empty_tensor():
+    xb = torch.zeros((0, 64), dtype=torch.bfloat16, device=DEV)
+    q = B.tf4_quantize_capture(xb, seg_off=[0, 0, 0])
+    assert q.s_t.shape == (2,) and not q.s_t.any()
+
+
+def test_ste_identity_backward():
+    from fp4_block_scaled_quantizer_b200 import ste
+    xb = W.random_bf16((16, 256), seed=41, device=DEV).requires_grad_(True)
+    q = B.tf4_quantize_capture(xb.detach())
+    y = ste.guided_fake_quant(xb, q, out_dtype=torch.bfloat16)
+    g = torch.randn_like(y)
+    y.backward(g)
+    assert torch.equal(xb.grad, g)
+    d = B.tf4_dequantize(q)
+    assert torch.equal(y.float(), d.to(torch.bfloat16).float())
+
+
+# ------------------------------------------------------ full-size workloads
+def sample_rows(rows, seg=None, k=24, seed=0):
+    rng = np.random.default_rng(seed)
+    pick = {0, rows - 1, rows // 2}
+    if seg is not None:
+        for s in seg[1:-1]:
+            if 0 < s < rows:
+                pick |= {s - 1, s}
+    pick |= set(int(v) for v in rng.integers(0, rows, k))
+    return sorted(pick)
+
+
+def check_sampled(xb, q, fmt, seg=None, mode=O.RTN, seed=0, guided_x=None, g_codes=None):
+    rows, cols = xb.shape
+    xs = W.bf16_bits(xb)
+    s_t = None
+    if fmt == O.NVFP4:
+        s_t, st = O.segment_scales(xs, seg)
+        assert st == 0
+        assert_same("s_t", f32_bits(host(q.s_t)), f32_bits(s_t))
+    blk = O.BLOCK[fmt]
+    gcodes, gsc = host(q.codes), host(q.scales).reshape(-1)
+    gbits = host(q.bits) if q.bits is not None else None
+    xt = W.bf16_bits(guided_x) if guided_x is not None else None
+    gg = host(g_codes) if g_codes is not None else None
+    for r in sample_rows(rows, seg):
+        rr = O.quantize(xs, fmt, mode, seg_off=seg, seed=seed, s_t=s_t, row_range=(r, r + 1),
+                        bits=gbits is not None)
+        c0, c1 = r * cols // 2, (r + 1) * cols // 2
+        assert_same(f"codes row {r}", gcodes[c0:c1], rr["codes"][c0:c1])
+        assert_same(f"scales row {r}", gsc[r * cols // blk:(r + 1) * cols // blk],
+                    rr["scales"][r * cols // blk:(r + 1) * cols // blk])
+        if gbits is not None:
+            assert_same(f"bits row {r}", gbits[r * cols // 8:(r + 1) * cols // 8],
+                        rr["bits"][r * cols // 8:(r + 1) * cols // 8])
+        if xt is not None:
+            wg, _ = O.quantize_guided(xt, rr["scales"], rr["bits"], fmt, rec_s_t=s_t, seg_off=seg,
+                                      row_range=(r, r + 1))
+            assert_same(f"guided row {r}", gg[c0:c1], wg[c0:c1])
+
+
+def test_activation_outliers_full():
+    w = W.activation_outliers(DEV)
+    q, r = check_quant(w["x"], O.NVFP4)
+    for xt in (w["x_train"], w["x"]):
+        g = B.tf4_quantize_guided(xt, q)
+        want, _ = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], O.NVFP4, rec_s_t=r["s_t"])
+        assert_same("guided", host(g), want)
+
+
+@pytest.mark.parametrize("layer", [0, 39])
+def test_layer_stack_layer_sampled(layer):
+    x = W.layer_stack_layer(layer, DEV)
+    q = B.tf4_quantize_capture(x, guidance=layer >= 20)
+    g = B.tf4_quantize_guided(x, q) if layer >= 20 else None
+    assert B.read_status(x.device) == 0
+    check_sampled(x, q, O.NVFP4, g_codes=g, guided_x=x if g is not None else None)
+    if g is not None:
+        assert torch.equal(g, q.codes)
+
+
+def test_moe_dispatch_sampled():
+    w = W.moe_dispatch(DEV)
+    seg = w["seg_off"]
+    q = B.tf4_quantize_capture(w["x"], seg_off=seg)
+    g = B.tf4_quantize_guided(w["x_train"], q)
+    assert B.read_status(w["x"].device) == 0
+    check_sampled(w["x"], q, O.NVFP4, seg=seg, guided_x=w["x_train"], g_codes=g)
+
+
+def test_weights_sampled():
+    x = W.weights(DEV)
+    q = B.tf4_quantize_sr(x, 0)
+    check_sampled(x, q, O.NVFP4, mode=O.SR, seed=0)
+    qm = B.tf4_quantize_rtn(x, fmt=B.MXFP4)
+    check_sampled(x, qm, O.MXFP4)
+
+
+def test_kv_cache_sampled():
+    w = W.kv_cache(DEV)
+    for name in ("k", "v"):
+        x, xt = w[name], w[name + "_train"]
+        q = B.tf4_quantize_capture(x)
+        g = B.tf4_quantize_guided(xt, q)
+        check_sampled(x, q, O.NVFP4, guided_x=xt, g_codes=g)
+        assert torch.equal(B.tf4_quantize_guided(x, q), q.codes)
+
+
+def test_sr_counter_beyond_2_32():
+    """Element indices above 2^32 use the counter's high word: MXFP4 SR on a
+    (2^32 + 2^20)-element tensor, rows sampled across the boundary."""
+    cols = 4096
+    rows = (2**32 + 2**20) // cols
+    g = torch.Generator(device=DEV).manual_seed(8)
+    x = (torch.rand((rows, cols), generator=g, device=DEV) * 2 - 1).to(torch.bfloat16)
+    q = B.tf4_quantize_sr(x, 2**33 + 5, fmt=B.MXFP4)
+    torch.cuda.synchronize()
+    r0 = 2**32 // cols
+    for r in (0, r0 - 1, r0, r0 + 1, rows - 1):
+        want = _oracle_row_with_offset(W.bf16_bits(x[r:r + 1])[0], r * cols, 2**33 + 5)
+        assert_same(f"row {r}", host(q.codes[r * cols // 2:(r + 1) * cols // 2]), want)
+    del x, q
+    torch.cuda.empty_cache()
+
+
+def _oracle_row_with_offset(row_bits, base_index, seed):
+    """Oracle SR codes of one MXFP4 row whose first element has flat index
+    base_index (element-level oracle calls)."""
+    cols = len(row_bits)
+    out = np.zeros(cols // 2, np.uint8)
+    xf = (row_bits.astype(np.uint32) << 16).view(np.float32)
+    for b in range(cols // 32):
+        blk = row_bits[32 * b:32 * b + 32]
+        bamax = float(np.abs(xf[32 * b:32 * b + 32]).max())
+        e = O.e8m0_exponent(bamax)
+        S = 2.0 ** e
+        for k in range(32):
+            i = 32 * b + k
+            m3 = O.sr_m3(abs(float(xf[i])), S, O.sr_uniform24(base_index + i, seed))
+            nib = ((int(blk[k]) >> 15) << 3) | m3
+            out[i >> 1] |= nib << (4 * (i & 1))
+    return out
