@@ -304,6 +304,132 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, 
   if (tid == 0) ws[seg.count()] = 0u;
 }
 
+// ------------------------------------------------ per-segment scale tables
+// Within one segment (tensor scale s_t) an NVFP4 block with E4M3 scale code
+// b = (e_b, m_b), e_b >= 1, has S = fl(s_t * (1 + m_b/8) * 2^(e_b-7))
+// = S_c[m_b] * 2^(e_b-7) with S_c[m] = fl(s_t * (1 + m/8)) (power-of-two
+// scaling commutes with rounding in the normal range).  So a segment has
+// only 8 scale classes, and a few per-class constants replace the per-block
+// divisions:
+//  * rho[c]: a multiplier near 1/S_c such that, for every bf16 value v,
+//    RN(v * rho) lies on the same side of every decision point (E2M1
+//    midpoints for round-to-nearest, codewords for guided rounding) as the
+//    exact quotient v / S_c, and equals a decision point exactly iff v / S_c
+//    does.  Only the bf16 values next to a point * S_c can break this (all
+//    others are >= 2^-8 away, relative, while rho's error is < 2^-20), so
+//    each candidate (RN(1/S_c) +- up to 4 ulps) is checked on exactly those
+//    values with an exact FMA test; rho = 0 marks a class for which no
+//    candidate works (its blocks take the exact per-element path).
+//  * code[m]: the E4M3 scale code of bamax = (1 + m/128) * 2^(E0-127); for
+//    bamax = that * 2^k the code is code[m] + 8k while it stays a normal,
+//    unsaturated E4M3 value (both roundings are scale-invariant there).
+struct SegTables {
+  float rho[8];
+  uint32_t mask[8];  // candidate pass bits: [0, 9) round-to-nearest, [9, 18) toward zero
+  int E0;
+  int fast;
+  int rz;            // 1: the multiplies round toward zero (chosen per segment)
+  uint8_t code[128];
+};
+
+constexpr int kCand = 9;
+// candidate k -> ulp offset 0, +1, -1, +2, -2, ...
+__device__ __forceinline__ int cand_offset(int k) { return (k & 1) ? ((k + 1) >> 1) : -(k >> 1); }
+
+// Decision points: E2M1 midpoints (i = 0..6, tie -> upper iff i odd) or the
+// nonzero codewords (i = 0..6 -> V[i+1]).
+template <bool MIDPOINTS>
+__device__ __forceinline__ float decision_point(int i) {
+  return MIDPOINTS ? 0.5f * (e2m1_value((uint32_t)i) + e2m1_value((uint32_t)i + 1u))
+                   : e2m1_value((uint32_t)i + 1u);
+}
+
+template <bool RZ>
+__device__ __forceinline__ float mul(float a, float b) {
+  return RZ ? __fmul_rz(a, b) : __fmul_rn(a, b);
+}
+
+// All threads of the CTA call this (it synchronizes).  The multiplies may
+// round to nearest or toward zero (both are odd functions, so signed inputs
+// keep their symmetry); one mode is chosen per segment so that the block
+// loop stays uniform: toward zero if every class has a safe multiplier in
+// that mode, else to nearest if every class has one there, else the mode
+// with more safe classes (the others take the exact path).
+template <bool MIDPOINTS>
+__device__ void build_tables(float st, SegTables& t) {
+  const int tid = threadIdx.x;
+  __syncthreads();  // the previous piece is done with t
+  const bool fast = st >= 0x1p-90f && st <= 0x1p100f;
+  if (tid < 8) t.mask[tid] = (1u << (2 * kCand)) - 1u;
+  if (MIDPOINTS) {
+    const int E0 = fast ? (int)((__float_as_uint(__fmul_rn(st, 2688.0f)) >> 23) & 0xFFu) - 2 : 0;
+    if (tid == 0) {
+      t.E0 = E0;
+      t.fast = fast && E0 >= 4;
+    }
+    if (fast && E0 >= 4 && tid < 128) {
+      const float bam = __uint_as_float(((uint32_t)E0 << 23) | ((uint32_t)tid << 16));
+      t.code[tid] = (uint8_t)e4m3_encode(__fdiv_rn(__fdiv_rn(bam, 6.0f), st));
+    }
+  } else if (tid == 0) {
+    t.fast = fast;
+  }
+  __syncthreads();
+  if (fast && tid < 8 * 28) {
+    const int c = tid / 28, r = tid % 28, i = r >> 2, o = (r & 3) - 1;
+    const float Sc = __fmul_rn(st, 1.0f + 0.125f * (float)c);
+    const float pt = decision_point<MIDPOINTS>(i);
+    const float P = __fmul_rn(pt, Sc);
+    const float v = __uint_as_float((uint32_t)((int)(__float_as_uint(P) >> 16) + o) << 16);
+    const float e = fmaf(-pt, Sc, v);  // exact sign: Sc >= 2^-96
+    const uint32_t r0 = __float_as_uint(__frcp_rn(Sc));
+    const bool up = (i & 1) != 0;
+    uint32_t pass = 0;
+#pragma unroll
+    for (int k = 0; k < 2 * kCand; ++k) {
+      const float rk = __uint_as_float(r0 + cand_offset(k % kCand));
+      const float p = k < kCand ? __fmul_rn(v, rk) : __fmul_rz(v, rk);
+      bool ok;
+      if (MIDPOINTS) ok = ((e > 0.0f) || (e == 0.0f && up)) == ((p > pt) || (p == pt && up));
+      else ok = ((e > 0.0f) == (p > pt)) && ((e == 0.0f) == (p == pt));
+      pass |= (ok ? 1u : 0u) << k;
+    }
+    atomicAnd(&t.mask[c], pass);
+  }
+  __syncthreads();
+  if (tid < 32) {
+    const uint32_t m = tid < 8 ? t.mask[tid] : 0u;
+    const uint32_t lane = tid < 8 ? 0xFFu : 0u;
+    const uint32_t rz_ok = __ballot_sync(0xFFFFFFFFu, (m >> kCand) != 0u) & lane;
+    const uint32_t rn_ok = __ballot_sync(0xFFFFFFFFu, (m & ((1u << kCand) - 1u)) != 0u) & lane;
+    const bool rz = rz_ok == 0xFFu ? true : rn_ok == 0xFFu ? false : __popc(rz_ok) >= __popc(rn_ok);
+    if (tid < 8) {
+      const uint32_t mm = rz ? (m >> kCand) : (m & ((1u << kCand) - 1u));
+      float rho = 0.0f;
+      if (fast && mm) {
+        const float Sc = __fmul_rn(st, 1.0f + 0.125f * (float)tid);
+        rho = __uint_as_float(__float_as_uint(__frcp_rn(Sc)) + cand_offset(__ffs(mm) - 1));
+      }
+      t.rho[tid] = rho;
+    }
+    if (tid == 0) t.rz = rz;
+  }
+  __syncthreads();
+}
+
+// rho of class m_b scaled by 2^(7 - e_b) (exact exponent shift).
+__device__ __forceinline__ float block_rho(float rho_c, uint32_t e_b) {
+  return __uint_as_float(__float_as_uint(rho_c) + (uint32_t)((7 - (int)e_b) << 23));
+}
+
+// Eight bf16 (four words) times rho -> eight E2M1 nibbles (signed, RNE).
+template <bool RZ = false>
+__device__ __forceinline__ uint32_t cvt_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r) {
+  return cvt_e2m1x8(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r),
+                    mul<RZ>(bf_hi(w1), r), mul<RZ>(bf_lo(w2), r), mul<RZ>(bf_hi(w2), r),
+                    mul<RZ>(bf_lo(w3), r), mul<RZ>(bf_hi(w3), r));
+}
+
 // --------------------------------------------------------- quantize pass
 enum { kRTN = 0, kSR = 1, kCAPTURE = 2 };
 
@@ -321,36 +447,36 @@ struct QuantArgs {
 };
 
 // One NVFP4 block (16 bf16 in w[0..7]) -> code words, scale byte, flags.
-template <int MODE>
-__device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, int64_t blk,
-                                            uint64_t seed, uint32_t& c0, uint32_t& c1,
+template <int MODE, bool RZ>
+__device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, const SegTables& t,
+                                            int64_t blk, uint64_t seed, uint32_t& c0, uint32_t& c1,
                                             uint32_t& sc, bool& bad) {
   const uint32_t mb = block_absmax_bits(w);
   bad = mb >= 0x7F80u;
+  if (MODE != kSR && t.fast && !bad) {
+    const int E = (int)(mb >> 7);
+    const int code = (int)t.code[mb & 0x7Fu] + 8 * (E - t.E0);
+    if (E >= 4 && code >= 8) {
+      sc = (uint32_t)min(code, 0x7E);
+      const float rho = t.rho[sc & 7u];
+      if (rho != 0.0f) {
+        const float r = block_rho(rho, sc >> 3);
+        c0 = cvt_words<RZ>(w[0], w[1], w[2], w[3], r);
+        c1 = cvt_words<RZ>(w[4], w[5], w[6], w[7], r);
+        return;
+      }
+    }
+  }
+  // Exact path: scale by the defining divisions, decisions by exact
+  // comparisons (E4M3-subnormal or zero scales, classes without a safe
+  // multiplier, tiny segments, stochastic rounding).
   float S = 0.0f;
   sc = 0;
   if (st > 0.0f) {  // st == 0: zero segment; NaN: non-finite segment
     const float bamax = __uint_as_float(mb << 16);
-    const float q = __fdiv_rn(bamax, 6.0f);
-    const float r = __fdiv_rn(q, st);
-    sc = e4m3_encode(r);
+    sc = e4m3_encode(__fdiv_rn(__fdiv_rn(bamax, 6.0f), st));
     S = __fmul_rn(st, e4m3_decode(sc));
   }
-  if (MODE != kSR && S > 0.0f &&
-      !(S < 0x1p-100f || near_bf16(S) || near_bf16(__fmul_rn(3.0f, S)) ||
-        near_bf16(__fmul_rn(5.0f, S)) || near_bf16(__fmul_rn(7.0f, S)))) {
-    // Fast path: no bf16 value lies within 2^-21 (relative) of any
-    // midpoint * S, so the rounded quotient x * RN(1/S) (relative error
-    // < 2^-22.9) falls on the same side of every midpoint as the exact one
-    // and never on a midpoint: hardware RNE of it is the exact answer.
-    const float rS = __frcp_rn(S);
-    c0 = cvt_e2m1x8(bf_lo(w[0]) * rS, bf_hi(w[0]) * rS, bf_lo(w[1]) * rS, bf_hi(w[1]) * rS,
-                    bf_lo(w[2]) * rS, bf_hi(w[2]) * rS, bf_lo(w[3]) * rS, bf_hi(w[3]) * rS);
-    c1 = cvt_e2m1x8(bf_lo(w[4]) * rS, bf_hi(w[4]) * rS, bf_lo(w[5]) * rS, bf_hi(w[5]) * rS,
-                    bf_lo(w[6]) * rS, bf_hi(w[6]) * rS, bf_lo(w[7]) * rS, bf_hi(w[7]) * rS);
-    return;
-  }
-  // Exact path (near-tie scales, tiny or zero scales, stochastic rounding).
   uint32_t out[2] = {0u, 0u};
 #pragma unroll
   for (int k = 0; k < 16; ++k) {
@@ -384,11 +510,7 @@ __device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk
     // so hardware RNE of y is the exact answer.
     const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
 #pragma unroll
-    for (int q = 0; q < 4; ++q)
-      c[q] = cvt_e2m1x8(bf_lo(w[4 * q]) * inv, bf_hi(w[4 * q]) * inv, bf_lo(w[4 * q + 1]) * inv,
-                        bf_hi(w[4 * q + 1]) * inv, bf_lo(w[4 * q + 2]) * inv,
-                        bf_hi(w[4 * q + 2]) * inv, bf_lo(w[4 * q + 3]) * inv,
-                        bf_hi(w[4 * q + 3]) * inv);
+    for (int q = 0; q < 4; ++q) c[q] = cvt_words(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], inv);
     return;
   }
   const float S = __uint_as_float(e >= -126 ? (uint32_t)(e + 127) << 23 : 0x00400000u);
@@ -413,6 +535,7 @@ __device__ __forceinline__ void report_bad(bool bad, int32_t* status) {
 template <int FMT, int MODE, class SEG>
 __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
   constexpr int U = 2;  // blocks per lane per iteration
+  __shared__ SegTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   const int tid = threadIdx.x;
@@ -423,7 +546,19 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
     const int s = seg.find(hi - 1);
     const int64_t lo = max(b0, seg.start(s));
     float st = 0.0f;
-    if constexpr (FMT == TF4_NVFP4) st = a.st_from_amax ? tensor_scale(a.st_src[s], nullptr) : a.st_src[s];
+    if constexpr (FMT == TF4_NVFP4) {
+      st = a.st_from_amax ? tensor_scale(a.st_src[s], nullptr) : a.st_src[s];
+      if (MODE != kSR) {
+        build_tables<true>(st, tb);
+      } else {
+        __syncthreads();
+        if (tid == 0) {
+          tb.fast = 0;
+          tb.rz = 0;
+        }
+        __syncthreads();
+      }
+    }
     const int64_t n = hi - lo;
     for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
       if constexpr (FMT == TF4_NVFP4) {
@@ -445,7 +580,10 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
           bool bad = false;
           if (valid) {
             uint32_t c0, c1, sc;
-            nvfp4_block<MODE>(w[u], st, blk[u], a.seed, c0, c1, sc, bad);
+            if (tb.rz)
+              nvfp4_block<MODE, true>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
+            else
+              nvfp4_block<MODE, false>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
             reinterpret_cast<uint2*>(a.codes)[blk[u]] = make_uint2(c0, c1);
             a.scales[blk[u]] = (uint8_t)sc;
             if (MODE == kCAPTURE && a.bits)
@@ -492,6 +630,13 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
 }
 
 // ----------------------------------------------------------- guided pass
+// Guided rounding = nearest rounding whenever the nearest neighbour already
+// carries the recorded mantissa bit: of the two neighbours lo < y < hi the
+// nearest is one of them, and exactly one has m3 & 1 == g.  So each block
+// is rounded to nearest on the fast path (a multiplier that decides every
+// codeword comparison exactly), the code words are compared with the
+// recorded bits nibble-wise, and only mismatching elements are moved to the
+// other neighbour (or kept: a value equal to a codeword, y >= 6).
 struct GuidedArgs {
   const uint4* x;
   int64_t nblocks;
@@ -502,10 +647,44 @@ struct GuidedArgs {
   int32_t* status;
 };
 
+// 8 guidance bits -> bit 0 of 8 nibbles
+__device__ __forceinline__ uint32_t spread_bits(uint32_t b) {
+  uint32_t x = b & 0xFFu;
+  x = (x | (x << 12)) & 0x000F000Fu;
+  x = (x | (x << 6)) & 0x03030303u;
+  x = (x | (x << 3)) & 0x11111111u;
+  return x;
+}
+
+// Fix the nibbles of code word c (values in the four bf16-pair words
+// w0..w3) whose m3 & 1 differs from the recorded bit (mm: mismatch bits at
+// nibble bit 0): keep exact codewords and the saturated top, otherwise step
+// to the other neighbour.
+template <bool RZ>
+__device__ __forceinline__ uint32_t fix_mismatches(uint32_t c, uint32_t mm, uint32_t w0, uint32_t w1,
+                                                   uint32_t w2, uint32_t w3, float r) {
+  while (mm) {
+    const int e = (__ffs(mm) - 1) >> 2;  // element within the word
+    mm &= mm - 1u;
+    const uint32_t wsel = (e & 4) ? ((e & 2) ? w3 : w2) : ((e & 2) ? w1 : w0);
+    const uint32_t h = (e & 1) ? (wsel >> 16) : (wsel & 0xFFFFu);
+    const float y = mul<RZ>(__uint_as_float((h & 0x7FFFu) << 16), r);
+    const uint32_t n = (c >> (4 * e)) & 7u;
+    const float v = e2m1_value(n);
+    if (!(y == v || (n == 7u && y >= 6.0f))) {
+      const uint32_t n2 = y > v ? n + 1u : n - 1u;
+      c = (c & ~(7u << (4 * e))) | (n2 << (4 * e));
+    }
+  }
+  return c;
+}
+
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
   constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;  // elements per block
   constexpr int NW = BE / 2;                       // bf16 pair words per block
+  constexpr int NQ = BE / 8;                       // code words per block
+  __shared__ SegTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   const int tid = threadIdx.x;
@@ -513,7 +692,11 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
   while (lo < b1) {
     const int s = seg.find(lo);
     const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
-    const float st = FMT == TF4_NVFP4 ? a.rec_s_t[s] : 0.0f;
+    float st = 0.0f;
+    if constexpr (FMT == TF4_NVFP4) {
+      st = a.rec_s_t[s];
+      build_tables<false>(st, tb);
+    }
     const int64_t n = hi - lo;
     for (int64_t j = 0; j < n; j += kThreads) {
       const int64_t k = j + tid;
@@ -531,19 +714,39 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
         uint32_t g;
         if constexpr (FMT == TF4_NVFP4) g = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
         else g = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
-        float S;
-        if constexpr (FMT == TF4_NVFP4) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
-        else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
         bad = block_absmax_bits(w) >= 0x7F80u;
-        uint32_t c[BE / 8];
+        uint32_t c[NQ];
+        float r = 0.0f;
+        if constexpr (FMT == TF4_NVFP4) {
+          if (tb.fast && (sc >> 3) >= 1u && sc < 0x7Fu) r = block_rho(tb.rho[sc & 7u], sc >> 3);
+          if (tb.rho[sc & 7u] == 0.0f) r = 0.0f;
+        } else {
+          if (sc >= 1u && sc <= 252u) r = __uint_as_float((254u - sc) << 23);  // 2^-(sc-127), exact
+        }
+        if (r != 0.0f) {
+          const bool rz = FMT == TF4_NVFP4 && tb.rz;
 #pragma unroll
-        for (int q = 0; q < BE / 8; ++q) c[q] = 0u;
+          for (int q = 0; q < NQ; ++q) {
+            c[q] = rz ? cvt_words<true>(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], r)
+                      : cvt_words<false>(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], r);
+            const uint32_t mm = (c[q] ^ spread_bits(g >> (8 * q))) & 0x11111111u;
+            if (mm)
+              c[q] = rz ? fix_mismatches<true>(c[q], mm, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], r)
+                        : fix_mismatches<false>(c[q], mm, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], r);
+          }
+        } else {
+          float S;
+          if constexpr (FMT == TF4_NVFP4) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
+          else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
 #pragma unroll
-        for (int e = 0; e < BE; ++e) {
-          const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-          const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-          const uint32_t m3 = S > 0.0f ? guided_m3_exact(ax, S, (g >> e) & 1u) : 0u;
-          c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
+          for (int q = 0; q < NQ; ++q) c[q] = 0u;
+#pragma unroll
+          for (int e = 0; e < BE; ++e) {
+            const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+            const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+            const uint32_t m3 = S > 0.0f ? guided_m3_exact(ax, S, (g >> e) & 1u) : 0u;
+            c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
+          }
         }
         if constexpr (FMT == TF4_NVFP4) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
         else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);

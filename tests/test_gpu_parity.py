@@ -206,6 +206,19 @@ def test_guided_parity(fmt, perturb):
 
 
 @pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+def test_guided_unrelated_train_tensor(fmt):
+    """Train-side values unrelated to the rollout's (about half the nibbles
+    disagree with the recorded bit): every element still lands on the
+    neighbour the oracle picks."""
+    xb = W.random_bf16((80, 2048), seed=19, device=DEV, outlier_frac=0.005)
+    q, r = check_quant(xb, fmt)
+    xt = W.random_bf16((80, 2048), seed=20, device=DEV, outlier_frac=0.005)
+    g = B.tf4_quantize_guided(xt, q)
+    want, _ = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"])
+    assert_same("guided", host(g), want)
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
 def test_guided_reproduces_sr_capture(fmt):
     xb = W.random_bf16((64, 512), seed=29, device=DEV)
     q = B.tf4_quantize_sr(xb, 77, fmt=fmt)
