@@ -40,7 +40,8 @@ EXPORTS = (
     "tf4_workspace_bytes", "tf4_codes_bytes", "tf4_scales_bytes", "tf4_guidance_bytes",
     "tf4_record_bytes", "tf4_segment_amax", "tf4_quantize_rtn", "tf4_quantize_sr",
     "tf4_quantize_capture", "tf4_quantize_guided", "tf4_dequantize", "tf4_pack_guidance",
-    "tf4_unpack_guidance", "tf4_read_status", "tf4_status_string", "tf4_version",
+    "tf4_unpack_guidance", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
+    "tf4_version",
 )
 
 
@@ -91,6 +92,7 @@ def lib():
                     "tf4_dequantize": (st, [dp, vp, vp, vp, vp, vp]),
                     "tf4_pack_guidance": (st, [dp, vp, vp, vp]),
                     "tf4_unpack_guidance": (st, [dp, vp, vp, vp]),
+                    "tf4_quantize_capture_noalloc": (st, [dp, vp, vp, vp, vp, vp, i32p, vp]),
                     "tf4_read_status": (st, [i32p, vp]),
                     "tf4_status_string": (ctypes.c_char_p, [st]),
                     "tf4_version": (ctypes.c_int, []),

@@ -191,6 +191,33 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
   return launched();
 }
 
+// Scratch of the allocation-free capture: the amax pass's per-segment
+// maxima and its completion counter, in a fixed device array owned by the
+// library (zero at load; cleared again by every call that uses it).  Sized
+// like a workspace for TF4_NOALLOC_MAX_SEGMENTS segments (whole 256-byte
+// units: 1280 bytes).
+constexpr int kNoAllocWords = ((TF4_NOALLOC_MAX_SEGMENTS + 1) * 4 + 255) / 256 * 64;
+static __device__ __align__(256) uint32_t tf4_noalloc_scratch[kNoAllocWords];
+
+// Device address of tf4_noalloc_scratch on the current device, looked up
+// once per device (with that device current) and cached.
+uint32_t* noalloc_scratch() {
+  static uint32_t* addr[128] = {nullptr};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, tf4_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    addr[dev] = static_cast<uint32_t*>(p);
+  }
+  return addr[dev];
+}
+
 }  // namespace
 
 extern "C" {
@@ -361,6 +388,22 @@ tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_
   const int64_t g = wave_grid(tf4::k_unpack, units > 0 ? units : 1);
   tf4::k_unpack<<<(unsigned)g, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(bits, mant, units, tail);
   return launched();
+}
+
+tf4_status tf4_quantize_capture_noalloc(const tf4_desc* desc, const void* x, uint8_t* codes, uint8_t* scales,
+                                        float* s_t, uint8_t* bits, int32_t* status, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.nseg > TF4_NOALLOC_MAX_SEGMENTS) return TF4_ERR_WORKSPACE;
+  uint32_t* scratch = noalloc_scratch();
+  if (!scratch) return TF4_ERR_CUDA;
+  const size_t need = sizeof(uint32_t) * (size_t)(sh.nseg + 1);
+  if (sh.fmt == TF4_NVFP4 && sh.n > 0 &&
+      cudaMemsetAsync(scratch, 0, need, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return TF4_ERR_CUDA;
+  return tf4_quantize_capture(desc, x, nullptr, codes, scales, s_t, bits, scratch, sizeof(tf4_noalloc_scratch),
+                              status, stream);
 }
 
 tf4_status tf4_read_status(int32_t* dev_status, tf4_stream_t stream) {

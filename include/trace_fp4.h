@@ -172,6 +172,31 @@ tf4_status tf4_pack_guidance(const tf4_desc* desc, const uint8_t* codes, uint8_t
 tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_t* mant,
                                tf4_stream_t stream);
 
+/* Allocation-free capture (the paper has no counterpart; this is a library
+ * convenience).  Some callers cannot allocate device memory or hand out a
+ * workspace: for example a plug-in running inside an engine that owns all
+ * device memory, or code on a path where an allocation, which can
+ * synchronize the device, is not allowed.  This variant of
+ * tf4_quantize_capture takes no workspace: the scratch of its amax pass
+ * (num_segments + 1 words) lives in a fixed array of device memory inside
+ * the library, which every GPU that loads the library holds until the
+ * process exits (1280 bytes per GPU).
+ *  - Limit: desc->num_segments <= TF4_NOALLOC_MAX_SEGMENTS, else
+ *    TF4_ERR_WORKSPACE is returned and nothing is launched.
+ *  - The first call on a device looks up that device's address of the
+ *    array; make that first call before any stream capture.
+ *  - Each call clears the scratch it needs (an asynchronous memset on
+ *    `stream`) and then behaves exactly like tf4_quantize_capture with
+ *    amax_in = NULL.  It calls no cudaMalloc or cudaFree.
+ *  - All calls on a device share the one array: calls that may overlap on
+ *    the GPU (different streams without ordering) race and must not be
+ *    issued; serialize them, or use tf4_quantize_capture with one
+ *    workspace per stream. */
+#define TF4_NOALLOC_MAX_SEGMENTS 256
+tf4_status tf4_quantize_capture_noalloc(const tf4_desc* desc, const void* x, uint8_t* codes,
+                                        uint8_t* scales, float* s_t, uint8_t* guidance_bits,
+                                        int32_t* dev_status, tf4_stream_t stream);
+
 /* Synchronizes `stream`, reads *dev_status (device), returns TF4_OK,
  * TF4_ERR_NONFINITE, TF4_ERR_TIMEOUT or TF4_ERR_CUDA, and clears it. */
 tf4_status tf4_read_status(int32_t* dev_status, tf4_stream_t stream);
