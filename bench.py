@@ -61,6 +61,8 @@ def parse():
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=256, help="rows per layer in the oracle sample")
     p.add_argument("--ref-rows", type=int, default=48, help="rows per layer per reference step")
+    p.add_argument("--suite", action="store_true",
+                   help="time every call of the path on every workload (a table, not the bench line)")
     return p.parse_args()
 
 
@@ -295,7 +297,8 @@ def run_ours(args, world, rank, local):
         calls[k] = dict(us=round(v["ms"] * 1e3, 2), gbs=round(gbs, 1), frac=round(gbs / peak, 4),
                         share=round(shares[k] / tot, 4))
     dom = max(shares, key=shares.get)
-    kname = {"amax": "k_amax", "quant": "k_quant(NVFP4, capture)", "guided": "k_guided(NVFP4)"}[dom]
+    kname = {"amax": "k_amax", "quant": "k_quant (NVFP4: RTN layers 0-19, capture layers 20-39)",
+             "guided": "k_guided(NVFP4)"}[dom]
     achieved = per_kernel[dom]["bytes"] / (per_kernel[dom]["ms"] * 1e-3) / 1e9
     tr = ncu_traffic(dom)
     roofline = dict(bound="hbm", kernel=kname, achieved=round(achieved, 1), peak=peak, unit="GB/s",
@@ -494,8 +497,111 @@ def run_reference(args, world, rank):
                 e2e=dict(value=v, unit="GB/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
 
 
+# ------------------------------------------------------------------ suite
+# algorithmic bytes per element of each call (reads the definition forces on
+# a tensor larger than on-chip memory, plus the writes)
+CALL_BYTES = {
+    ("nvfp4", "rtn"): 4.5625, ("nvfp4", "sr"): 4.5625, ("nvfp4", "capture"): 4.6875,
+    ("nvfp4", "guided"): 2.6875, ("nvfp4", "dequant"): 4.5625, ("nvfp4", "amax"): 2.0,
+    ("mxfp4", "rtn"): 2.53125, ("mxfp4", "sr"): 2.53125, ("mxfp4", "capture"): 2.65625,
+    ("mxfp4", "guided"): 2.65625, ("mxfp4", "dequant"): 4.53125,
+    ("any", "pack"): 0.625, ("any", "unpack"): 1.125,
+}
+
+
+def run_suite(args):
+    """Every call of the path on every workload, CUDA-event timed (3 warm-up
+    calls, then the mean of 10); GB/s from the algorithmic bytes above."""
+    from fp4_block_scaled_quantizer_b200 import binding as B
+    from fp4_block_scaled_quantizer_b200 import build as libbuild
+    from fp4_block_scaled_quantizer_b200 import workloads as W
+
+    libbuild.build()
+    dev = torch.device("cuda", 0)
+    peak, peak_kind = hbm_peak()
+    rows_out = []
+
+    def timed(fn, reps=10):
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(reps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / reps * 1e3  # us
+
+    def record(workload, fmt, call, n, us):
+        gbs = CALL_BYTES[(fmt, call)] * n / (us * 1e-6) / 1e9
+        rows_out.append(dict(workload=workload, format=fmt, call=call, elements=n, us=round(us, 2),
+                             gbs=round(gbs, 1), frac=round(gbs / peak, 4)))
+
+    def nv_calls(name, x, xt, seg=None):
+        n = x.numel()
+        q = B.tf4_quantize_capture(x, seg_off=seg)
+        amax = B.tf4_segment_amax(x, seg)
+        g = torch.empty_like(q.codes)
+        out = torch.empty(x.shape, dtype=torch.float32, device=dev)
+        bits = torch.empty(n // 8, dtype=torch.uint8, device=dev)
+        mant = torch.empty(n, dtype=torch.uint8, device=dev)
+        qr = B.tf4_quantize_rtn(x, seg_off=seg)
+        record(name, "nvfp4", "amax", n, timed(lambda: B.tf4_segment_amax(x, seg, out=amax)))
+        record(name, "nvfp4", "rtn", n, timed(lambda: B.tf4_quantize_rtn(x, seg_off=seg, out=qr)))
+        record(name, "nvfp4", "capture", n, timed(lambda: B.tf4_quantize_capture(x, seg_off=seg, out=q)))
+        record(name, "nvfp4", "guided", n, timed(lambda: B.tf4_quantize_guided(xt, q, out=g)))
+        record(name, "nvfp4", "sr", n, timed(lambda: B.tf4_quantize_sr(x, 4, seg_off=seg, out=qr)))
+        record(name, "nvfp4", "dequant", n, timed(lambda: B.tf4_dequantize(q, out=out)))
+        rows, cols = x.shape
+        record(name, "any", "pack", n, timed(lambda: B.tf4_pack_guidance(q.codes, rows, cols, out=bits)))
+        record(name, "any", "unpack", n, timed(lambda: B.tf4_unpack_guidance(bits, rows, cols, out=mant)))
+        del q, g, out, bits, mant, qr
+
+    def mx_calls(name, x, xt):
+        if x.shape[1] % 32:
+            return
+        n = x.numel()
+        q = B.tf4_quantize_capture(x, fmt=B.MXFP4)
+        g = torch.empty_like(q.codes)
+        out = torch.empty(x.shape, dtype=torch.float32, device=dev)
+        qr = B.tf4_quantize_rtn(x, fmt=B.MXFP4)
+        record(name, "mxfp4", "rtn", n, timed(lambda: B.tf4_quantize_rtn(x, fmt=B.MXFP4, out=qr)))
+        record(name, "mxfp4", "capture", n, timed(lambda: B.tf4_quantize_capture(x, fmt=B.MXFP4, out=q)))
+        record(name, "mxfp4", "guided", n, timed(lambda: B.tf4_quantize_guided(xt, q, out=g)))
+        record(name, "mxfp4", "sr", n, timed(lambda: B.tf4_quantize_sr(x, 4, fmt=B.MXFP4, out=qr)))
+        record(name, "mxfp4", "dequant", n, timed(lambda: B.tf4_dequantize(q, out=out)))
+        del q, g, out, qr
+
+    w = W.activation_outliers(dev)
+    nv_calls("activation_outliers 4096x2048", w["x"], w["x_train"])
+    mx_calls("activation_outliers 4096x2048", w["x"], w["x_train"])
+    del w
+    x = W.layer_stack_layer(20, dev)
+    xt = W.perturb(x, 1020)
+    nv_calls("layer_stack layer 65536x4096", x, xt)
+    mx_calls("layer_stack layer 65536x4096", x, xt)
+    del x, xt
+    w = W.moe_dispatch(dev)
+    nv_calls("moe_dispatch 262144x2048, 128 experts", w["x"], w["x_train"], seg=w["seg_off"])
+    del w
+    x = W.weights(dev)
+    nv_calls("weights 8192x28672", x, W.perturb(x, 44))
+    mx_calls("weights 8192x28672", x, W.perturb(x, 44))
+    del x
+    w = W.kv_cache(dev)
+    nv_calls("kv_cache K 1048576x128", w["k"], w["k_train"])
+    mx_calls("kv_cache K 1048576x128", w["k"], w["k_train"])
+    del w
+    torch.cuda.empty_cache()
+    return dict(peak_gbs=peak, peak_kind=peak_kind, rows=rows_out)
+
+
 def main():
     args = parse()
+    if args.suite:
+        print(json.dumps(run_suite(args)), flush=True)
+        return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
         rank = int(os.environ.get("RANK", "0"))
