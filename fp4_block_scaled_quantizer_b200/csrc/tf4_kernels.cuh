@@ -93,18 +93,6 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float v0, float v1, float v2, flo
   return r;
 }
 
-// Four packed e2m1 pairs (4 bytes) -> eight halves (hardware conversion).
-__device__ __forceinline__ void e2m1x8_to_half(uint32_t c, uint32_t (&h)[4]) {
-  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-      "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
-      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
-      : "r"(c));
-}
-
 // m3 & 1 of eight nibbles -> eight bits (nibble k -> bit k).
 __device__ __forceinline__ uint32_t nibble_lsbs(uint32_t c) {
   uint32_t t = c & 0x11111111u;
@@ -225,6 +213,27 @@ __device__ __forceinline__ uint32_t sr_m3_exact(float axf, float Sf, uint32_t r2
   const double lhs = (double)r24 * (vhi - vlo) * S;
   const double rhs = 16777216.0 * (ax - vlo * S);
   return lhs < rhs ? f + 1u : f;
+}
+
+// Stochastic rounding from y = |x| / S given either exactly (MXFP4) or as a
+// product that is on the correct side of every codeword and equals one iff
+// y does (NVFP4 fast path).  lo / gap come from the fp32 bits of y (for
+// y >= 1 the grid is the 1-mantissa-bit truncation, gap 2^(E-1); below 1 it
+// is {0, 0.5} with gap 0.5), and the threshold t = 2^24 (y - V_lo) / gap is
+// exact arithmetic on y (Sterbenz subtraction, power-of-two scaling).  With
+// an approximate y, |t - T_exact| < 64, so a uniform within 128 of t is
+// flagged `amb` for the exact test.  Returns the chosen codeword value.
+__device__ __forceinline__ float sr_pick(float y, uint32_t r24, bool margin, bool& amb) {
+  const uint32_t yb = __float_as_uint(y);
+  const bool ge1 = y >= 1.0f;
+  const float vlo = ge1 ? __uint_as_float(yb & 0xFFC00000u) : (y >= 0.5f ? 0.5f : 0.0f);
+  const float gap = ge1 ? __uint_as_float((yb & 0x7F800000u) - 0x00800000u) : 0.5f;
+  const float inv = ge1 ? __uint_as_float((279u - (yb >> 23)) << 23) : 0x1p25f;  // 2^24 / gap
+  const float t = __fmul_rn(__fsub_rn(y, vlo), inv);
+  const float rf = __uint2float_rn(r24);  // exact: r24 < 2^24
+  amb = margin && fabsf(rf - t) <= 128.0f;
+  const float v = rf < t ? __fadd_rn(vlo, gap) : vlo;
+  return fminf(v, 6.0f);
 }
 
 // -------------------------------------------------------------- amax pass
@@ -355,13 +364,13 @@ __device__ __forceinline__ float mul(float a, float b) {
 // loop stays uniform: toward zero if every class has a safe multiplier in
 // that mode, else to nearest if every class has one there, else the mode
 // with more safe classes (the others take the exact path).
-template <bool MIDPOINTS>
+template <bool MIDPOINTS, bool CODE_TABLE = MIDPOINTS>
 __device__ void build_tables(float st, SegTables& t) {
   const int tid = threadIdx.x;
   __syncthreads();  // the previous piece is done with t
   const bool fast = st >= 0x1p-90f && st <= 0x1p100f;
   if (tid < 8) t.mask[tid] = (1u << (2 * kCand)) - 1u;
-  if (MIDPOINTS) {
+  if (CODE_TABLE) {
     const int E0 = fast ? (int)((__float_as_uint(__fmul_rn(st, 2688.0f)) >> 23) & 0xFFu) - 2 : 0;
     if (tid == 0) {
       t.E0 = E0;
@@ -453,7 +462,7 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
                                             uint32_t& sc, bool& bad) {
   const uint32_t mb = block_absmax_bits(w);
   bad = mb >= 0x7F80u;
-  if (MODE != kSR && t.fast && !bad) {
+  if (t.fast && !bad) {
     const int E = (int)(mb >> 7);
     const int code = (int)t.code[mb & 0x7Fu] + 8 * (E - t.E0);
     if (E >= 4 && code >= 8) {
@@ -461,15 +470,35 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
       const float rho = t.rho[sc & 7u];
       if (rho != 0.0f) {
         const float r = block_rho(rho, sc >> 3);
-        c0 = cvt_words<RZ>(w[0], w[1], w[2], w[3], r);
-        c1 = cvt_words<RZ>(w[4], w[5], w[6], w[7], r);
-        return;
+        if (MODE != kSR) {
+          c0 = cvt_words<RZ>(w[0], w[1], w[2], w[3], r);
+          c1 = cvt_words<RZ>(w[4], w[5], w[6], w[7], r);
+          return;
+        } else {
+          // stochastic rounding on the codeword-safe product; rare
+          // ambiguous thresholds are decided exactly
+          const float S = __fmul_rn(st, e4m3_decode(sc));
+          float v[16];
+#pragma unroll
+          for (int k = 0; k < 16; ++k) {
+            const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
+            const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+            const uint32_t r24 = philox_w0((uint64_t)blk * 16u + k, seed) >> 8;
+            bool amb;
+            float val = sr_pick(mul<RZ>(ax, r), r24, true, amb);
+            if (amb) val = e2m1_value(sr_m3_exact(ax, S, r24));
+            v[k] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
+          }
+          c0 = cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+          c1 = cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+          return;
+        }
       }
     }
   }
   // Exact path: scale by the defining divisions, decisions by exact
   // comparisons (E4M3-subnormal or zero scales, classes without a safe
-  // multiplier, tiny segments, stochastic rounding).
+  // multiplier, tiny segments).
   float S = 0.0f;
   sc = 0;
   if (st > 0.0f) {  // st == 0: zero segment; NaN: non-finite segment
@@ -513,16 +542,21 @@ __device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk
     for (int q = 0; q < 4; ++q) c[q] = cvt_words(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], inv);
     return;
   }
-  const float S = __uint_as_float(e >= -126 ? (uint32_t)(e + 127) << 23 : 0x00400000u);
-#pragma unroll
-  for (int q = 0; q < 4; ++q) c[q] = 0u;
+  // stochastic rounding on the exact quotient y = |x| * 2^-e
+  const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+  float v[32];
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
     const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
     const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-    const uint32_t m3 = sr_m3_exact(ax, S, philox_w0((uint64_t)blk * 32u + k, seed) >> 8);
-    c[k >> 3] |= (((h >> 15) << 3) | m3) << (4 * (k & 7));
+    bool amb;
+    const float val = sr_pick(__fmul_rn(ax, inv), philox_w0((uint64_t)blk * 32u + k, seed) >> 8, false, amb);
+    v[k] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
   }
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    c[q] = cvt_e2m1x8(v[8 * q], v[8 * q + 1], v[8 * q + 2], v[8 * q + 3], v[8 * q + 4], v[8 * q + 5],
+                      v[8 * q + 6], v[8 * q + 7]);
 }
 
 __device__ __forceinline__ void report_bad(bool bad, int32_t* status) {
@@ -548,16 +582,8 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
     float st = 0.0f;
     if constexpr (FMT == TF4_NVFP4) {
       st = a.st_from_amax ? tensor_scale(a.st_src[s], nullptr) : a.st_src[s];
-      if (MODE != kSR) {
-        build_tables<true>(st, tb);
-      } else {
-        __syncthreads();
-        if (tid == 0) {
-          tb.fast = 0;
-          tb.rz = 0;
-        }
-        __syncthreads();
-      }
+      if (MODE != kSR) build_tables<true>(st, tb);
+      else build_tables<false, true>(st, tb);
     }
     const int64_t n = hi - lo;
     for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
@@ -766,44 +792,49 @@ struct DequantArgs {
   int64_t nblocks;
 };
 
+// Work unit = one quad of 4 consecutive elements (2 code bytes in, one
+// 16-byte float4 out), consecutive lanes on consecutive quads, so every warp
+// store covers 512 contiguous bytes.  Segment pieces are whole blocks.
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
   constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;
+  constexpr int QPB = BE / 4;  // quads per block
+  constexpr int U = 4;         // quads per lane per iteration
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   const int tid = threadIdx.x;
+  const uint16_t* codes2 = reinterpret_cast<const uint16_t*>(a.codes);
   int64_t lo = b0;
   while (lo < b1) {
     const int s = seg.find(lo);
     const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
     const float st = FMT == TF4_NVFP4 ? a.s_t[s] : 0.0f;
-    for (int64_t blk = lo + tid; blk < hi; blk += kThreads) {
-      const uint32_t sc = a.scales[blk];
-      float S;
-      if constexpr (FMT == TF4_NVFP4) S = __fmul_rn(st, e4m3_decode(sc));
-      else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
-      uint32_t cw[BE / 8];
-      if constexpr (FMT == TF4_NVFP4) {
-        const uint2 v = __ldg(reinterpret_cast<const uint2*>(a.codes) + blk);
-        cw[0] = v.x; cw[1] = v.y;
-      } else {
-        const uint4 v = __ldg(reinterpret_cast<const uint4*>(a.codes) + blk);
-        cw[0] = v.x; cw[1] = v.y; cw[2] = v.z; cw[3] = v.w;
+    const int64_t q0 = lo * QPB, q1 = hi * QPB;
+    for (int64_t qb = q0; qb < q1; qb += (int64_t)U * kThreads) {
+      uint32_t cw[U], sc[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t q = qb + u * kThreads + tid;
+        if (q < q1) {
+          cw[u] = __ldg(codes2 + q);
+          sc[u] = __ldg(a.scales + q / QPB);
+        }
       }
 #pragma unroll
-      for (int q = 0; q < BE / 8; ++q) {
-        uint32_t h[4];
-        e2m1x8_to_half(cw[q], h);
-        float f[8];
+      for (int u = 0; u < U; ++u) {
+        const int64_t q = qb + u * kThreads + tid;
+        if (q < q1) {
+          float S;
+          if constexpr (FMT == TF4_NVFP4) S = __fmul_rn(st, e4m3_decode(sc[u]));
+          else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
+          float v[4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-          const float2 t = __half22float2(*reinterpret_cast<const __half2*>(&h[p]));
-          f[2 * p] = __fmul_rn(t.x, S);
-          f[2 * p + 1] = __fmul_rn(t.y, S);
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t nib = (cw[u] >> (4 * e)) & 0xFu;
+            v[e] = __uint_as_float(__float_as_uint(e2m1_value(nib & 7u)) | ((nib & 8u) << 28));
+          }
+          a.out[q] = make_float4(__fmul_rn(v[0], S), __fmul_rn(v[1], S), __fmul_rn(v[2], S), __fmul_rn(v[3], S));
         }
-        float4* o = a.out + (blk * BE + q * 8) / 4;
-        o[0] = make_float4(f[0], f[1], f[2], f[3]);
-        o[1] = make_float4(f[4], f[5], f[6], f[7]);
       }
     }
     lo = hi;
@@ -815,12 +846,24 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
 // unit (16 elements, when rows*cols % 32 == 16) is done by the last thread.
 __global__ void __launch_bounds__(kThreads) k_pack(const uint8_t* __restrict__ codes, uint8_t* bits,
                                                    int64_t nunits, int tail) {
+  constexpr int U = 4;
   const int64_t u0 = cta_begin(blockIdx.x, gridDim.x, nunits);
   const int64_t u1 = cta_begin(blockIdx.x + 1, gridDim.x, nunits);
-  for (int64_t u = u0 + threadIdx.x; u < u1; u += kThreads) {
-    const uint4 c = __ldg(reinterpret_cast<const uint4*>(codes) + u);
-    reinterpret_cast<uint32_t*>(bits)[u] = nibble_lsbs(c.x) | (nibble_lsbs(c.y) << 8) |
-                                           (nibble_lsbs(c.z) << 16) | (nibble_lsbs(c.w) << 24);
+  const uint4* c4 = reinterpret_cast<const uint4*>(codes);
+  for (int64_t ub = u0; ub < u1; ub += (int64_t)U * kThreads) {
+    uint4 c[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int64_t u = ub + k * kThreads + threadIdx.x;
+      if (u < u1) c[k] = __ldg(c4 + u);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int64_t u = ub + k * kThreads + threadIdx.x;
+      if (u < u1)
+        reinterpret_cast<uint32_t*>(bits)[u] = nibble_lsbs(c[k].x) | (nibble_lsbs(c[k].y) << 8) |
+                                               (nibble_lsbs(c[k].z) << 16) | (nibble_lsbs(c[k].w) << 24);
+    }
   }
   if (tail && blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
     const uint2 c = *reinterpret_cast<const uint2*>(codes + 16 * nunits);
@@ -839,23 +882,30 @@ __device__ __forceinline__ uint2 spread8(uint32_t b) {
   return make_uint2(o[0], o[1]);
 }
 
-// Units of 32 elements: 4 guidance bytes -> 32 bytes of 0/1.
+// Units of 16 elements: 2 guidance bytes -> 16 bytes of 0/1; consecutive
+// lanes on consecutive units, so every warp store covers 512 contiguous bytes.
 __global__ void __launch_bounds__(kThreads) k_unpack(const uint8_t* __restrict__ bits, uint8_t* mant,
-                                                     int64_t nunits, int tail) {
+                                                     int64_t nunits) {
+  constexpr int U = 4;
   const int64_t u0 = cta_begin(blockIdx.x, gridDim.x, nunits);
   const int64_t u1 = cta_begin(blockIdx.x + 1, gridDim.x, nunits);
+  const uint16_t* b2 = reinterpret_cast<const uint16_t*>(bits);
   uint4* out = reinterpret_cast<uint4*>(mant);
-  for (int64_t u = u0 + threadIdx.x; u < u1; u += kThreads) {
-    const uint32_t b = __ldg(reinterpret_cast<const uint32_t*>(bits) + u);
-    const uint2 a0 = spread8(b & 0xFFu), a1 = spread8((b >> 8) & 0xFFu);
-    const uint2 a2 = spread8((b >> 16) & 0xFFu), a3 = spread8(b >> 24);
-    out[2 * u] = make_uint4(a0.x, a0.y, a1.x, a1.y);
-    out[2 * u + 1] = make_uint4(a2.x, a2.y, a3.x, a3.y);
-  }
-  if (tail && blockIdx.x == gridDim.x - 1 && threadIdx.x == 0) {
-    const uint32_t b = reinterpret_cast<const uint16_t*>(bits)[2 * nunits];
-    const uint2 a0 = spread8(b & 0xFFu), a1 = spread8(b >> 8);
-    out[2 * nunits] = make_uint4(a0.x, a0.y, a1.x, a1.y);
+  for (int64_t ub = u0; ub < u1; ub += (int64_t)U * kThreads) {
+    uint32_t b[U];
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int64_t u = ub + k * kThreads + threadIdx.x;
+      if (u < u1) b[k] = __ldg(b2 + u);
+    }
+#pragma unroll
+    for (int k = 0; k < U; ++k) {
+      const int64_t u = ub + k * kThreads + threadIdx.x;
+      if (u < u1) {
+        const uint2 lo = spread8(b[k] & 0xFFu), hi = spread8(b[k] >> 8);
+        out[u] = make_uint4(lo.x, lo.y, hi.x, hi.y);
+      }
+    }
   }
 }
 

@@ -383,10 +383,9 @@ tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_
   if (sh.n == 0) return TF4_OK;
   if (!bits || !mant) return TF4_ERR_INVALID_ARG;
   if (!aligned(bits, 4) || !aligned(mant, 16)) return TF4_ERR_ALIGN;
-  const int64_t units = sh.n / 32;
-  const int tail = (sh.n % 32) != 0;
-  const int64_t g = wave_grid(tf4::k_unpack, units > 0 ? units : 1);
-  tf4::k_unpack<<<(unsigned)g, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(bits, mant, units, tail);
+  const int64_t units = sh.n / 16;  // rows*cols is a multiple of 16
+  const int64_t g = wave_grid(tf4::k_unpack, units);
+  tf4::k_unpack<<<(unsigned)g, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(bits, mant, units);
   return launched();
 }
 

@@ -85,6 +85,15 @@ def test_sr_parity(fmt, seed):
     check_quant(xb, fmt, O.SR, seed=seed)
 
 
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+def test_sr_full_compare_16m(fmt):
+    """Every element of a 16.8M-element SR call against the oracle: enough
+    elements for ~80 uniforms to fall within the fast path's safety margin
+    of their threshold, which then takes the exact comparison."""
+    xb = W.random_bf16((4096, 4096), seed=77, device=DEV, outlier_frac=0.001)
+    check_quant(xb, fmt, O.SR, seed=2**35 + 17)
+
+
 def test_rtn_equals_capture_without_guidance():
     xb = W.random_bf16((64, 512), seed=3, device=DEV)
     a = B.tf4_quantize_rtn(xb)
