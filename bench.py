@@ -506,6 +506,9 @@ CALL_BYTES = {
     ("mxfp4", "rtn"): 2.53125, ("mxfp4", "sr"): 2.53125, ("mxfp4", "capture"): 2.65625,
     ("mxfp4", "guided"): 2.65625, ("mxfp4", "dequant"): 4.53125,
     ("any", "pack"): 0.625, ("any", "unpack"): 1.125,
+    ("nvfp4", "guided_fq_f32"): 6.1875, ("nvfp4", "guided_fq_bf16"): 4.1875,
+    ("mxfp4", "guided_fq_f32"): 6.15625, ("mxfp4", "guided_fq_bf16"): 4.15625,
+    ("nvfp4", "mismatch"): 2.5625, ("mxfp4", "mismatch"): 2.53125,
 }
 
 
@@ -533,10 +536,22 @@ def run_suite(args):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / reps * 1e3  # us
 
-    def record(workload, fmt, call, n, us):
+    def record(workload, fmt, call, n, us, **extra):
         gbs = CALL_BYTES[(fmt, call)] * n / (us * 1e-6) / 1e9
         rows_out.append(dict(workload=workload, format=fmt, call=call, elements=n, us=round(us, 2),
-                             gbs=round(gbs, 1), frac=round(gbs / peak, 4)))
+                             gbs=round(gbs, 1), frac=round(gbs / peak, 4), **extra))
+
+    def fq_and_diag(name, fmt, q, x, xt):
+        n = x.numel()
+        yf = torch.empty(x.shape, dtype=torch.float32, device=dev)
+        yb = torch.empty(x.shape, dtype=torch.bfloat16, device=dev)
+        record(name, fmt, "guided_fq_f32", n, timed(lambda: B.tf4_guided_fake_quant(xt, q, out=yf)))
+        record(name, fmt, "guided_fq_bf16", n, timed(lambda: B.tf4_guided_fake_quant(xt, q, out=yb)))
+        cnt = torch.zeros(4, dtype=torch.int64, device=dev)
+        us = timed(lambda: B.tf4_mismatch_stats(xt, q, counts=cnt.zero_()))
+        c = [int(v) for v in B.tf4_mismatch_stats(xt, q).tolist()]
+        record(name, fmt, "mismatch", n, us, counts=dict(mismatch=c[0], adjacent=c[1], far=c[2], after_guidance=c[3]),
+               adjacent_fraction=(round(c[1] / c[0], 6) if c[0] else None))
 
     def nv_calls(name, x, xt, seg=None):
         n = x.numel()
@@ -556,6 +571,7 @@ def run_suite(args):
         rows, cols = x.shape
         record(name, "any", "pack", n, timed(lambda: B.tf4_pack_guidance(q.codes, rows, cols, out=bits)))
         record(name, "any", "unpack", n, timed(lambda: B.tf4_unpack_guidance(bits, rows, cols, out=mant)))
+        fq_and_diag(name, "nvfp4", q, x, xt)
         del q, g, out, bits, mant, qr
 
     def mx_calls(name, x, xt):
@@ -571,6 +587,7 @@ def run_suite(args):
         record(name, "mxfp4", "guided", n, timed(lambda: B.tf4_quantize_guided(xt, q, out=g)))
         record(name, "mxfp4", "sr", n, timed(lambda: B.tf4_quantize_sr(x, 4, fmt=B.MXFP4, out=qr)))
         record(name, "mxfp4", "dequant", n, timed(lambda: B.tf4_dequantize(q, out=out)))
+        fq_and_diag(name, "mxfp4", q, x, xt)
         del q, g, out, qr
 
     w = W.activation_outliers(dev)

@@ -40,7 +40,7 @@ EXPORTS = (
     "tf4_workspace_bytes", "tf4_codes_bytes", "tf4_scales_bytes", "tf4_guidance_bytes",
     "tf4_record_bytes", "tf4_segment_amax", "tf4_quantize_rtn", "tf4_quantize_sr",
     "tf4_quantize_capture", "tf4_quantize_guided", "tf4_dequantize", "tf4_pack_guidance",
-    "tf4_unpack_guidance", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
+    "tf4_unpack_guidance", "tf4_guided_fake_quant", "tf4_mismatch_stats", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
     "tf4_version",
 )
 
@@ -93,6 +93,8 @@ def lib():
                     "tf4_pack_guidance": (st, [dp, vp, vp, vp]),
                     "tf4_unpack_guidance": (st, [dp, vp, vp, vp]),
                     "tf4_quantize_capture_noalloc": (st, [dp, vp, vp, vp, vp, vp, i32p, vp]),
+                    "tf4_guided_fake_quant": (st, [dp, vp, vp, vp, vp, vp, vp, ctypes.c_int, i32p, vp]),
+                    "tf4_mismatch_stats": (st, [dp, vp, vp, vp, vp, vp, i32p, vp]),
                     "tf4_read_status": (st, [i32p, vp]),
                     "tf4_status_string": (ctypes.c_char_p, [st]),
                     "tf4_version": (ctypes.c_int, []),
@@ -279,6 +281,38 @@ def tf4_quantize_guided(x, rec: Quantized, stream=None, out=None, rec_bits=None)
     _check(lib().tf4_quantize_guided(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(bits), _ptr(codes),
                                      _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_quantize_guided")
     return codes
+
+
+def tf4_guided_fake_quant(x, rec: Quantized, out_dtype=torch.float32, want_codes=False, stream=None,
+                          out=None, codes=None, rec_bits=None):
+    """Guided quantization + dequantization in one pass.  Returns (values,
+    codes): values [rows, cols] in out_dtype (float32, or bfloat16 = RNE of
+    the fp32 value); codes only if want_codes (else None)."""
+    assert out_dtype in (torch.float32, torch.bfloat16)
+    x2 = _as_2d(x)
+    d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
+    bits = rec_bits if rec_bits is not None else rec.bits
+    assert bits is not None, "the record holds no guidance bits"
+    o = out if out is not None else torch.empty(x2.shape, dtype=out_dtype, device=x.device)
+    c = codes if codes is not None else (
+        torch.empty(d.n // 2, dtype=torch.uint8, device=x.device) if want_codes else None)
+    _check(lib().tf4_guided_fake_quant(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(bits), _ptr(c),
+                                       _ptr(o), 1 if o.dtype == torch.bfloat16 else 0,
+                                       _ptr(status_word(x.device)), _stream(stream, x.device)),
+           "tf4_guided_fake_quant")
+    return o, c
+
+
+def tf4_mismatch_stats(x, rec: Quantized, counts=None, stream=None) -> torch.Tensor:
+    """Mismatch diagnostics of train values x against a rollout record
+    (codes + scales): adds [#mismatch, #adjacent, #far, #after-guidance] to
+    `counts` (int64 [4], zero-initialised if not given) and returns it."""
+    x2 = _as_2d(x)
+    d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
+    c = counts if counts is not None else torch.zeros(4, dtype=torch.int64, device=x.device)
+    _check(lib().tf4_mismatch_stats(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(rec.codes), _ptr(c),
+                                    _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_mismatch_stats")
+    return c
 
 
 def tf4_dequantize(q: Quantized, codes=None, stream=None, out=None) -> torch.Tensor:

@@ -12,7 +12,9 @@
 // exact definition.
 #pragma once
 
+#include <cuda_bf16.h>
 #include <cuda_fp16.h>
+#include <cuda_fp4.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -91,6 +93,17 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float v0, float v1, float v2, flo
       : "=r"(r)
       : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
   return r;
+}
+
+// Four E2M1 nibbles (16 bits, element k in bits [4k, 4k+4)) -> their values
+// times S, using CUDA's fp4x2 -> half2 conversion (exact: every E2M1 value
+// is an f16 value) and one fp32 multiply each.
+__device__ __forceinline__ float4 decode4(uint32_t c, float S) {
+  const __half2_raw h0 = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)(c & 0xFFu), __NV_E2M1);
+  const __half2_raw h1 = __nv_cvt_fp4x2_to_halfraw2((__nv_fp4x2_storage_t)((c >> 8) & 0xFFu), __NV_E2M1);
+  const float2 f0 = __half22float2(__half2(h0));
+  const float2 f1 = __half22float2(__half2(h1));
+  return make_float4(__fmul_rn(f0.x, S), __fmul_rn(f0.y, S), __fmul_rn(f1.x, S), __fmul_rn(f1.y, S));
 }
 
 // m3 & 1 of eight nibbles -> eight bits (nibble k -> bit k).
@@ -783,6 +796,203 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
   }
 }
 
+// --------------------------------------------- fused guided fake-quant
+// Train-side forward in one pass: guided quantization of x against the
+// rollout record, then dequantization of the chosen codes, written as fp32
+// or as bf16 (round-to-nearest-even of the fp32 value), and optionally the
+// codes.  Work unit = a quad of 4 consecutive elements (8 B of x in), so
+// consecutive lanes write consecutive 16-B (fp32) / 8-B (bf16) outputs.
+struct GuidedFqArgs {
+  const uint2* x;         // bf16 quads
+  int64_t nblocks;
+  const uint8_t* rec_scales;
+  const float* rec_s_t;
+  const uint8_t* rec_bits;
+  uint8_t* codes;         // may be NULL
+  void* out;              // float4 (fp32) or uint2 (bf16) per quad
+  int32_t* status;
+};
+
+// Four bf16 (two words) times r -> four E2M1 nibbles (16 bits).
+template <bool RZ>
+__device__ __forceinline__ uint32_t cvt_words4(uint32_t w0, uint32_t w1, float r) {
+  uint32_t c;
+  asm("{\n\t.reg .b8 q0, q1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "mov.b32 %0, {q0, q1, q1, q1};\n\t}"
+      : "=r"(c)
+      : "f"(mul<RZ>(bf_lo(w0), r)), "f"(mul<RZ>(bf_hi(w0), r)), "f"(mul<RZ>(bf_lo(w1), r)),
+        "f"(mul<RZ>(bf_hi(w1), r)));
+  return c & 0xFFFFu;
+}
+
+template <int FMT, class SEG, bool BF16>
+__global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg) {
+  constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;
+  constexpr int QPB = BE / 4;  // quads per block
+  constexpr int U = 2;         // quads per lane per iteration
+  __shared__ SegTables tb;
+  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
+  const int tid = threadIdx.x;
+  int64_t lo = b0;
+  while (lo < b1) {
+    const int s = seg.find(lo);
+    const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
+    float st = 0.0f;
+    if constexpr (FMT == TF4_NVFP4) {
+      st = a.rec_s_t[s];
+      build_tables<false>(st, tb);
+    }
+    const int64_t q0 = lo * QPB, q1 = hi * QPB;
+    for (int64_t qb = q0; qb < q1; qb += (int64_t)U * kThreads) {
+      uint2 xv[U];
+      uint32_t sc[U], gq[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t q = qb + u * kThreads + tid;
+        if (q < q1) {
+          xv[u] = __ldg(a.x + q);
+          sc[u] = __ldg(a.rec_scales + q / QPB);
+          gq[u] = (__ldg(a.rec_bits + (q >> 1)) >> (4 * (q & 1))) & 0xFu;  // 4 bits of this quad
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t q = qb + u * kThreads + tid;
+        bool bad = false;
+        if (q < q1) {
+          const uint32_t m = vmax_u16x2(xv[u].x & 0x7FFF7FFFu, xv[u].y & 0x7FFF7FFFu);
+          bad = max(m & 0xFFFFu, m >> 16) >= 0x7F80u;
+          float r = 0.0f, S;
+          bool rz = false;
+          if constexpr (FMT == TF4_NVFP4) {
+            S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
+            if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu && tb.rho[sc[u] & 7u] != 0.0f) {
+              r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
+              rz = tb.rz;
+            }
+          } else {
+            S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
+            if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);
+          }
+          const uint32_t w0 = xv[u].x, w1 = xv[u].y;
+          uint32_t c;
+          if (r != 0.0f) {
+            c = rz ? cvt_words4<true>(w0, w1, r) : cvt_words4<false>(w0, w1, r);
+            const uint32_t mm = (c ^ spread_bits(gq[u])) & 0x1111u;
+            if (mm)
+              c = rz ? fix_mismatches<true>(c, mm, w0, w1, 0u, 0u, r) : fix_mismatches<false>(c, mm, w0, w1, 0u, 0u, r);
+          } else {
+            c = 0u;
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const uint32_t h = (e & 1) ? ((e & 2 ? w1 : w0) >> 16) : ((e & 2 ? w1 : w0) & 0xFFFFu);
+              const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+              const uint32_t m3 = S > 0.0f ? guided_m3_exact(ax, S, (gq[u] >> e) & 1u) : 0u;
+              c |= (((h >> 15) << 3) | m3) << (4 * e);
+            }
+          }
+          if (a.codes) reinterpret_cast<uint16_t*>(a.codes)[q] = (uint16_t)c;
+          const float4 v = decode4(c, S);
+          if constexpr (BF16) {
+            const __nv_bfloat162 p0 = __floats2bfloat162_rn(v.x, v.y), p1 = __floats2bfloat162_rn(v.z, v.w);
+            reinterpret_cast<uint2*>(a.out)[q] =
+                make_uint2(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1));
+          } else {
+            reinterpret_cast<float4*>(a.out)[q] = v;
+          }
+        }
+        report_bad(bad, a.status);
+      }
+    }
+    lo = hi;
+  }
+}
+
+// ------------------------------------------------ mismatch diagnostics
+// Train/rollout mismatch statistics (TRACE summary, section
+// "量子化情報キャッシュ": more than 99% of mismatches are between adjacent
+// codewords).  For each element, with the rollout's recorded scale: n_r =
+// nearest rounding of the train value, n_o = the rollout code, n_g = the
+// guided code (recorded bit = n_o's mantissa bit); codes compare by signed
+// grid index (sign ? -m3 : m3, so +0 and -0 are equal).  Accumulates
+// counts[0] += #(n_r != n_o), counts[1] += #(|n_r - n_o| == 1),
+// counts[2] += #(|n_r - n_o| >= 2), counts[3] += #(n_g != n_o).
+// Exact per-element comparisons (a diagnostic; not on the hot path).
+struct MismatchArgs {
+  const uint4* x;
+  int64_t nblocks;
+  const uint8_t* rec_scales;
+  const float* rec_s_t;
+  const uint8_t* rec_codes;
+  unsigned long long* counts;
+  int32_t* status;
+};
+
+__device__ __forceinline__ int grid_index(uint32_t nib) {
+  const int m = (int)(nib & 7u);
+  return (nib & 8u) ? -m : m;
+}
+
+template <int FMT, class SEG>
+__global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) {
+  constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;
+  constexpr int NW = BE / 2;
+  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
+  uint32_t cnt[4] = {0u, 0u, 0u, 0u};
+  int64_t lo = b0;
+  bool bad = false;
+  while (lo < b1) {
+    const int s = seg.find(lo);
+    const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
+    const float st = FMT == TF4_NVFP4 ? a.rec_s_t[s] : 0.0f;
+    for (int64_t blk = lo + threadIdx.x; blk < hi; blk += kThreads) {
+      uint32_t w[NW], cw[BE / 8];
+#pragma unroll
+      for (int q = 0; q < NW / 4; ++q) {
+        const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
+        w[4 * q] = p.x; w[4 * q + 1] = p.y; w[4 * q + 2] = p.z; w[4 * q + 3] = p.w;
+      }
+      if constexpr (FMT == TF4_NVFP4) {
+        const uint2 c = __ldg(reinterpret_cast<const uint2*>(a.rec_codes) + blk);
+        cw[0] = c.x; cw[1] = c.y;
+      } else {
+        const uint4 c = __ldg(reinterpret_cast<const uint4*>(a.rec_codes) + blk);
+        cw[0] = c.x; cw[1] = c.y; cw[2] = c.z; cw[3] = c.w;
+      }
+      const uint32_t sc = a.rec_scales[blk];
+      float S;
+      if constexpr (FMT == TF4_NVFP4) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
+      else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
+      bad |= block_absmax_bits(w) >= 0x7F80u;
+#pragma unroll
+      for (int e = 0; e < BE; ++e) {
+        const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+        const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+        const uint32_t no = (cw[e >> 3] >> (4 * (e & 7))) & 0xFu;
+        const uint32_t sg = (h >> 15) << 3;
+        const uint32_t nr = sg | (S > 0.0f ? rtn_m3_exact(ax, S) : 0u);
+        const uint32_t ng = sg | (S > 0.0f ? guided_m3_exact(ax, S, no & 1u) : 0u);
+        const int d = abs(grid_index(nr) - grid_index(no));
+        cnt[0] += d != 0;
+        cnt[1] += d == 1;
+        cnt[2] += d >= 2;
+        cnt[3] += grid_index(ng) != grid_index(no);
+      }
+    }
+    lo = hi;
+  }
+  report_bad(bad, a.status);
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t t = __reduce_add_sync(0xFFFFFFFFu, cnt[k]);
+    if ((threadIdx.x & 31) == 0 && t) atomicAdd(a.counts + k, (unsigned long long)t);
+  }
+}
+
 // ---------------------------------------------------------- dequantize
 struct DequantArgs {
   const uint8_t* codes;
@@ -827,13 +1037,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
           float S;
           if constexpr (FMT == TF4_NVFP4) S = __fmul_rn(st, e4m3_decode(sc[u]));
           else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
-          float v[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t nib = (cw[u] >> (4 * e)) & 0xFu;
-            v[e] = __uint_as_float(__float_as_uint(e2m1_value(nib & 7u)) | ((nib & 8u) << 28));
-          }
-          a.out[q] = make_float4(__fmul_rn(v[0], S), __fmul_rn(v[1], S), __fmul_rn(v[2], S), __fmul_rn(v[3], S));
+          a.out[q] = decode4(cw[u], S);
         }
       }
     }

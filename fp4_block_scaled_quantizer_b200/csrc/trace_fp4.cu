@@ -331,6 +331,82 @@ tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_
   return launched();
 }
 
+tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint8_t* rec_scales,
+                                 const float* rec_s_t, const uint8_t* rec_bits, uint8_t* codes, void* out,
+                                 int out_bf16, int32_t* status, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.n == 0) return TF4_OK;
+  const bool nv = sh.fmt == TF4_NVFP4;
+  if (!x || !rec_scales || !rec_bits || !out || (nv && !rec_s_t)) return TF4_ERR_INVALID_ARG;
+  if (out_bf16 != 0 && out_bf16 != 1) return TF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(out, 16) || !aligned(rec_bits, 4) || (codes && !aligned(codes, 16)) ||
+      (nv && !aligned(rec_s_t, 4)) || (status && !aligned(status, 4)))
+    return TF4_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tf4::GuidedFqArgs a;
+  a.x = static_cast<const uint2*>(x);
+  a.nblocks = sh.nblocks;
+  a.rec_scales = rec_scales;
+  a.rec_s_t = rec_s_t;
+  a.rec_bits = rec_bits;
+  a.codes = codes;
+  a.out = out;
+  a.status = status;
+#define TF4_LAUNCH_FQ(FMT, SEG, BF, segv)                                             \
+  do {                                                                                \
+    const int64_t g = wave_grid(tf4::k_guided_fq<FMT, SEG, BF>, sh.nblocks);          \
+    tf4::k_guided_fq<FMT, SEG, BF><<<(unsigned)g, kThreads, 0, st>>>(a, segv);        \
+  } while (0)
+  if (nv && multi(sh)) {
+    if (out_bf16) TF4_LAUNCH_FQ(TF4_NVFP4, tf4::SegN, true, make_segn(sh));
+    else TF4_LAUNCH_FQ(TF4_NVFP4, tf4::SegN, false, make_segn(sh));
+  } else if (nv) {
+    if (out_bf16) TF4_LAUNCH_FQ(TF4_NVFP4, tf4::Seg1, true, tf4::Seg1{});
+    else TF4_LAUNCH_FQ(TF4_NVFP4, tf4::Seg1, false, tf4::Seg1{});
+  } else {
+    if (out_bf16) TF4_LAUNCH_FQ(TF4_MXFP4, tf4::Seg1, true, tf4::Seg1{});
+    else TF4_LAUNCH_FQ(TF4_MXFP4, tf4::Seg1, false, tf4::Seg1{});
+  }
+#undef TF4_LAUNCH_FQ
+  return launched();
+}
+
+tf4_status tf4_mismatch_stats(const tf4_desc* desc, const void* x, const uint8_t* rec_scales, const float* rec_s_t,
+                              const uint8_t* rec_codes, unsigned long long* counts, int32_t* status,
+                              tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (!counts) return TF4_ERR_INVALID_ARG;
+  if (!aligned(counts, 8) || (status && !aligned(status, 4))) return TF4_ERR_ALIGN;
+  if (sh.n == 0) return TF4_OK;
+  const bool nv = sh.fmt == TF4_NVFP4;
+  if (!x || !rec_scales || !rec_codes || (nv && !rec_s_t)) return TF4_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(rec_codes, 16) || (nv && !aligned(rec_s_t, 4))) return TF4_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  tf4::MismatchArgs a;
+  a.x = static_cast<const uint4*>(x);
+  a.nblocks = sh.nblocks;
+  a.rec_scales = rec_scales;
+  a.rec_s_t = rec_s_t;
+  a.rec_codes = rec_codes;
+  a.counts = counts;
+  a.status = status;
+  if (nv && multi(sh)) {
+    const int64_t g = wave_grid(tf4::k_mismatch<TF4_NVFP4, tf4::SegN>, sh.nblocks);
+    tf4::k_mismatch<TF4_NVFP4, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+  } else if (nv) {
+    const int64_t g = wave_grid(tf4::k_mismatch<TF4_NVFP4, tf4::Seg1>, sh.nblocks);
+    tf4::k_mismatch<TF4_NVFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  } else {
+    const int64_t g = wave_grid(tf4::k_mismatch<TF4_MXFP4, tf4::Seg1>, sh.nblocks);
+    tf4::k_mismatch<TF4_MXFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  }
+  return launched();
+}
+
 tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint8_t* scales, const float* s_t,
                           float* out, tf4_stream_t stream) {
   Shape sh;

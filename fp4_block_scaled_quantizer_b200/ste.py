@@ -6,7 +6,8 @@ gradient through unchanged (straight-through estimator) -- TRACE summary
 (ai-papers.net), section "TRACEの仕組み": the gradient flows through the
 chosen quantized value as if rounding were the identity.
 
-Forward = one quantize kernel + one dequantize kernel of the CUDA library;
+Forward = one kernel of the CUDA library (guided: the fused
+quantize-dequantize pass; nearest / stochastic: quantize + dequantize);
 backward = no kernel (the same gradient tensor is returned when its dtype
 matches the input's).
 """
@@ -27,8 +28,11 @@ class GuidedFakeQuant(torch.autograd.Function):
     @staticmethod
     def forward(ctx, x: torch.Tensor, rec: B.Quantized, out_dtype=torch.float32):
         ctx.in_dtype = x.dtype
-        codes = B.tf4_quantize_guided(x, rec)
-        return B.tf4_dequantize(rec, codes=codes).reshape(x.shape).to(out_dtype)
+        if out_dtype in (torch.float32, torch.bfloat16):
+            y, _ = B.tf4_guided_fake_quant(x, rec, out_dtype=out_dtype)
+            return y.reshape(x.shape)
+        y, _ = B.tf4_guided_fake_quant(x, rec)
+        return y.reshape(x.shape).to(out_dtype)
 
     @staticmethod
     def backward(ctx, grad_out):

@@ -160,6 +160,32 @@ tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_
                                const float* rec_s_t, const uint8_t* rec_bits, uint8_t* codes,
                                int32_t* dev_status, tf4_stream_t stream);
 
+/* Train-side fake quantization in one pass (the trainer's forward value of
+ * the TRACE summary's "mechanism" section: the guided codeword, through
+ * which the straight-through gradient flows): tf4_quantize_guided followed
+ * by tf4_dequantize, without writing and re-reading the codes.  out
+ * receives the dequantized values [rows, cols] as fp32 (out_bf16 = 0) or as
+ * bf16, the round-to-nearest-even of that fp32 value (out_bf16 = 1);
+ * codes (may be NULL) receives the guided codes.  Alignment: x, out and
+ * codes 16 bytes, rec_bits and rec_s_t 4 bytes. */
+tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint8_t* rec_scales,
+                                 const float* rec_s_t, const uint8_t* rec_bits, uint8_t* codes,
+                                 void* out, int out_bf16, int32_t* dev_status, tf4_stream_t stream);
+
+/* Train/rollout mismatch diagnostics (TRACE summary, section
+ * "量子化情報キャッシュ": more than 99% of mismatches fall between adjacent
+ * codewords, which is why one mantissa bit suffices).  For each element of
+ * the train value x, with the rollout's recorded scale bytes / s_t: n_r =
+ * nearest rounding of x, n_o = the rollout code (rec_codes), n_g = the
+ * guided code (recorded bit = mantissa bit of n_o).  Codes compare by signed
+ * grid index (sign ? -m3 : m3; +0 == -0).  ADDS to counts (device, 4 x
+ * uint64, 8-byte aligned; the caller zeroes it):
+ *   counts[0] elements with n_r != n_o, counts[1] with |n_r - n_o| == 1,
+ *   counts[2] with |n_r - n_o| >= 2, counts[3] with n_g != n_o. */
+tf4_status tf4_mismatch_stats(const tf4_desc* desc, const void* x, const uint8_t* rec_scales,
+                              const float* rec_s_t, const uint8_t* rec_codes,
+                              unsigned long long* counts, int32_t* dev_status, tf4_stream_t stream);
+
 /* out[i] = (-1)^sign * fl32(V[m3] * S) as fp32 [rows, cols]. */
 tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint8_t* scales,
                           const float* s_t, float* out, tf4_stream_t stream);

@@ -59,6 +59,10 @@ def lib():
                                            f32p]),
             "orc_pack_guidance": (None, [u8p, i64, u8p]),
             "orc_unpack_guidance": (None, [u8p, i64, u8p]),
+            "orc_rtn_with_scales_rows": (None, [ctypes.c_int, u16p, i64, i64, i32, i64p, u8p, f32p, i64, i64,
+                                                u8p]),
+            "orc_f32_to_bf16": (ctypes.c_uint16, [ctypes.c_float]),
+            "orc_f32_to_bf16_array": (None, [f32p, i64, u16p]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -220,3 +224,53 @@ def unpack_codes(codes, n):
     out[0::2] = c & 0xF
     out[1::2] = c >> 4
     return out[:n]
+
+
+def f32_to_bf16(v):
+    """bf16 bit patterns (RNE) of an fp32 array."""
+    a = np.ascontiguousarray(v, dtype=np.float32).reshape(-1)
+    out = np.zeros(a.size, dtype=np.uint16)
+    lib().orc_f32_to_bf16_array(_p(a, ctypes.c_float), a.size, _p(out, ctypes.c_uint16))
+    return out.reshape(np.shape(v))
+
+
+def guided_fake_quant(x, rec_scales, rec_bits, fmt=NVFP4, rec_s_t=None, seg_off=None):
+    """Train-side fake quantization: guided codes, then their fp32 values."""
+    rows, cols = np.shape(x)
+    codes, status = quantize_guided(x, rec_scales, rec_bits, fmt, rec_s_t=rec_s_t, seg_off=seg_off)
+    return codes, dequantize(codes, rec_scales, rows, cols, fmt, s_t=rec_s_t, seg_off=seg_off), status
+
+
+def rtn_with_scales(x, scales, fmt=NVFP4, s_t=None, seg_off=None):
+    """Nearest rounding of x on a given (recorded) grid of scales."""
+    x = np.ascontiguousarray(x, dtype=np.uint16)
+    rows, cols = x.shape
+    nseg, so = _seg(seg_off, rows)
+    sc = np.ascontiguousarray(scales, dtype=np.uint8)
+    st = None if s_t is None else np.ascontiguousarray(s_t, dtype=np.float32)
+    codes = np.zeros(rows * cols // 2, dtype=np.uint8)
+    lib().orc_rtn_with_scales_rows(fmt, _p(x, ctypes.c_uint16), rows, cols, nseg, _p(so, ctypes.c_int64),
+                                   _p(sc, ctypes.c_uint8), _p(st, ctypes.c_float), 0, rows,
+                                   _p(codes, ctypes.c_uint8))
+    return codes
+
+
+def grid_index(codes, n):
+    """Signed grid index of each code (sign ? -m3 : m3)."""
+    nib = unpack_codes(codes, n).astype(np.int64)
+    m = nib & 7
+    return np.where(nib & 8, -m, m)
+
+
+def mismatch_stats(x, rec_scales, rec_codes, fmt=NVFP4, rec_s_t=None, seg_off=None):
+    """[#(n_r != n_o), #(|n_r - n_o| == 1), #(|n_r - n_o| >= 2), #(n_g != n_o)]
+    with n_r the train value's nearest rounding on the recorded grid, n_o the
+    rollout code, n_g the guided code."""
+    rows, cols = np.shape(x)
+    n = rows * cols
+    nr = rtn_with_scales(x, rec_scales, fmt, rec_s_t, seg_off)
+    bits = pack_guidance(rec_codes, n)
+    ng, _ = quantize_guided(x, rec_scales, bits, fmt, rec_s_t=rec_s_t, seg_off=seg_off)
+    io, ir, ig = grid_index(rec_codes, n), grid_index(nr, n), grid_index(ng, n)
+    d = np.abs(ir - io)
+    return np.array([(d != 0).sum(), (d == 1).sum(), (d >= 2).sum(), (ig != io).sum()], dtype=np.int64)

@@ -385,3 +385,39 @@ void orc_pack_guidance(const uint8_t* codes, int64_t n, uint8_t* bits) {
 void orc_unpack_guidance(const uint8_t* bits, int64_t n, uint8_t* mant) {
   for (int64_t i = 0; i < n; ++i) mant[i] = (uint8_t)get_bit(bits, i);
 }
+
+/* bf16 of a finite fp32 by round-to-nearest-even on the 16 dropped bits:
+ * the plain definition of the bf16 output of the train-side fake
+ * quantization (the fp32 dequantized value converted to bf16). */
+uint16_t orc_f32_to_bf16(float v) {
+  uint32_t b;
+  memcpy(&b, &v, sizeof b);
+  uint32_t lo = b & 0xFFFFu, hi = b >> 16;
+  if (lo > 0x8000u || (lo == 0x8000u && (hi & 1u))) hi += 1u;
+  return (uint16_t)hi;
+}
+
+void orc_f32_to_bf16_array(const float* v, int64_t n, uint16_t* out) {
+  for (int64_t i = 0; i < n; ++i) out[i] = orc_f32_to_bf16(v[i]);
+}
+
+/* Nearest rounding of x under GIVEN scale bytes (and s_t for NVFP4): the
+ * train value rounded on the rollout's grid (used by the mismatch
+ * diagnostics; [TRACE-JA] quantization-info cache section). */
+void orc_rtn_with_scales_rows(int fmt, const uint16_t* x, int64_t rows, int64_t cols, int32_t nseg,
+                              const int64_t* seg_off, const uint8_t* scales, const float* s_t,
+                              int64_t row_begin, int64_t row_end, uint8_t* codes) {
+  const int block = fmt == ORC_NVFP4 ? 16 : 32;
+  const int64_t nblk_row = cols / block;
+  (void)rows;
+  for (int64_t r = row_begin; r < row_end; ++r) {
+    float st = fmt == ORC_NVFP4 ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
+    for (int64_t c = 0; c < cols; ++c) {
+      const int64_t i = r * cols + c;
+      uint8_t sc = scales[r * nblk_row + c / block];
+      double S = fmt == ORC_NVFP4 ? (double)orc_nvfp4_block_scale(sc, st) : (double)orc_mxfp4_block_scale(sc);
+      uint16_t h = x[i];
+      put_code(codes, i, (bf16_sign(h) << 3) | orc_rtn_m3(bf16_abs(h), S));
+    }
+  }
+}

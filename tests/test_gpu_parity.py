@@ -256,6 +256,40 @@ def test_dequant_parity(fmt):
     assert_same("dequant", f32_bits(host(d)), f32_bits(want))
 
 
+@pytest.mark.parametrize("fmt,seg", [(O.NVFP4, None), (O.NVFP4, [0, 25, 25, 77]), (O.MXFP4, None)])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_guided_fake_quant_parity(fmt, seg, dtype):
+    """The fused train-side pass equals guided quantization followed by
+    dequantization (and, for bf16, RNE of the fp32 value), codes included."""
+    xb = W.random_bf16((77, 2048), seed=43, device=DEV, outlier_frac=0.01)
+    q, r = check_quant(xb, fmt, seg=seg)
+    xt = W.perturb(xb, 44, rel=0.05)
+    y, c = B.tf4_guided_fake_quant(xt, q, out_dtype=dtype, want_codes=True)
+    assert B.read_status(xb.device) == 0
+    codes, vals, st = O.guided_fake_quant(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"],
+                                          seg_off=seg)
+    assert_same("codes", host(c), codes)
+    if dtype == torch.float32:
+        assert_same("values", f32_bits(host(y)), f32_bits(vals))
+    else:
+        assert_same("values", host(y.view(torch.int16)).view(np.uint16), O.f32_to_bf16(vals))
+
+
+@pytest.mark.parametrize("fmt,seg", [(O.NVFP4, None), (O.NVFP4, [0, 30, 30, 64]), (O.MXFP4, None)])
+@pytest.mark.parametrize("rel", [1e-3, 0.05, None])
+def test_mismatch_stats_parity(fmt, seg, rel):
+    """Mismatch diagnostics equal the oracle's counts (None: unrelated train tensor)."""
+    xb = W.random_bf16((64, 2048), seed=51, device=DEV, outlier_frac=0.005)
+    q, r = check_quant(xb, fmt, seg=seg)
+    xt = W.perturb(xb, 52, rel=rel) if rel else W.random_bf16((64, 2048), seed=53, device=DEV)
+    c = B.tf4_mismatch_stats(xt, q)
+    assert B.read_status(xb.device) == 0
+    want = O.mismatch_stats(W.bf16_bits(xt), r["scales"], r["codes"], fmt, rec_s_t=r["s_t"], seg_off=seg)
+    assert host(c).tolist() == want.tolist()
+    if rel == 1e-3:
+        assert want[0] == want[1] + want[2]
+
+
 @pytest.mark.parametrize("shape", [(1, 16), (3, 48), (64, 1024), (5, 16 * 33)])
 def test_pack_unpack_parity(shape):
     rows, cols = shape

@@ -481,3 +481,34 @@ def test_retained_information_one_sixth():
     # the closed form generalises: MXFP4 with a 32-block
     mx = (F(1) + F(8, 32)) / (F(4) + F(8, 32)) * F(1, 2)
     assert abs(float(mx) - 0.147) < 1e-3
+
+
+def test_f32_to_bf16_vs_torch(orc):
+    """The bf16 output rounding (RNE of the fp32 value) against torch's
+    fp32 -> bf16 conversion, on random values and around every tie."""
+    rng = np.random.default_rng(9)
+    v = np.concatenate([rng.standard_normal(200000).astype(np.float32) * np.float32(1e3),
+                        (np.arange(1 << 16, dtype=np.uint32) << 16 | 0x8000).view(np.float32),
+                        (np.arange(1 << 16, dtype=np.uint32) << 16 | 0x7FFF).view(np.float32),
+                        (np.arange(1 << 16, dtype=np.uint32) << 16 | 0x8001).view(np.float32)])
+    v = v[np.isfinite(v) & (np.abs(v) < 3e38)]
+    want = torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(orc.f32_to_bf16(v), want)
+
+
+def test_mismatch_stats_closed_form(orc):
+    """Mismatch counts on constructed cases: identical inputs -> all zero; a
+    train value moved across one midpoint -> one adjacent mismatch that
+    guidance removes; moved across two codewords -> one far mismatch."""
+    x = np.zeros((1, 32), np.uint16)
+    vals = np.array([4.0, 2.4, 1.0, 0.3] + [0.0] * 28, np.float32)
+    x[0] = W.bf16_bits(torch.from_numpy(vals).to(torch.bfloat16).reshape(1, 32))[0]
+    r = orc.quantize(x, orc.MXFP4, bits=True)  # block max 4 -> S = 1
+    assert orc.mismatch_stats(x, r["scales"], r["codes"], orc.MXFP4).tolist() == [0, 0, 0, 0]
+    xt = x.copy()
+    vt = vals.copy()
+    vt[1] = 2.6   # 2.4 -> 2 (rollout), 2.6 -> 3: adjacent
+    vt[2] = 1.9   # 1.0 -> 1, 1.9 -> 2: two codewords apart (1 -> 1.5 -> 2)
+    xt[0] = W.bf16_bits(torch.from_numpy(vt).to(torch.bfloat16).reshape(1, 32))[0]
+    st = orc.mismatch_stats(xt, r["scales"], r["codes"], orc.MXFP4)
+    assert st.tolist() == [2, 1, 1, 1]
