@@ -106,13 +106,13 @@ __device__ __forceinline__ float4 decode4(uint32_t c, float S) {
   return make_float4(__fmul_rn(f0.x, S), __fmul_rn(f0.y, S), __fmul_rn(f1.x, S), __fmul_rn(f1.y, S));
 }
 
-// m3 & 1 of eight nibbles -> eight bits (nibble k -> bit k).
+// m3 & 1 of eight nibbles -> eight bits (nibble k -> bit k).  The masked
+// bits sit at 4k; multiplying by 0x1248 (= 2^3 + 2^6 + 2^9 + 2^12) sends bit
+// 4k to 12 + k for k < 4 and to 24 + k for k >= 4, and every other partial
+// product lands on a distinct position outside those bits (no carries).
 __device__ __forceinline__ uint32_t nibble_lsbs(uint32_t c) {
-  uint32_t t = c & 0x11111111u;
-  t = (t | (t >> 3)) & 0x03030303u;
-  t = (t | (t >> 6)) & 0x000F000Fu;
-  t = (t | (t >> 12)) & 0xFFu;
-  return t;
+  const uint32_t p = (c & 0x11111111u) * 0x1248u;
+  return ((p >> 12) & 0xFu) | ((p >> 24) & 0xF0u);
 }
 
 // E4M3 (fn) scale byte of a non-negative fp32 (hardware RNE, satfinite).
@@ -577,14 +577,16 @@ __device__ __forceinline__ void report_bad(bool bad, int32_t* status) {
     atomicOr(status, TF4_DEV_NONFINITE);
 }
 
-// Quantize pass.  Each CTA walks its block range backwards, so that the
-// first blocks it reads are the ones the amax pass read last (still in L2).
+// Quantize pass.  CTAs take the amax pass's ranges in reverse order (CTA i
+// gets range G-1-i) and walk them backwards, so that the first blocks read
+// are the ones the amax pass read last (still in L2).
 template <int FMT, int MODE, class SEG>
 __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
   constexpr int U = 2;  // blocks per lane per iteration
   __shared__ SegTables tb;
-  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
-  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
+  const int64_t ci = (int64_t)gridDim.x - 1 - blockIdx.x;
+  const int64_t b0 = cta_begin(ci, gridDim.x, a.nblocks);
+  const int64_t b1 = cta_begin(ci + 1, gridDim.x, a.nblocks);
   const int tid = threadIdx.x;
   if (FMT == TF4_NVFP4 && a.st_from_amax && blockIdx.x == 0 && a.s_t_out)
     for (int k = tid; k < seg.count(); k += kThreads) a.s_t_out[k] = tensor_scale(a.st_src[k], a.status);
@@ -686,12 +688,13 @@ struct GuidedArgs {
   int32_t* status;
 };
 
-// 8 guidance bits -> bit 0 of 8 nibbles
+// 8 guidance bits -> bit 0 of 8 nibbles (shift-or steps written as
+// multiplies: the shifted copies never overlap).
 __device__ __forceinline__ uint32_t spread_bits(uint32_t b) {
   uint32_t x = b & 0xFFu;
-  x = (x | (x << 12)) & 0x000F000Fu;
-  x = (x | (x << 6)) & 0x03030303u;
-  x = (x | (x << 3)) & 0x11111111u;
+  x = (x * 0x1001u) & 0x000F000Fu;
+  x = (x * 0x41u) & 0x03030303u;
+  x = (x * 0x9u) & 0x11111111u;
   return x;
 }
 
@@ -737,60 +740,69 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
       build_tables<false>(st, tb);
     }
     const int64_t n = hi - lo;
-    for (int64_t j = 0; j < n; j += kThreads) {
-      const int64_t k = j + tid;
-      const bool valid = k < n;
-      bool bad = false;
-      if (valid) {
-        const int64_t blk = lo + k;
-        uint32_t w[NW];
+    constexpr int U = 2;  // blocks per lane per iteration
+    for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
+      uint32_t w[U][NW], sc[U], g[U];
 #pragma unroll
-        for (int q = 0; q < NW / 4; ++q) {
-          const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
-          w[4 * q] = p.x; w[4 * q + 1] = p.y; w[4 * q + 2] = p.z; w[4 * q + 3] = p.w;
-        }
-        const uint32_t sc = a.rec_scales[blk];
-        uint32_t g;
-        if constexpr (FMT == TF4_NVFP4) g = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
-        else g = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
-        bad = block_absmax_bits(w) >= 0x7F80u;
-        uint32_t c[NQ];
-        float r = 0.0f;
-        if constexpr (FMT == TF4_NVFP4) {
-          if (tb.fast && (sc >> 3) >= 1u && sc < 0x7Fu) r = block_rho(tb.rho[sc & 7u], sc >> 3);
-          if (tb.rho[sc & 7u] == 0.0f) r = 0.0f;
-        } else {
-          if (sc >= 1u && sc <= 252u) r = __uint_as_float((254u - sc) << 23);  // 2^-(sc-127), exact
-        }
-        if (r != 0.0f) {
-          const bool rz = FMT == TF4_NVFP4 && tb.rz;
+      for (int u = 0; u < U; ++u) {
+        const int64_t k = j + u * kThreads + tid;
+        if (k < n) {
+          const int64_t blk = lo + k;
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            c[q] = rz ? cvt_words<true>(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], r)
-                      : cvt_words<false>(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], r);
-            const uint32_t mm = (c[q] ^ spread_bits(g >> (8 * q))) & 0x11111111u;
-            if (mm)
-              c[q] = rz ? fix_mismatches<true>(c[q], mm, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], r)
-                        : fix_mismatches<false>(c[q], mm, w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], r);
+          for (int q = 0; q < NW / 4; ++q) {
+            const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
+            w[u][4 * q] = p.x; w[u][4 * q + 1] = p.y; w[u][4 * q + 2] = p.z; w[u][4 * q + 3] = p.w;
           }
-        } else {
-          float S;
-          if constexpr (FMT == TF4_NVFP4) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
-          else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
-#pragma unroll
-          for (int q = 0; q < NQ; ++q) c[q] = 0u;
-#pragma unroll
-          for (int e = 0; e < BE; ++e) {
-            const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-            const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-            const uint32_t m3 = S > 0.0f ? guided_m3_exact(ax, S, (g >> e) & 1u) : 0u;
-            c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
-          }
+          sc[u] = a.rec_scales[blk];
+          if constexpr (FMT == TF4_NVFP4) g[u] = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
+          else g[u] = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
         }
-        if constexpr (FMT == TF4_NVFP4) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
-        else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);
       }
-      report_bad(bad, a.status);
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t k = j + u * kThreads + tid;
+        bool bad = false;
+        if (k < n) {
+          const int64_t blk = lo + k;
+          bad = block_absmax_bits(w[u]) >= 0x7F80u;
+          uint32_t c[NQ];
+          float r = 0.0f;
+          if constexpr (FMT == TF4_NVFP4) {
+            if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu) r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
+            if (tb.rho[sc[u] & 7u] == 0.0f) r = 0.0f;
+          } else {
+            if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);  // 2^-(sc-127), exact
+          }
+          if (r != 0.0f) {
+            const bool rz = FMT == TF4_NVFP4 && tb.rz;
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) {
+              const uint32_t* wq = &w[u][4 * q];
+              c[q] = rz ? cvt_words<true>(wq[0], wq[1], wq[2], wq[3], r) : cvt_words<false>(wq[0], wq[1], wq[2], wq[3], r);
+              const uint32_t mm = (c[q] ^ spread_bits(g[u] >> (8 * q))) & 0x11111111u;
+              if (mm)
+                c[q] = rz ? fix_mismatches<true>(c[q], mm, wq[0], wq[1], wq[2], wq[3], r)
+                          : fix_mismatches<false>(c[q], mm, wq[0], wq[1], wq[2], wq[3], r);
+            }
+          } else {
+            float S;
+            if constexpr (FMT == TF4_NVFP4) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
+            else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
+#pragma unroll
+            for (int q = 0; q < NQ; ++q) c[q] = 0u;
+#pragma unroll
+            for (int e = 0; e < BE; ++e) {
+              const uint32_t h = (e & 1) ? (w[u][e >> 1] >> 16) : (w[u][e >> 1] & 0xFFFFu);
+              const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+              const uint32_t m3 = S > 0.0f ? guided_m3_exact(ax, S, (g[u] >> e) & 1u) : 0u;
+              c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
+            }
+          }
+          if constexpr (FMT == TF4_NVFP4) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
+          else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);
+        }
+        report_bad(bad, a.status);
+      }
     }
     lo = hi;
   }

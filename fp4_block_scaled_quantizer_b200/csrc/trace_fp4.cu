@@ -94,10 +94,16 @@ int occupancy(const void* kernel) {
   return occ;
 }
 
-// One wave: SMs x resident CTAs of `kernel`, never more CTAs than units.
+// Grid = waves x SMs x resident CTAs of `kernel`: up to 4 waves while every
+// CTA still gets at least 2048 units (smaller ranges let CTAs that finish
+// early pick up the next wave's ranges, which shortens the tail of a single
+// wave of equal ranges), never more CTAs than units.
 template <class K>
 int64_t wave_grid(K kernel, int64_t units) {
-  const int64_t g = (int64_t)sm_count() * occupancy(reinterpret_cast<const void*>(kernel));
+  const int64_t wave = (int64_t)sm_count() * occupancy(reinterpret_cast<const void*>(kernel));
+  int64_t waves = units / (wave * 2048);
+  waves = waves < 1 ? 1 : (waves > 4 ? 4 : waves);
+  const int64_t g = wave * waves;
   return units < g ? (units > 0 ? units : 1) : g;
 }
 
