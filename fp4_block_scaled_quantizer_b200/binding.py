@@ -40,7 +40,8 @@ EXPORTS = (
     "tf4_workspace_bytes", "tf4_codes_bytes", "tf4_scales_bytes", "tf4_guidance_bytes",
     "tf4_record_bytes", "tf4_segment_amax", "tf4_quantize_rtn", "tf4_quantize_sr",
     "tf4_quantize_capture", "tf4_quantize_guided", "tf4_dequantize", "tf4_pack_guidance",
-    "tf4_unpack_guidance", "tf4_guided_fake_quant", "tf4_mismatch_stats", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
+    "tf4_unpack_guidance", "tf4_guided_fake_quant", "tf4_mismatch_stats", "tf4_workspace_bytes_batched",
+    "tf4_quantize_capture_batched", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
     "tf4_version",
 )
 
@@ -95,6 +96,9 @@ def lib():
                     "tf4_quantize_capture_noalloc": (st, [dp, vp, vp, vp, vp, vp, i32p, vp]),
                     "tf4_guided_fake_quant": (st, [dp, vp, vp, vp, vp, vp, vp, ctypes.c_int, i32p, vp]),
                     "tf4_mismatch_stats": (st, [dp, vp, vp, vp, vp, vp, i32p, vp]),
+                    "tf4_workspace_bytes_batched": (sz, [ctypes.c_int32]),
+                    "tf4_quantize_capture_batched": (st, [dp, ctypes.c_int32, vp, vp, vp, vp, ctypes.c_int32, vp,
+                                                          vp, sz, i32p, vp]),
                     "tf4_read_status": (st, [i32p, vp]),
                     "tf4_status_string": (ctypes.c_char_p, [st]),
                     "tf4_version": (ctypes.c_int, []),
@@ -168,7 +172,10 @@ _status_cache: dict = {}
 def workspace(desc: Desc, device, stream=None) -> torch.Tensor:
     """A zero-filled workspace for this device/stream (reused: every call
     returns it to zero when it completes)."""
-    need = lib().tf4_workspace_bytes(desc.ptr)
+    return _workspace_bytes(lib().tf4_workspace_bytes(desc.ptr), device, stream)
+
+
+def _workspace_bytes(need: int, device, stream=None) -> torch.Tensor:
     s = stream if stream is not None else torch.cuda.current_stream(device)
     key = (torch.device(device).index, s.cuda_stream)
     ws = _ws_cache.get(key)
@@ -269,6 +276,50 @@ def tf4_quantize_capture(x, fmt=NVFP4, seg_off=None, guidance=True, amax_in=None
                                       _ptr(status_word(x.device)), _stream(stream, x.device)),
            "tf4_quantize_capture")
     return q
+
+
+@dataclass
+class BatchedCapture:
+    codes: torch.Tensor            # uint8 [L, rows*cols/2]
+    scales: torch.Tensor           # uint8 [L, rows, cols/block]
+    s_t: Optional[torch.Tensor]    # float [L] (NVFP4)
+    info_bits: Optional[torch.Tensor]  # uint8 [keep, rows*cols/8]: the info cache
+    fmt: int
+    rows: int
+    cols: int
+    keep: int
+
+    def layer(self, i: int) -> Quantized:
+        """Layer i as a record usable by tf4_quantize_guided / tf4_dequantize."""
+        L = self.codes.shape[0]
+        bits = self.info_bits[i - (L - self.keep)] if i >= L - self.keep else None
+        s_t = self.s_t[i:i + 1] if self.s_t is not None else None
+        return Quantized(self.codes[i], self.scales[i], s_t, bits, self.fmt, self.rows, self.cols, None)
+
+
+def tf4_quantize_capture_batched(xs, fmt=NVFP4, keep=0, stream=None, out: Optional[BatchedCapture] = None):
+    """Capture a list of same-shaped bf16 tensors (layers) in two launches;
+    guidance is kept for the last `keep` layers, in one contiguous buffer."""
+    L = len(xs)
+    x2 = [_as_2d(x) for x in xs]
+    rows, cols = x2[0].shape
+    assert all(t.shape == (rows, cols) for t in x2)
+    dev = x2[0].device
+    d = Desc(fmt, rows, cols)
+    if out is None:
+        n = rows * cols
+        out = BatchedCapture(torch.empty((L, n // 2), dtype=torch.uint8, device=dev),
+                             torch.empty((L, rows, cols // BLOCK[fmt]), dtype=torch.uint8, device=dev),
+                             torch.empty(L, dtype=torch.float32, device=dev) if fmt == NVFP4 else None,
+                             torch.empty((keep, n // 8), dtype=torch.uint8, device=dev) if keep else None,
+                             fmt, rows, cols, keep)
+    ptrs = (ctypes.c_void_p * L)(*[t.data_ptr() for t in x2])
+    ws = _workspace_bytes(lib().tf4_workspace_bytes_batched(L), dev, stream)
+    _check(lib().tf4_quantize_capture_batched(d.ptr, L, ptrs, _ptr(out.codes), _ptr(out.scales), _ptr(out.s_t),
+                                              keep, _ptr(out.info_bits), _ptr(ws), ws.numel(),
+                                              _ptr(status_word(dev)), _stream(stream, dev)),
+           "tf4_quantize_capture_batched")
+    return out
 
 
 def tf4_quantize_guided(x, rec: Quantized, stream=None, out=None, rec_bits=None) -> torch.Tensor:

@@ -31,6 +31,10 @@ struct Seg1 {
   __device__ __forceinline__ int find(int64_t /*block*/) const { return 0; }
   __device__ __forceinline__ int64_t start(int /*s*/) const { return 0; }
   __device__ __forceinline__ int count() const { return 1; }
+  // input / guidance base pointers of segment s, addressed by the global
+  // block index (one tensor: the call's own pointers)
+  __device__ __forceinline__ const uint4* xptr(int /*s*/, const uint4* x) const { return x; }
+  __device__ __forceinline__ uint8_t* bitsptr(int /*s*/, uint8_t* b) const { return b; }
 };
 
 // Ragged segments (row offsets, passed by value in the kernel parameters).
@@ -51,6 +55,35 @@ struct SegN {
   }
   __device__ __forceinline__ int64_t start(int s) const { return (int64_t)off[s] * bpr; }
   __device__ __forceinline__ int count() const { return nseg; }
+  __device__ __forceinline__ const uint4* xptr(int /*s*/, const uint4* x) const { return x; }
+  __device__ __forceinline__ uint8_t* bitsptr(int /*s*/, uint8_t* b) const { return b; }
+};
+
+// A batch of same-shaped tensors (layers) quantized by one launch: segment s
+// is layer s with its own input pointer and its own tensor scale; codes and
+// scales are contiguous across layers (global block index), guidance bits
+// are kept only for layers s >= first_kept and stored contiguously from
+// there (the info cache).  The returned bases are offset so that
+// base + (units per block) * global_block addresses the layer's data.
+struct SegBatch {
+  int32_t nlayers;
+  int32_t first_kept;       // layers >= first_kept write guidance
+  int64_t bpl;              // blocks per layer
+  int32_t units_per_block;  // 16-byte input units per block (2 NVFP4, 4 MXFP4)
+  int32_t bits_per_block;   // guidance bytes per block (2 NVFP4, 4 MXFP4)
+  const uint4* x[TF4_MAX_BATCH];
+  __device__ __forceinline__ int find(int64_t block) const { return (int)(block / bpl); }
+  __device__ __forceinline__ int64_t start(int s) const { return (int64_t)s * bpl; }
+  __device__ __forceinline__ int count() const { return nlayers; }
+  __device__ __forceinline__ const uint4* xptr(int s, const uint4*) const {
+    return reinterpret_cast<const uint4*>(reinterpret_cast<uintptr_t>(x[s]) -
+                                          (uintptr_t)(start(s) * units_per_block * 16));
+  }
+  __device__ __forceinline__ uint8_t* bitsptr(int s, uint8_t* b) const {
+    if (!b || s < first_kept) return nullptr;
+    return reinterpret_cast<uint8_t*>(reinterpret_cast<uintptr_t>(b) -
+                                      (uintptr_t)(start(first_kept) * bits_per_block));
+  }
 };
 
 __device__ __forceinline__ int64_t cta_begin(int64_t i, int64_t grid, int64_t n) {
@@ -269,6 +302,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, 
   while (lo < b1) {
     const int s = seg.find(lo);
     const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
+    const uint4* xs = seg.xptr(s, x);
     // chunks [2lo, 2hi), 8 in flight per thread
     const int64_t c0 = 2 * lo, c1 = 2 * hi;
     uint32_t m = 0;
@@ -276,7 +310,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, 
     for (; c + 7 * kThreads < c1; c += 8 * kThreads) {
       uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldg(x + c + u * kThreads);
+      for (int u = 0; u < 8; ++u) v[u] = __ldg(xs + c + u * kThreads);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         m = vmax_u16x2(m, v[u].x & 0x7FFF7FFFu);
@@ -286,7 +320,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, 
       }
     }
     for (; c < c1; c += kThreads) {
-      const uint4 v = __ldg(x + c);
+      const uint4 v = __ldg(xs + c);
       m = vmax_u16x2(m, v.x & 0x7FFF7FFFu);
       m = vmax_u16x2(m, v.y & 0x7FFF7FFFu);
       m = vmax_u16x2(m, v.z & 0x7FFF7FFFu);
@@ -600,6 +634,8 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
       if (MODE != kSR) build_tables<true>(st, tb);
       else build_tables<false, true>(st, tb);
     }
+    const uint4* xs = seg.xptr(s, a.x);
+    uint8_t* bits = seg.bitsptr(s, a.bits);
     const int64_t n = hi - lo;
     for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
       if constexpr (FMT == TF4_NVFP4) {
@@ -610,7 +646,7 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
           const int64_t k = j + u * kThreads + tid;
           blk[u] = hi - 1 - k;
           if (k < n) {
-            const uint4 p = __ldg(a.x + 2 * blk[u]), q = __ldg(a.x + 2 * blk[u] + 1);
+            const uint4 p = __ldg(xs + 2 * blk[u]), q = __ldg(xs + 2 * blk[u] + 1);
             w[u][0] = p.x; w[u][1] = p.y; w[u][2] = p.z; w[u][3] = p.w;
             w[u][4] = q.x; w[u][5] = q.y; w[u][6] = q.z; w[u][7] = q.w;
           }
@@ -627,8 +663,8 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
               nvfp4_block<MODE, false>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
             reinterpret_cast<uint2*>(a.codes)[blk[u]] = make_uint2(c0, c1);
             a.scales[blk[u]] = (uint8_t)sc;
-            if (MODE == kCAPTURE && a.bits)
-              reinterpret_cast<uint16_t*>(a.bits)[blk[u]] =
+            if (MODE == kCAPTURE && bits)
+              reinterpret_cast<uint16_t*>(bits)[blk[u]] =
                   (uint16_t)(nibble_lsbs(c0) | (nibble_lsbs(c1) << 8));
           }
           report_bad(bad, a.status);
@@ -643,7 +679,7 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
           if (k < n) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
-              const uint4 p = __ldg(a.x + 4 * blk[u] + q);
+              const uint4 p = __ldg(xs + 4 * blk[u] + q);
               w[u][4 * q] = p.x; w[u][4 * q + 1] = p.y; w[u][4 * q + 2] = p.z; w[u][4 * q + 3] = p.w;
             }
           }
@@ -657,8 +693,8 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
             mxfp4_block<MODE>(w[u], blk[u], a.seed, c, sc, bad);
             reinterpret_cast<uint4*>(a.codes)[blk[u]] = make_uint4(c[0], c[1], c[2], c[3]);
             a.scales[blk[u]] = (uint8_t)sc;
-            if (MODE == kCAPTURE && a.bits)
-              reinterpret_cast<uint32_t*>(a.bits)[blk[u]] =
+            if (MODE == kCAPTURE && bits)
+              reinterpret_cast<uint32_t*>(bits)[blk[u]] =
                   nibble_lsbs(c[0]) | (nibble_lsbs(c[1]) << 8) | (nibble_lsbs(c[2]) << 16) |
                   (nibble_lsbs(c[3]) << 24);
           }

@@ -301,6 +301,74 @@ tf4_status tf4_quantize_capture(const tf4_desc* desc, const void* x, const float
                                       stream);
 }
 
+size_t tf4_workspace_bytes_batched(int32_t num_layers) {
+  if (num_layers < 1 || num_layers > TF4_MAX_BATCH) return 0;
+  return ((size_t)(num_layers + 1) * sizeof(uint32_t) + 255) & ~(size_t)255;
+}
+
+tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const void* const* x, uint8_t* codes,
+                                        uint8_t* scales, float* s_t, int32_t keep, uint8_t* info_bits, void* ws,
+                                        size_t ws_bytes, int32_t* status, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.nseg != 1) return TF4_ERR_INVALID_ARG;
+  if (nl < 1 || nl > TF4_MAX_BATCH || !x) return TF4_ERR_INVALID_ARG;
+  if (keep < 0 || keep > nl || ((keep > 0) != (info_bits != nullptr))) return TF4_ERR_INVALID_ARG;
+  const bool nv = sh.fmt == TF4_NVFP4;
+  if (nv && !s_t) return TF4_ERR_INVALID_ARG;
+  if ((nv && !aligned(s_t, 4)) || (status && !aligned(status, 4))) return TF4_ERR_ALIGN;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (sh.n == 0) {
+    if (nv) return cudaMemsetAsync(s_t, 0, sizeof(float) * nl, st) == cudaSuccess ? TF4_OK : TF4_ERR_CUDA;
+    return TF4_OK;
+  }
+  if (!codes || !scales) return TF4_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || (info_bits && !aligned(info_bits, 4))) return TF4_ERR_ALIGN;
+  for (int k = 0; k < nl; ++k) {
+    if (!x[k]) return TF4_ERR_INVALID_ARG;
+    if (!aligned(x[k], 16)) return TF4_ERR_ALIGN;
+  }
+  if (nv) {
+    if (!ws) return TF4_ERR_WORKSPACE;
+    if (!aligned(ws, 4)) return TF4_ERR_ALIGN;
+    if (ws_bytes < tf4_workspace_bytes_batched(nl)) return TF4_ERR_WORKSPACE;
+  }
+  tf4::SegBatch sb;
+  std::memset(&sb, 0, sizeof sb);
+  sb.nlayers = nl;
+  sb.first_kept = nl - keep;
+  sb.bpl = sh.nblocks;
+  sb.units_per_block = sh.be / 8;
+  sb.bits_per_block = sh.be / 8;
+  for (int k = 0; k < nl; ++k) sb.x[k] = static_cast<const uint4*>(x[k]);
+  const int64_t total = sh.nblocks * nl;
+  tf4::QuantArgs a;
+  a.x = nullptr;
+  a.nblocks = total;
+  a.codes = codes;
+  a.scales = scales;
+  a.bits = info_bits;
+  a.seed = 0;
+  a.status = status;
+  a.s_t_out = s_t;
+  a.st_src = s_t;
+  a.st_from_amax = 0;
+  if (nv) {
+    const int64_t grid = wave_grid(tf4::k_quant<TF4_NVFP4, tf4::kCAPTURE, tf4::SegBatch>, total);
+    tf4::k_amax<tf4::SegBatch><<<(unsigned)grid, kThreads, 0, st>>>(nullptr, total, sb, static_cast<uint32_t*>(ws),
+                                                                    s_t, nullptr, status);
+    if ((e = launched()) != TF4_OK) return e;
+    tf4::k_quant<TF4_NVFP4, tf4::kCAPTURE, tf4::SegBatch><<<(unsigned)grid, kThreads, 0, st>>>(a, sb);
+  } else {
+    a.s_t_out = nullptr;
+    a.st_src = nullptr;
+    const int64_t grid = wave_grid(tf4::k_quant<TF4_MXFP4, tf4::kCAPTURE, tf4::SegBatch>, total);
+    tf4::k_quant<TF4_MXFP4, tf4::kCAPTURE, tf4::SegBatch><<<(unsigned)grid, kThreads, 0, st>>>(a, sb);
+  }
+  return launched();
+}
+
 tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_t* rec_scales,
                                const float* rec_s_t, const uint8_t* rec_bits, uint8_t* codes, int32_t* status,
                                tf4_stream_t stream) {

@@ -101,6 +101,7 @@ typedef enum {
 typedef enum { TF4_NVFP4 = 0, TF4_MXFP4 = 1 } tf4_format;
 
 #define TF4_MAX_SEGMENTS 1024
+#define TF4_MAX_BATCH 64
 #define TF4_DEV_NONFINITE 1 /* bit OR-ed into *dev_status */
 #define TF4_DEV_TIMEOUT 2   /* bit OR-ed into *dev_status */
 
@@ -152,6 +153,28 @@ tf4_status tf4_quantize_capture(const tf4_desc* desc, const void* x, const float
                                 uint8_t* codes, uint8_t* scales, float* s_t,
                                 uint8_t* guidance_bits, void* workspace, size_t workspace_bytes,
                                 int32_t* dev_status, tf4_stream_t stream);
+
+/* Batched rollout-side capture of num_layers (1..TF4_MAX_BATCH) tensors of
+ * the same shape (desc; num_segments must be 1) in two launches instead of
+ * two per layer -- the whole activation stack of a rollout step at once,
+ * with the compact records of the deepest `keep` layers written into one
+ * contiguous buffer: the quantization-info cache of the TRACE summary's
+ * "量子化情報キャッシュ" section, ready to be shipped to the trainer.
+ *   x          HOST array [num_layers] of device pointers (16-byte aligned)
+ *   codes      device [num_layers][rows*cols/2], contiguous
+ *   scales     device [num_layers][rows*cols/block], contiguous
+ *   s_t        NVFP4: device [num_layers] (per-layer tensor scale); MXFP4: NULL
+ *   keep       0..num_layers: layers [num_layers-keep, num_layers) keep guidance
+ *   info_bits  device [keep][rows*cols/8], contiguous (NULL iff keep == 0)
+ *   workspace  NVFP4: tf4_workspace_bytes_batched(num_layers) zero-filled bytes
+ *              (left zero-filled); MXFP4: unused
+ * Per layer the results equal tf4_quantize_capture on that layer alone. */
+size_t tf4_workspace_bytes_batched(int32_t num_layers);
+tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t num_layers,
+                                        const void* const* x, uint8_t* codes, uint8_t* scales,
+                                        float* s_t, int32_t keep, uint8_t* info_bits,
+                                        void* workspace, size_t workspace_bytes,
+                                        int32_t* dev_status, tf4_stream_t stream);
 
 /* Train-side guided quantization of x (the trainer's value) with the
  * rollout's recorded scale bytes, recorded s_t (NVFP4; NULL for MXFP4) and

@@ -131,3 +131,21 @@ def test_package_exports_entry_points():
     for n in ("tf4_quantize_rtn", "tf4_quantize_sr", "tf4_quantize_capture", "tf4_quantize_guided",
               "tf4_dequantize", "tf4_pack_guidance", "tf4_unpack_guidance", "tf4_segment_amax"):
         assert callable(getattr(tf4, n))
+
+
+def test_batched_capture_rejects_bad_arguments(L):
+    d = B.Desc(B.NVFP4, 4, 32)
+    ptrs = (ctypes.c_void_p * 2)(0x10000, 0x20000)
+    call = lambda desc, nl, x, keep, info, ws=GOOD, wsb=4096, s_t=GOOD: L.tf4_quantize_capture_batched(
+        desc.ptr, nl, x, GOOD, GOOD, s_t, keep, info, ws, wsb, None, None)
+    assert call(d, 0, ptrs, 0, None) == 1                       # no layers
+    assert call(d, 65, ptrs, 0, None) == 1                      # more than TF4_MAX_BATCH
+    assert call(d, 2, None, 0, None) == 1                       # no pointer array
+    assert call(d, 2, ptrs, 3, GOOD) == 1                       # keep > num_layers
+    assert call(d, 2, ptrs, 1, None) == 1                       # keep > 0 without a buffer
+    assert call(d, 2, ptrs, 0, GOOD) == 1                       # buffer without keep
+    assert call(B.Desc(B.NVFP4, 4, 32, [0, 2, 4]), 2, ptrs, 0, None) == 1  # segmented layers
+    assert call(d, 2, (ctypes.c_void_p * 2)(0x10000, 0x20001), 0, None) == 3  # misaligned layer
+    assert call(d, 2, ptrs, 0, None, wsb=4) == 4                # workspace too small
+    assert call(d, 2, ptrs, 0, None, s_t=None) == 1
+    assert L.tf4_workspace_bytes_batched(3) == 256 and L.tf4_workspace_bytes_batched(0) == 0

@@ -290,6 +290,26 @@ def test_mismatch_stats_parity(fmt, seg, rel):
         assert want[0] == want[1] + want[2]
 
 
+@pytest.mark.parametrize("fmt,L,keep", [(O.NVFP4, 5, 2), (O.NVFP4, 3, 3), (O.NVFP4, 1, 0), (O.MXFP4, 4, 1)])
+def test_capture_batched_parity(fmt, L, keep):
+    """One batched call = per-layer capture (oracle) for every layer; the
+    deepest `keep` layers' guidance lands contiguously in the info cache."""
+    xs = [W.random_bf16((96, 1024), seed=60 + i, device=DEV, outlier_frac=0.01 * (i % 2)) for i in range(L)]
+    out = B.tf4_quantize_capture_batched(xs, fmt=fmt, keep=keep)
+    assert B.read_status(xs[0].device) == 0
+    for i, x in enumerate(xs):
+        r = O.quantize(W.bf16_bits(x), fmt, O.RTN, bits=True)
+        assert_same(f"codes {i}", host(out.codes[i]), r["codes"])
+        assert_same(f"scales {i}", host(out.scales[i]), r["scales"])
+        if fmt == O.NVFP4:
+            assert_same(f"s_t {i}", f32_bits(host(out.s_t[i:i + 1])), f32_bits(r["s_t"]))
+        if i >= L - keep:
+            assert_same(f"bits {i}", host(out.info_bits[i - (L - keep)]), r["bits"])
+    if keep:
+        g = B.tf4_quantize_guided(xs[-1], out.layer(L - 1))
+        assert torch.equal(g, out.codes[L - 1])
+
+
 @pytest.mark.parametrize("shape", [(1, 16), (3, 48), (64, 1024), (5, 16 * 33)])
 def test_pack_unpack_parity(shape):
     rows, cols = shape
