@@ -301,6 +301,12 @@ tf4_status tf4_quantize_capture(const tf4_desc* desc, const void* x, const float
                                       stream);
 }
 
+// Layers of at least this many elements (256 MiB of bf16) are captured by
+// one launch pair per layer; smaller layers by one pair for the whole batch
+// (measured on B200: batching wins up to 128 MiB layers -- by 1.35x there
+// and by 3-9x for 4-16 MiB layers -- and loses about 5% at 512 MiB).
+constexpr int64_t kBatchPerLayerElems = int64_t(1) << 27;
+
 size_t tf4_workspace_bytes_batched(int32_t num_layers) {
   if (num_layers < 1 || num_layers > TF4_MAX_BATCH) return 0;
   return ((size_t)(num_layers + 1) * sizeof(uint32_t) + 255) & ~(size_t)255;
@@ -333,6 +339,21 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const 
     if (!ws) return TF4_ERR_WORKSPACE;
     if (!aligned(ws, 4)) return TF4_ERR_ALIGN;
     if (ws_bytes < tf4_workspace_bytes_batched(nl)) return TF4_ERR_WORKSPACE;
+  }
+  if (sh.n >= kBatchPerLayerElems) {
+    // Large layers: the per-layer launch pair is as fast as it gets (the
+    // quantize pass re-reads the amax pass's last blocks from L2, and the
+    // single-tensor kernels run at higher occupancy); launch gaps are
+    // negligible next to a layer's run time.
+    const int64_t first_kept = nl - keep;
+    for (int k = 0; k < nl; ++k) {
+      uint8_t* bk = k >= first_kept ? info_bits + (size_t)(k - first_kept) * (size_t)(sh.n / 8) : nullptr;
+      e = tf4_quantize_capture(desc, x[k], nullptr, codes + (size_t)k * (size_t)(sh.n / 2),
+                               scales + (size_t)k * (size_t)sh.nblocks, nv ? s_t + k : nullptr, bk, ws, ws_bytes,
+                               status, stream);
+      if (e != TF4_OK) return e;
+    }
+    return TF4_OK;
   }
   tf4::SegBatch sb;
   std::memset(&sb, 0, sizeof sb);

@@ -156,7 +156,9 @@ tf4_status tf4_quantize_capture(const tf4_desc* desc, const void* x, const float
 
 /* Batched rollout-side capture of num_layers (1..TF4_MAX_BATCH) tensors of
  * the same shape (desc; num_segments must be 1) in two launches instead of
- * two per layer -- the whole activation stack of a rollout step at once,
+ * two per layer (layers of 2^27 elements or more -- where launch gaps no
+ * longer matter -- are run as one launch pair per layer inside the call,
+ * with the same results) -- the whole activation stack of a rollout step at once,
  * with the compact records of the deepest `keep` layers written into one
  * contiguous buffer: the quantization-info cache of the TRACE summary's
  * "量子化情報キャッシュ" section, ready to be shipped to the trainer.

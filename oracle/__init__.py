@@ -15,10 +15,11 @@ import numpy as np
 
 from . import build as _build
 
-NVFP4, MXFP4 = 0, 1
+NVFP4, MXFP4, UFP4 = 0, 1, 2
 RTN, SR = 0, 1
 NONFINITE = 1
-BLOCK = {NVFP4: 16, MXFP4: 32}
+BLOCK = {NVFP4: 16, MXFP4: 32, UFP4: 16}
+HAS_TENSOR_SCALE = {NVFP4: True, MXFP4: False, UFP4: True}
 
 _lib = None
 
@@ -37,20 +38,26 @@ def lib():
         sig = {
             "orc_bf16_to_float": (ctypes.c_float, [ctypes.c_uint16]),
             "orc_e2m1_value": (d, [ctypes.c_int]),
+            "orc_grid_value": (d, [ctypes.c_int, ctypes.c_int]),
             "orc_e4m3_value": (d, [ctypes.c_uint8]),
             "orc_e4m3_encode": (ctypes.c_uint8, [ctypes.c_float]),
             "orc_e8m0_exponent": (ctypes.c_int, [ctypes.c_float]),
+            "orc_tensor_scale": (ctypes.c_float, [ctypes.c_int, ctypes.c_float]),
             "orc_nvfp4_tensor_scale": (ctypes.c_float, [ctypes.c_float]),
+            "orc_block_scale_code": (ctypes.c_uint8, [ctypes.c_int, ctypes.c_float, ctypes.c_float]),
             "orc_nvfp4_block_scale_code": (ctypes.c_uint8, [ctypes.c_float, ctypes.c_float]),
             "orc_nvfp4_block_scale": (ctypes.c_float, [ctypes.c_uint8, ctypes.c_float]),
             "orc_mxfp4_block_scale": (ctypes.c_float, [ctypes.c_uint8]),
             "orc_rtn_m3": (ctypes.c_int, [d, d]),
             "orc_sr_m3": (ctypes.c_int, [d, d, ctypes.c_uint32]),
             "orc_guided_m3": (ctypes.c_int, [d, d, ctypes.c_int]),
+            "orc_rtn_code": (ctypes.c_int, [ctypes.c_int, d, d]),
+            "orc_sr_code": (ctypes.c_int, [ctypes.c_int, d, d, ctypes.c_uint32]),
+            "orc_guided_code": (ctypes.c_int, [ctypes.c_int, d, d, ctypes.c_int]),
             "orc_philox4x32_10": (None, [u32p, u32p, u32p]),
             "orc_sr_uniform24": (ctypes.c_uint32, [u64, u64]),
             "orc_segment_amax": (ctypes.c_int, [u16p, i64, i64, i32, i64p, f32p]),
-            "orc_segment_scales": (ctypes.c_int, [u16p, i64, i64, i32, i64p, f32p]),
+            "orc_segment_scales": (ctypes.c_int, [ctypes.c_int, u16p, i64, i64, i32, i64p, f32p]),
             "orc_quantize_rows": (ctypes.c_int, [ctypes.c_int, ctypes.c_int, u16p, i64, i64, i32, i64p,
                                                  f32p, u64, i64, i64, u8p, u8p, u8p]),
             "orc_quantize_guided_rows": (ctypes.c_int, [ctypes.c_int, u16p, i64, i64, i32, i64p, u8p,
@@ -104,6 +111,30 @@ def nvfp4_tensor_scale(amax: float) -> float:
     return float(lib().orc_nvfp4_tensor_scale(float(amax)))
 
 
+def tensor_scale(fmt: int, amax: float) -> float:
+    return float(lib().orc_tensor_scale(int(fmt), float(amax)))
+
+
+def block_scale_code(fmt: int, bamax: float, s_t: float) -> int:
+    return int(lib().orc_block_scale_code(int(fmt), float(bamax), float(s_t)))
+
+
+def grid_value(fmt: int, m3: int) -> float:
+    return float(lib().orc_grid_value(int(fmt), int(m3)))
+
+
+def rtn_code(fmt: int, ax: float, S: float) -> int:
+    return int(lib().orc_rtn_code(int(fmt), float(ax), float(S)))
+
+
+def sr_code(fmt: int, ax: float, S: float, r24: int) -> int:
+    return int(lib().orc_sr_code(int(fmt), float(ax), float(S), int(r24)))
+
+
+def guided_code(fmt: int, ax: float, S: float, g: int) -> int:
+    return int(lib().orc_guided_code(int(fmt), float(ax), float(S), int(g)))
+
+
 def rtn_m3(ax: float, S: float) -> int:
     return int(lib().orc_rtn_m3(float(ax), float(S)))
 
@@ -139,28 +170,29 @@ def segment_amax(x, seg_off=None):
     return out, st
 
 
-def segment_scales(x, seg_off=None):
+def segment_scales(x, seg_off=None, fmt=NVFP4):
     x = np.ascontiguousarray(x, dtype=np.uint16)
     rows, cols = x.shape
     nseg, so = _seg(seg_off, rows)
     out = np.zeros(nseg, dtype=np.float32)
-    st = lib().orc_segment_scales(_p(x, ctypes.c_uint16), rows, cols, nseg, _p(so, ctypes.c_int64),
+    st = lib().orc_segment_scales(int(fmt), _p(x, ctypes.c_uint16), rows, cols, nseg, _p(so, ctypes.c_int64),
                                   _p(out, ctypes.c_float))
     return out, st
 
 
 def quantize(x, fmt=NVFP4, mode=RTN, seg_off=None, seed=0, bits=False, s_t=None, row_range=None):
     """Returns dict(codes, scales, s_t, bits, status).  ``s_t`` may be given
-    (NVFP4) to quantize a row range of a larger tensor without a full pass."""
+    (NVFP4 / UFP4) to quantize a row range of a larger tensor without a full
+    pass."""
     x = np.ascontiguousarray(x, dtype=np.uint16)
     rows, cols = x.shape
     blk = BLOCK[fmt]
     assert cols % blk == 0
     nseg, so = _seg(seg_off, rows)
     status = 0
-    if fmt == NVFP4:
+    if HAS_TENSOR_SCALE[fmt]:
         if s_t is None:
-            s_t, status = segment_scales(x, seg_off)
+            s_t, status = segment_scales(x, seg_off, fmt)
         s_t = np.ascontiguousarray(s_t, dtype=np.float32)
     else:
         s_t = None

@@ -8,8 +8,9 @@
  *
  * Exactness notes used throughout:
  *  - a bf16 value has at most 8 significant bits, an fp32 scale S at most
- *    24, and every E2M1 codeword or midpoint is k/4 with k < 32, so a
- *    product (codeword or midpoint) * S is exact in double (<= 29 bits);
+ *    24, and every codeword or midpoint of either grid (E2M1, uniform) is
+ *    k/4 with k < 32, so a product (codeword or midpoint) * S is exact in
+ *    double (<= 29 bits);
  *  - every decision below is a comparison between two such exact doubles,
  *    never a comparison of a rounded quotient; "y = |x| / S" is the real
  *    quotient, compared through |x| vs c*S.
@@ -23,6 +24,16 @@
  * [FQT] section 3: E2M1 = 2-bit exponent, 1-bit mantissa. */
 static const double kE2M1[8] = {0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0};
 
+/* Uniform 4-bit grid ([UFP4] design section: E1M2 / INT4): magnitudes
+ * 0..7 in steps of one, indexed by the same 3-bit magnitude code.  (E1M2's
+ * grid is this one divided by 4; with the tensor scale defined from the
+ * grid maximum the two give the same codes and scale bytes.) */
+static const double kUniform[8] = {0.0, 1.0, 2.0, 3.0, 4.0, 5.0, 6.0, 7.0};
+
+static const double* grid_of(int fmt) { return fmt == ORC_UFP4 ? kUniform : kE2M1; }
+static int block_of(int fmt) { return fmt == ORC_MXFP4 ? 32 : 16; }
+static int has_tensor_scale(int fmt) { return fmt != ORC_MXFP4; }
+
 float orc_bf16_to_float(uint16_t h) {
   uint32_t u = (uint32_t)h << 16; /* bf16 is the top half of an fp32 */
   float f;
@@ -35,6 +46,7 @@ static int bf16_sign(uint16_t h) { return (h >> 15) & 1; }
 static double bf16_abs(uint16_t h) { return (double)orc_bf16_to_float((uint16_t)(h & 0x7FFFu)); }
 
 double orc_e2m1_value(int m3) { return kE2M1[m3 & 7]; }
+double orc_grid_value(int fmt, int m3) { return grid_of(fmt)[m3 & 7]; }
 
 /* E4M3 ("fn" variant: no infinities, 0x7F/0xFF are NaN): bias 7,
  * subnormals m * 2^-9, largest finite 448 (0x7E).  [FQT] section 3 names
@@ -77,23 +89,29 @@ int orc_e8m0_exponent(float bamax) {
   return e;
 }
 
-/* NVFP4 per-tensor scale s_t = amax / (6 * 448) in fp32.  A result below
- * the smallest normal fp32 (including amax == 0) makes the whole segment
+/* Per-tensor scale s_t = amax / (grid max * 448) in fp32: 2688 = 6 * 448
+ * for NVFP4, 3136 = 7 * 448 for the uniform grid.  A result below the
+ * smallest normal fp32 (including amax == 0) makes the whole segment
  * quantize to signed zeros with s_t = 0. */
-float orc_nvfp4_tensor_scale(float amax) {
-  float s = amax / 2688.0f;
+float orc_tensor_scale(int fmt, float amax) {
+  float s = amax / (fmt == ORC_UFP4 ? 3136.0f : 2688.0f);
   if (!(s >= 0x1p-126f)) s = 0.0f;
   return s;
 }
 
-/* NVFP4 block scale code: b = E4M3( (bamax / 6) / s_t ), two fp32 divides
- * in that order; s_t == 0 gives 0. */
-uint8_t orc_nvfp4_block_scale_code(float bamax, float s_t) {
+float orc_nvfp4_tensor_scale(float amax) { return orc_tensor_scale(ORC_NVFP4, amax); }
+
+/* E4M3 block scale code: b = E4M3( (bamax / grid max) / s_t ), two fp32
+ * divides in that order (grid max 6 for NVFP4, 7 for the uniform grid);
+ * s_t == 0 gives 0. */
+uint8_t orc_block_scale_code(int fmt, float bamax, float s_t) {
   if (s_t == 0.0f) return 0;
-  float q = bamax / 6.0f;
+  float q = bamax / (fmt == ORC_UFP4 ? 7.0f : 6.0f);
   float r = q / s_t;
   return orc_e4m3_encode(r);
 }
+
+uint8_t orc_nvfp4_block_scale_code(float bamax, float s_t) { return orc_block_scale_code(ORC_NVFP4, bamax, s_t); }
 
 /* Effective block scale S = s_t * dec(b), one fp32 multiply. */
 float orc_nvfp4_block_scale(uint8_t code, float s_t) {
@@ -104,69 +122,79 @@ float orc_nvfp4_block_scale(uint8_t code, float s_t) {
 float orc_mxfp4_block_scale(uint8_t code) { return (float)ldexp(1.0, (int)code - 127); }
 
 /* Round-to-nearest: the codeword nearest to y = ax / S (real quotient),
- * ties to the even m3; saturation at 6 is the nearest-codeword rule itself.
- * [TRACE-JA] mismatch section: plain nearest rounding is what the rollout
- * does; [FQT] section 3: round-to-nearest in the forward pass.
+ * ties to the even m3; saturation at the grid maximum is the
+ * nearest-codeword rule itself.  [TRACE-JA] mismatch section: plain
+ * nearest rounding is what the rollout does; [FQT] section 3:
+ * round-to-nearest in the forward pass.
  * Scan the sorted grid; codeword j beats the current best b (< j) iff y is
  * above their midpoint, i.e. 2*ax > (V_b + V_j) * S (both sides exact). */
-int orc_rtn_m3(double ax, double S) {
+static int rtn_on(const double* V, double ax, double S) {
   if (S == 0.0) return 0;
   int best = 0;
   for (int j = 1; j < 8; ++j) {
-    double lhs = 2.0 * ax, rhs = (kE2M1[best] + kE2M1[j]) * S;
+    double lhs = 2.0 * ax, rhs = (V[best] + V[j]) * S;
     if (lhs > rhs || (lhs == rhs && (j % 2) == 0)) best = j;
   }
   return best;
 }
 
-/* Neighbours of y = ax / S on the grid (S > 0, y < 6, y not a codeword):
- * lo = the largest j with V_j * S < ax. */
-static int grid_floor(double ax, double S) {
+/* Neighbours of y = ax / S on the grid (S > 0, y below the grid maximum,
+ * y not a codeword): lo = the largest j with V_j * S < ax. */
+static int grid_floor(const double* V, double ax, double S) {
   int lo = 0;
   for (int j = 1; j < 8; ++j)
-    if (kE2M1[j] * S < ax) lo = j;
+    if (V[j] * S < ax) lo = j;
   return lo;
 }
 
 /* Index of the codeword equal to y, or -1. */
-static int grid_exact(double ax, double S) {
+static int grid_exact(const double* V, double ax, double S) {
   for (int j = 0; j < 8; ++j)
-    if (kE2M1[j] * S == ax) return j;
+    if (V[j] * S == ax) return j;
   return -1;
 }
 
 /* Stochastic rounding with a 24-bit uniform integer r: between the two
  * neighbours lo < y < hi round up iff r < 2^24 (y - lo) / (hi - lo), i.e.
  * r * (V_hi - V_lo) * S < 2^24 * (ax - V_lo * S).  Left side: <= 48 bits;
- * right side: ax and V_lo*S within a factor 2 (or V_lo = 0), so the
- * difference is exact (Sterbenz) -- both sides exact in double.
- * y >= 6 saturates to 6; a codeword keeps itself.  [FQT] section 3. */
-int orc_sr_m3(double ax, double S, uint32_t r24) {
+ * right side: ax and V_lo*S within a factor 2 (or V_lo = 0; on the uniform
+ * grid ax - V_lo*S is a multiple of ulp(S) below S), so the difference is
+ * exact -- both sides exact in double.
+ * y >= grid max saturates; a codeword keeps itself.  [FQT] section 3. */
+static int sr_on(const double* V, double ax, double S, uint32_t r24) {
   if (S == 0.0) return 0;
-  if (ax >= 6.0 * S) return 7;
-  int ex = grid_exact(ax, S);
+  if (ax >= V[7] * S) return 7;
+  int ex = grid_exact(V, ax, S);
   if (ex >= 0) return ex;
-  int lo = grid_floor(ax, S), hi = lo + 1;
-  double lhs = (double)r24 * (kE2M1[hi] - kE2M1[lo]) * S;
-  double rhs = 16777216.0 * (ax - kE2M1[lo] * S);
+  int lo = grid_floor(V, ax, S), hi = lo + 1;
+  double lhs = (double)r24 * (V[hi] - V[lo]) * S;
+  double rhs = 16777216.0 * (ax - V[lo] * S);
   return lhs < rhs ? hi : lo;
 }
 
 /* Rollout-guided rounding: of the two grid neighbours of y, take the one
  * whose mantissa bit (m3 & 1) equals the recorded bit g.  Adjacent
- * codewords always differ in that bit, so exactly one qualifies.  A value
- * that is a codeword keeps it; y >= 6 gives 6 (both neighbours are 6).
+ * codewords always differ in that bit (on E2M1 and on the uniform grid), so
+ * exactly one qualifies.  A value that is a codeword keeps it; y at or
+ * above the grid maximum gives the maximum (both neighbours are it).
  * [TRACE-JA] mechanism section (the candidates are the two adjacent
  * codewords, chosen by a light comparison) and quantization-info cache
  * section (mantissa bit + scale identify the codeword). */
-int orc_guided_m3(double ax, double S, int g) {
+static int guided_on(const double* V, double ax, double S, int g) {
   if (S == 0.0) return 0;
-  if (ax >= 6.0 * S) return 7;
-  int ex = grid_exact(ax, S);
+  if (ax >= V[7] * S) return 7;
+  int ex = grid_exact(V, ax, S);
   if (ex >= 0) return ex;
-  int lo = grid_floor(ax, S), hi = lo + 1;
+  int lo = grid_floor(V, ax, S), hi = lo + 1;
   return ((lo & 1) == (g & 1)) ? lo : hi;
 }
+
+int orc_rtn_m3(double ax, double S) { return rtn_on(kE2M1, ax, S); }
+int orc_sr_m3(double ax, double S, uint32_t r24) { return sr_on(kE2M1, ax, S, r24); }
+int orc_guided_m3(double ax, double S, int g) { return guided_on(kE2M1, ax, S, g); }
+int orc_rtn_code(int fmt, double ax, double S) { return rtn_on(grid_of(fmt), ax, S); }
+int orc_sr_code(int fmt, double ax, double S, uint32_t r24) { return sr_on(grid_of(fmt), ax, S, r24); }
+int orc_guided_code(int fmt, double ax, double S, int g) { return guided_on(grid_of(fmt), ax, S, g); }
 
 /* Philox4x32-10 [PHILOX]: 10 rounds of the 4x32 Philox S-box; between
  * rounds the 2-word key is bumped by the Weyl constants.  One round:
@@ -249,12 +277,18 @@ int orc_segment_amax(const uint16_t* x, int64_t rows, int64_t cols, int32_t nseg
   return status;
 }
 
-int orc_segment_scales(const uint16_t* x, int64_t rows, int64_t cols, int32_t nseg,
+int orc_segment_scales(int fmt, const uint16_t* x, int64_t rows, int64_t cols, int32_t nseg,
                        const int64_t* seg_off, float* s_t_out) {
   int status = orc_segment_amax(x, rows, cols, nseg, seg_off, s_t_out);
   for (int32_t s = 0; s < nseg; ++s)
-    s_t_out[s] = isnan(s_t_out[s]) ? NAN : orc_nvfp4_tensor_scale(s_t_out[s]);
+    s_t_out[s] = isnan(s_t_out[s]) ? NAN : orc_tensor_scale(fmt, s_t_out[s]);
   return status;
+}
+
+/* Effective block scale of scale byte sc: s_t * dec(b) for the E4M3
+ * formats, 2^(sc - 127) for MXFP4. */
+static double block_scale(int fmt, uint8_t sc, float st) {
+  return has_tensor_scale(fmt) ? (double)orc_nvfp4_block_scale(sc, st) : (double)orc_mxfp4_block_scale(sc);
 }
 
 static void put_code(uint8_t* codes, int64_t i, int nib) {
@@ -272,20 +306,21 @@ static void put_bit(uint8_t* bits, int64_t i, int b) {
 static int get_bit(const uint8_t* bits, int64_t i) { return (bits[i >> 3] >> (i & 7)) & 1; }
 
 /* Quantize rows [row_begin, row_end) with RTN (mode 0) or SR (mode 1).
- * NVFP4 takes the per-segment s_t (from orc_segment_scales); MXFP4 ignores
- * s_t.  Writes the codes, the scale bytes and, if bits != NULL, the
+ * NVFP4 and the uniform grid take the per-segment s_t (from
+ * orc_segment_scales); MXFP4 ignores s_t.  Writes the codes, the scale bytes and, if bits != NULL, the
  * guidance bits of those rows (arrays are full-tensor sized). */
 int orc_quantize_rows(int fmt, int mode, const uint16_t* x, int64_t rows, int64_t cols,
                       int32_t nseg, const int64_t* seg_off, const float* s_t, uint64_t seed,
                       int64_t row_begin, int64_t row_end, uint8_t* codes, uint8_t* scales,
                       uint8_t* bits) {
-  const int block = fmt == ORC_NVFP4 ? 16 : 32;
+  const int block = block_of(fmt);
+  const double* V = grid_of(fmt);
   const int64_t nblk_row = cols / block;
   int status = 0;
   (void)rows;
   for (int64_t r = row_begin; r < row_end; ++r) {
-    float st = fmt == ORC_NVFP4 ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
-    if (fmt == ORC_NVFP4 && isnan(st)) status |= ORC_NONFINITE;
+    float st = has_tensor_scale(fmt) ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
+    if (has_tensor_scale(fmt) && isnan(st)) status |= ORC_NONFINITE;
     for (int64_t b = 0; b < nblk_row; ++b) {
       const int64_t base = r * cols + b * block;
       float bamax = 0.0f;
@@ -298,9 +333,9 @@ int orc_quantize_rows(int fmt, int mode, const uint16_t* x, int64_t rows, int64_
       if (bad) status |= ORC_NONFINITE;
       uint8_t sc;
       double S;
-      if (fmt == ORC_NVFP4) {
-        sc = (isnan(st) || bad) ? 0 : orc_nvfp4_block_scale_code(bamax, st);
-        S = (isnan(st) || bad) ? 0.0 : (double)orc_nvfp4_block_scale(sc, st);
+      if (has_tensor_scale(fmt)) {
+        sc = (isnan(st) || bad) ? 0 : orc_block_scale_code(fmt, bamax, st);
+        S = (isnan(st) || bad) ? 0.0 : block_scale(fmt, sc, st);
       } else {
         int e = orc_e8m0_exponent(bamax);
         sc = (uint8_t)(e + 127);
@@ -313,7 +348,7 @@ int orc_quantize_rows(int fmt, int mode, const uint16_t* x, int64_t rows, int64_
         int m3 = 0;
         if (!bad) {
           double ax = bf16_abs(h);
-          m3 = mode == ORC_SR ? orc_sr_m3(ax, S, orc_sr_uniform24((uint64_t)i, seed)) : orc_rtn_m3(ax, S);
+          m3 = mode == ORC_SR ? sr_on(V, ax, S, orc_sr_uniform24((uint64_t)i, seed)) : rtn_on(V, ax, S);
         }
         put_code(codes, i, (bf16_sign(h) << 3) | m3);
         if (bits) put_bit(bits, i, m3 & 1);
@@ -330,16 +365,17 @@ int orc_quantize_guided_rows(int fmt, const uint16_t* x, int64_t rows, int64_t c
                              int32_t nseg, const int64_t* seg_off, const uint8_t* rec_scales,
                              const float* rec_s_t, const uint8_t* rec_bits, int64_t row_begin,
                              int64_t row_end, uint8_t* codes) {
-  const int block = fmt == ORC_NVFP4 ? 16 : 32;
+  const int block = block_of(fmt);
+  const double* V = grid_of(fmt);
   const int64_t nblk_row = cols / block;
   int status = 0;
   (void)rows;
   for (int64_t r = row_begin; r < row_end; ++r) {
-    float st = fmt == ORC_NVFP4 ? rec_s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
+    float st = has_tensor_scale(fmt) ? rec_s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
     for (int64_t b = 0; b < nblk_row; ++b) {
       const int64_t base = r * cols + b * block;
       uint8_t sc = rec_scales[r * nblk_row + b];
-      double S = fmt == ORC_NVFP4 ? (double)orc_nvfp4_block_scale(sc, st) : (double)orc_mxfp4_block_scale(sc);
+      double S = block_scale(fmt, sc, st);
       int bad = 0;
       for (int k = 0; k < block; ++k)
         if (!bf16_is_finite(x[base + k])) bad = 1;
@@ -347,7 +383,7 @@ int orc_quantize_guided_rows(int fmt, const uint16_t* x, int64_t rows, int64_t c
       for (int k = 0; k < block; ++k) {
         const int64_t i = base + k;
         uint16_t h = x[i];
-        int m3 = bad ? 0 : orc_guided_m3(bf16_abs(h), S, get_bit(rec_bits, i));
+        int m3 = bad ? 0 : guided_on(V, bf16_abs(h), S, get_bit(rec_bits, i));
         put_code(codes, i, (bf16_sign(h) << 3) | m3);
       }
     }
@@ -360,17 +396,18 @@ int orc_quantize_guided_rows(int fmt, const uint16_t* x, int64_t rows, int64_t c
 void orc_dequantize_rows(int fmt, const uint8_t* codes, const uint8_t* scales, const float* s_t,
                          int64_t rows, int64_t cols, int32_t nseg, const int64_t* seg_off,
                          int64_t row_begin, int64_t row_end, float* out) {
-  const int block = fmt == ORC_NVFP4 ? 16 : 32;
+  const int block = block_of(fmt);
+  const double* V = grid_of(fmt);
   const int64_t nblk_row = cols / block;
   (void)rows;
   for (int64_t r = row_begin; r < row_end; ++r) {
-    float st = fmt == ORC_NVFP4 ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
+    float st = has_tensor_scale(fmt) ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
     for (int64_t c = 0; c < cols; ++c) {
       const int64_t i = r * cols + c;
       uint8_t sc = scales[r * nblk_row + c / block];
-      double S = fmt == ORC_NVFP4 ? (double)orc_nvfp4_block_scale(sc, st) : (double)orc_mxfp4_block_scale(sc);
+      double S = block_scale(fmt, sc, st);
       int nib = get_code(codes, i);
-      float mag = (float)(kE2M1[nib & 7] * S);
+      float mag = (float)(V[nib & 7] * S);
       out[i] = (nib & 8) ? -mag : mag;
     }
   }
@@ -407,17 +444,18 @@ void orc_f32_to_bf16_array(const float* v, int64_t n, uint16_t* out) {
 void orc_rtn_with_scales_rows(int fmt, const uint16_t* x, int64_t rows, int64_t cols, int32_t nseg,
                               const int64_t* seg_off, const uint8_t* scales, const float* s_t,
                               int64_t row_begin, int64_t row_end, uint8_t* codes) {
-  const int block = fmt == ORC_NVFP4 ? 16 : 32;
+  const int block = block_of(fmt);
+  const double* V = grid_of(fmt);
   const int64_t nblk_row = cols / block;
   (void)rows;
   for (int64_t r = row_begin; r < row_end; ++r) {
-    float st = fmt == ORC_NVFP4 ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
+    float st = has_tensor_scale(fmt) ? s_t[segment_of_row(seg_off, nseg, r)] : 0.0f;
     for (int64_t c = 0; c < cols; ++c) {
       const int64_t i = r * cols + c;
       uint8_t sc = scales[r * nblk_row + c / block];
-      double S = fmt == ORC_NVFP4 ? (double)orc_nvfp4_block_scale(sc, st) : (double)orc_mxfp4_block_scale(sc);
+      double S = block_scale(fmt, sc, st);
       uint16_t h = x[i];
-      put_code(codes, i, (bf16_sign(h) << 3) | orc_rtn_m3(bf16_abs(h), S));
+      put_code(codes, i, (bf16_sign(h) << 3) | rtn_on(V, bf16_abs(h), S));
     }
   }
 }

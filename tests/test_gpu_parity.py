@@ -310,6 +310,28 @@ def test_capture_batched_parity(fmt, L, keep):
         assert torch.equal(g, out.codes[L - 1])
 
 
+def test_capture_batched_large_layers_per_layer_path():
+    """Layers of 2^27 elements take the per-layer launch path inside the
+    batched call: per layer the same bytes as tf4_quantize_capture, and
+    sampled rows of the middle layer against the oracle."""
+    rows, cols, L, keep = 8192, 16384, 3, 2
+    xs = [W.random_bf16((rows, cols), seed=70 + i, device=DEV, outlier_frac=0.001) for i in range(L)]
+    out = B.tf4_quantize_capture_batched(xs, keep=keep)
+    assert B.read_status(xs[0].device) == 0
+    for i, x in enumerate(xs):
+        ref = B.tf4_quantize_capture(x, guidance=i >= L - keep)
+        assert torch.equal(out.codes[i], ref.codes) and torch.equal(out.scales[i].reshape(-1), ref.scales.reshape(-1))
+        assert torch.equal(out.s_t[i:i + 1].view(torch.int32), ref.s_t.view(torch.int32))
+        if i >= L - keep:
+            assert torch.equal(out.info_bits[i - (L - keep)], ref.bits)
+    x1 = W.bf16_bits(xs[1])
+    for r0 in (0, 4093, rows - 3):
+        r = O.quantize(x1, O.NVFP4, bits=True, s_t=host(out.s_t[1:2]), row_range=(r0, r0 + 3))
+        lo, hi = r0 * cols, (r0 + 3) * cols
+        assert_same("codes rows", host(out.codes[1])[lo // 2:hi // 2], r["codes"][lo // 2:hi // 2])
+        assert_same("bits rows", host(out.info_bits[0])[lo // 8:hi // 8], r["bits"][lo // 8:hi // 8])
+
+
 @pytest.mark.parametrize("shape", [(1, 16), (3, 48), (64, 1024), (5, 16 * 33)])
 def test_pack_unpack_parity(shape):
     rows, cols = shape
