@@ -509,7 +509,11 @@ CALL_BYTES = {
     ("nvfp4", "guided_fq_f32"): 6.1875, ("nvfp4", "guided_fq_bf16"): 4.1875,
     ("mxfp4", "guided_fq_f32"): 6.15625, ("mxfp4", "guided_fq_bf16"): 4.15625,
     ("nvfp4", "mismatch"): 2.5625, ("mxfp4", "mismatch"): 2.53125,
+    # a stack of layers captured with guidance kept for the deeper half
+    ("nvfp4", "capture_stack_half_kept"): 4.625, ("mxfp4", "capture_stack_half_kept"): 2.59375,
 }
+# the uniform grid uses NVFP4's container: same bytes per element
+CALL_BYTES.update({("ufp4", c): v for (f, c), v in list(CALL_BYTES.items()) if f == "nvfp4"})
 
 
 def run_suite(args):
@@ -574,6 +578,37 @@ def run_suite(args):
         fq_and_diag(name, "nvfp4", q, x, xt)
         del q, g, out, bits, mant, qr
 
+    def uf_calls(name, x, xt, seg=None):
+        n = x.numel()
+        U = B.UFP4
+        q = B.tf4_quantize_capture(x, fmt=U, seg_off=seg)
+        g = torch.empty_like(q.codes)
+        out = torch.empty(x.shape, dtype=torch.float32, device=dev)
+        qr = B.tf4_quantize_rtn(x, fmt=U, seg_off=seg)
+        record(name, "ufp4", "rtn", n, timed(lambda: B.tf4_quantize_rtn(x, fmt=U, seg_off=seg, out=qr)))
+        record(name, "ufp4", "capture", n, timed(lambda: B.tf4_quantize_capture(x, fmt=U, seg_off=seg, out=q)))
+        record(name, "ufp4", "guided", n, timed(lambda: B.tf4_quantize_guided(xt, q, out=g)))
+        record(name, "ufp4", "sr", n, timed(lambda: B.tf4_quantize_sr(x, 4, fmt=U, seg_off=seg, out=qr)))
+        record(name, "ufp4", "dequant", n, timed(lambda: B.tf4_dequantize(q, out=out)))
+        fq_and_diag(name, "ufp4", q, x, xt)
+        del q, g, out, qr
+
+    def stack_calls(name, xs, fmt, fname):
+        """A stack of layers captured (deeper half keeps guidance): one
+        batched call against one capture call per layer."""
+        L, keep = len(xs), len(xs) // 2
+        n = sum(x.numel() for x in xs)
+        ob = B.tf4_quantize_capture_batched(xs, fmt=fmt, keep=keep)
+        per = [B.tf4_quantize_capture(x, fmt=fmt, guidance=i >= L - keep) for i, x in enumerate(xs)]
+
+        def per_layer():
+            for i, x in enumerate(xs):
+                B.tf4_quantize_capture(x, fmt=fmt, guidance=i >= L - keep, out=per[i])
+        record(name, fname, "capture_stack_half_kept", n, timed(per_layer), launch="per_layer")
+        record(name, fname, "capture_stack_half_kept", n,
+               timed(lambda: B.tf4_quantize_capture_batched(xs, fmt=fmt, keep=keep, out=ob)), launch="batched")
+        del ob, per
+
     def mx_calls(name, x, xt):
         if x.shape[1] % 32:
             return
@@ -593,14 +628,21 @@ def run_suite(args):
     w = W.activation_outliers(dev)
     nv_calls("activation_outliers 4096x2048", w["x"], w["x_train"])
     mx_calls("activation_outliers 4096x2048", w["x"], w["x_train"])
+    uf_calls("activation_outliers 4096x2048", w["x"], w["x_train"])
     del w
+    xs = [W.random_bf16((4096, 2048), seed=300 + i, device=dev, outlier_frac=0.001) for i in range(40)]
+    stack_calls("40 layers of 4096x2048", xs, B.NVFP4, "nvfp4")
+    stack_calls("40 layers of 4096x2048", xs, B.MXFP4, "mxfp4")
+    del xs
     x = W.layer_stack_layer(20, dev)
     xt = W.perturb(x, 1020)
     nv_calls("layer_stack layer 65536x4096", x, xt)
     mx_calls("layer_stack layer 65536x4096", x, xt)
+    uf_calls("layer_stack layer 65536x4096", x, xt)
     del x, xt
     w = W.moe_dispatch(dev)
     nv_calls("moe_dispatch 262144x2048, 128 experts", w["x"], w["x_train"], seg=w["seg_off"])
+    uf_calls("moe_dispatch 262144x2048, 128 experts", w["x"], w["x_train"], seg=w["seg_off"])
     del w
     x = W.weights(dev)
     nv_calls("weights 8192x28672", x, W.perturb(x, 44))

@@ -25,8 +25,10 @@ import torch
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtrace_fp4.so")
 
-NVFP4, MXFP4 = 0, 1
-BLOCK = {NVFP4: 16, MXFP4: 32}
+NVFP4, MXFP4, UFP4 = 0, 1, 2
+BLOCK = {NVFP4: 16, MXFP4: 32, UFP4: 16}
+# formats with an fp32 per-segment tensor scale (and segments, a workspace)
+HAS_TENSOR_SCALE = {NVFP4: True, MXFP4: False, UFP4: True}
 MAX_SEGMENTS = 1024
 DEV_NONFINITE, DEV_TIMEOUT = 1, 2
 
@@ -213,7 +215,7 @@ def sizes(fmt: int, rows: int, cols: int, seg_off=None) -> dict:
 class Quantized:
     codes: torch.Tensor                  # uint8 [rows*cols/2]
     scales: torch.Tensor                 # uint8 [rows, cols/block]
-    s_t: Optional[torch.Tensor]          # float [num_segments] (NVFP4)
+    s_t: Optional[torch.Tensor]          # float [num_segments] (NVFP4, UFP4)
     bits: Optional[torch.Tensor] = None  # uint8 [rows*cols/8] (capture)
     fmt: int = NVFP4
     rows: int = 0
@@ -226,7 +228,8 @@ def _outputs(desc: Desc, device, want_bits: bool, out: Optional[Quantized]):
         return out
     codes = torch.empty(desc.n // 2, dtype=torch.uint8, device=device)
     scales = torch.empty((desc.rows, desc.cols // BLOCK[desc.fmt]), dtype=torch.uint8, device=device)
-    s_t = torch.empty(desc.num_segments, dtype=torch.float32, device=device) if desc.fmt == NVFP4 else None
+    s_t = (torch.empty(desc.num_segments, dtype=torch.float32, device=device) if HAS_TENSOR_SCALE[desc.fmt]
+           else None)
     bits = torch.empty(desc.n // 8, dtype=torch.uint8, device=device) if want_bits else None
     return Quantized(codes, scales, s_t, bits, desc.fmt, desc.rows, desc.cols, desc.seg_off)
 
@@ -282,7 +285,7 @@ def tf4_quantize_capture(x, fmt=NVFP4, seg_off=None, guidance=True, amax_in=None
 class BatchedCapture:
     codes: torch.Tensor            # uint8 [L, rows*cols/2]
     scales: torch.Tensor           # uint8 [L, rows, cols/block]
-    s_t: Optional[torch.Tensor]    # float [L] (NVFP4)
+    s_t: Optional[torch.Tensor]    # float [L] (NVFP4, UFP4)
     info_bits: Optional[torch.Tensor]  # uint8 [keep, rows*cols/8]: the info cache
     fmt: int
     rows: int
@@ -310,7 +313,7 @@ def tf4_quantize_capture_batched(xs, fmt=NVFP4, keep=0, stream=None, out: Option
         n = rows * cols
         out = BatchedCapture(torch.empty((L, n // 2), dtype=torch.uint8, device=dev),
                              torch.empty((L, rows, cols // BLOCK[fmt]), dtype=torch.uint8, device=dev),
-                             torch.empty(L, dtype=torch.float32, device=dev) if fmt == NVFP4 else None,
+                             torch.empty(L, dtype=torch.float32, device=dev) if HAS_TENSOR_SCALE[fmt] else None,
                              torch.empty((keep, n // 8), dtype=torch.uint8, device=dev) if keep else None,
                              fmt, rows, cols, keep)
     ptrs = (ctypes.c_void_p * L)(*[t.data_ptr() for t in x2])

@@ -25,6 +25,17 @@ namespace tf4 {
 
 constexpr int kThreads = 256;
 
+// Formats with an E4M3 block scale and an fp32 tensor scale (16-element
+// blocks, segments): NVFP4 (E2M1 grid) and UFP4 (uniform grid 0..7).
+template <int FMT>
+constexpr bool kE4M3 = FMT != TF4_MXFP4;
+template <int FMT>
+constexpr bool kUni = FMT == TF4_UFP4;
+// Largest grid value (6 on E2M1, 7 on the uniform grid): the block-scale
+// divisor, and 448 times it is the tensor-scale divisor.
+template <bool U>
+constexpr float kGridMax = U ? 7.0f : 6.0f;
+
 // ------------------------------------------------------------- segments
 // One per-tensor-scale segment covering everything (the common case).
 struct Seg1 {
@@ -128,6 +139,30 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float v0, float v1, float v2, flo
   return r;
 }
 
+// Eight fp32 values -> eight uniform-grid nibbles: round |v| to the nearest
+// integer, ties to even (adding 2^23 does exactly that: the sum is rounded
+// once, to a neighbouring integer), saturating at 7; sign bit kept.  Element
+// k in bits [4k, 4k+4).
+__device__ __forceinline__ uint32_t cvt_uni_x8(float v0, float v1, float v2, float v3, float v4, float v5,
+                                               float v6, float v7) {
+  const float v[8] = {v0, v1, v2, v3, v4, v5, v6, v7};
+  uint32_t r = 0u;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const uint32_t t = __float_as_uint(__fadd_rn(fminf(fabsf(v[k]), 7.0f), 0x1p23f));
+    r |= ((t & 7u) | ((__float_as_uint(v[k]) >> 28) & 8u)) << (4 * k);
+  }
+  return r;
+}
+
+// Eight fp32 values -> eight nibbles of the format's grid.
+template <bool U>
+__device__ __forceinline__ uint32_t cvt_grid_x8(float v0, float v1, float v2, float v3, float v4, float v5,
+                                                float v6, float v7) {
+  if constexpr (U) return cvt_uni_x8(v0, v1, v2, v3, v4, v5, v6, v7);
+  else return cvt_e2m1x8(v0, v1, v2, v3, v4, v5, v6, v7);
+}
+
 // Four E2M1 nibbles (16 bits, element k in bits [4k, 4k+4)) -> their values
 // times S, using CUDA's fp4x2 -> half2 conversion (exact: every E2M1 value
 // is an f16 value) and one fp32 multiply each.
@@ -137,6 +172,24 @@ __device__ __forceinline__ float4 decode4(uint32_t c, float S) {
   const float2 f0 = __half22float2(__half2(h0));
   const float2 f1 = __half22float2(__half2(h1));
   return make_float4(__fmul_rn(f0.x, S), __fmul_rn(f0.y, S), __fmul_rn(f1.x, S), __fmul_rn(f1.y, S));
+}
+
+// Four uniform-grid nibbles -> +-RN(k * S); k as fp32 via 2^23 + k - 2^23.
+__device__ __forceinline__ float4 decode4_uni(uint32_t c, float S) {
+  float v[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const uint32_t n = (c >> (4 * e)) & 0xFu;
+    const float k = __fsub_rn(__uint_as_float(0x4B000000u | (n & 7u)), 0x1p23f);
+    v[e] = __uint_as_float(__float_as_uint(__fmul_rn(k, S)) | ((n & 8u) << 28));
+  }
+  return make_float4(v[0], v[1], v[2], v[3]);
+}
+
+template <bool U>
+__device__ __forceinline__ float4 decode4_grid(uint32_t c, float S) {
+  if constexpr (U) return decode4_uni(c, S);
+  else return decode4(c, S);
 }
 
 // m3 & 1 of eight nibbles -> eight bits (nibble k -> bit k).  The masked
@@ -160,13 +213,15 @@ __device__ __forceinline__ float e4m3_decode(uint32_t b) {
   return __uint_as_float(((e + 120u) << 23) | (m << 20));
 }
 
-// NVFP4 per-tensor scale from the segment amax; non-finite amax -> NaN.
+// Per-tensor scale from the segment amax, amax / (448 * grid max)
+// (2688 for E2M1, 3136 for the uniform grid); non-finite amax -> NaN.
+template <bool U = false>
 __device__ __forceinline__ float tensor_scale(float amax, int32_t* status) {
   if (!(amax <= 3.4028234663852886e38f)) {  // Inf or NaN
     if (status) atomicOr(status, TF4_DEV_NONFINITE);
     return __int_as_float(0x7FC00000);
   }
-  const float s = __fdiv_rn(amax, 2688.0f);
+  const float s = __fdiv_rn(amax, 448.0f * kGridMax<U>);
   return s >= 0x1p-126f ? s : 0.0f;
 }
 
@@ -175,40 +230,62 @@ __device__ __forceinline__ bool near_bf16(float v) {
   return ((__float_as_uint(v) + 8u) & 0xFFFFu) < 16u;
 }
 
+// ------------------------------------------------------------ grid values
+// Magnitude of E2M1 code m3 (0..7) as fp32.
+__device__ __forceinline__ float e2m1_value(uint32_t m3) {
+  const uint32_t e = m3 >> 1, m = m3 & 1u;
+  return e ? __uint_as_float(((e + 126u) << 23) | (m << 22)) : (m ? 0.5f : 0.0f);
+}
+
+// Magnitude of code m3 on the format's grid (uniform: m3 itself).
+template <bool U>
+__device__ __forceinline__ float grid_value(uint32_t m3) {
+  if constexpr (U) return (float)m3;
+  else return e2m1_value(m3);
+}
+
+// Midpoint between codes i and i + 1.
+template <bool U>
+__device__ __forceinline__ float grid_mid(int i) {
+  return 0.5f * (grid_value<U>((uint32_t)i) + grid_value<U>((uint32_t)i + 1u));
+}
+
 // ------------------------------------------------- exact per-element paths
 // RTN m3 of |x| on scale S > 0 by exact comparisons.  fmaf(-mu, S, ax) is
 // rounded once, so its sign is the sign of ax - mu*S exactly as long as the
 // difference cannot underflow, which holds for S >= 2^-124; smaller S is
-// rescaled by 2^64 first (exact).  Three-level search over the midpoints
-// {.25,.75,1.25,1.75,2.5,3.5,5}; ">=" at odd-index midpoints and ">" at
-// even-index ones give ties to the even m3.
+// rescaled by 2^64 first (exact).  Three-level search over the 7 midpoints
+// (E2M1: .25,.75,1.25,1.75,2.5,3.5,5; uniform: .5, 1.5, ..., 6.5); ">=" at
+// odd-index midpoints and ">" at even-index ones give ties to the even m3.
+template <bool U = false>
 __device__ __forceinline__ uint32_t rtn_m3_exact(float ax, float S) {
   if (S < 0x1p-100f) {
     ax *= 0x1p64f;
     S *= 0x1p64f;
   }
-  const bool b2 = fmaf(-1.75f, S, ax) >= 0.0f;
-  const float mu = b2 ? 3.5f : 0.75f;
+  const bool b2 = fmaf(-grid_mid<U>(3), S, ax) >= 0.0f;
+  const float mu = b2 ? grid_mid<U>(5) : grid_mid<U>(1);
   const bool b1 = fmaf(-mu, S, ax) >= 0.0f;
-  const float mu3 = b2 ? (b1 ? 5.0f : 2.5f) : (b1 ? 1.25f : 0.25f);
+  const float mu3 = b2 ? (b1 ? grid_mid<U>(6) : grid_mid<U>(4)) : (b1 ? grid_mid<U>(2) : grid_mid<U>(0));
   const bool b0 = fmaf(-mu3, S, ax) > 0.0f;
   return (b2 ? 4u : 0u) | (b1 ? 2u : 0u) | (b0 ? 1u : 0u);
 }
 
 // Guided m3 of |x| on scale S > 0 with recorded bit g (exact comparisons as
-// above): f = number of codewords <= y; y >= 6 -> 7; y a codeword -> f;
-// otherwise the neighbour (f or f+1) whose m3 & 1 == g.
+// above): f = number of nonzero codewords <= y; y >= grid max -> 7; y a
+// codeword -> f; otherwise the neighbour (f or f+1) whose m3 & 1 == g.
+template <bool U = false>
 __device__ __forceinline__ uint32_t guided_m3_exact(float ax, float S, uint32_t g) {
   if (S < 0x1p-100f) {
     ax *= 0x1p64f;
     S *= 0x1p64f;
   }
-  const float d2 = fmaf(-2.0f, S, ax);
+  const float d2 = fmaf(-grid_value<U>(4), S, ax);
   const bool p2 = d2 >= 0.0f;
-  const float v1 = p2 ? 4.0f : 1.0f;
+  const float v1 = p2 ? grid_value<U>(6) : grid_value<U>(2);
   const float d1 = fmaf(-v1, S, ax);
   const bool p1 = d1 >= 0.0f;
-  const float v0 = p2 ? (p1 ? 6.0f : 3.0f) : (p1 ? 1.5f : 0.5f);
+  const float v0 = p2 ? (p1 ? grid_value<U>(7) : grid_value<U>(5)) : (p1 ? grid_value<U>(3) : grid_value<U>(1));
   const float d0 = fmaf(-v0, S, ax);
   const bool p0 = d0 >= 0.0f;
   const uint32_t f = (p2 ? 4u : 0u) | (p1 ? 2u : 0u) | (p0 ? 1u : 0u);
@@ -238,23 +315,20 @@ __device__ __forceinline__ uint32_t philox_w0(uint64_t idx, uint64_t seed) {
   return c0;
 }
 
-// Magnitude of E2M1 code m3 (0..7) as fp32.
-__device__ __forceinline__ float e2m1_value(uint32_t m3) {
-  const uint32_t e = m3 >> 1, m = m3 & 1u;
-  return e ? __uint_as_float(((e + 126u) << 23) | (m << 22)) : (m ? 0.5f : 0.0f);
-}
-
 // SR m3 of |x| on scale S > 0 with a 24-bit uniform r.  Every product of a
 // codeword (<= 4 significant bits) and S (24 bits) is exact in double, and
-// so are r * gap * S (<= 48 bits) and ax - V_lo * S (within a factor two of
-// each other, or V_lo = 0), so all comparisons are exact.
+// so are r * gap * S (<= 48 bits) and ax - V_lo * S (V_lo = 0, or
+// ax >= S/2 ends at or above bit 2^-8 S while V_lo * S ends at or above
+// 2^-25 S and both are below 2^4 S), so all comparisons are exact.
+template <bool U = false>
 __device__ __forceinline__ uint32_t sr_m3_exact(float axf, float Sf, uint32_t r24) {
   const double ax = axf, S = Sf;
-  if (ax >= 6.0 * S) return 7u;
+  if (ax >= (double)kGridMax<U> * S) return 7u;
   // f = number of nonzero codewords <= y
-  const uint32_t f = (0.5 * S <= ax) + (1.0 * S <= ax) + (1.5 * S <= ax) + (2.0 * S <= ax) +
-                     (3.0 * S <= ax) + (4.0 * S <= ax) + (6.0 * S <= ax);
-  const double vlo = (double)e2m1_value(f), vhi = (double)e2m1_value(f + 1u);
+  uint32_t f = 0u;
+#pragma unroll
+  for (uint32_t j = 1; j < 8; ++j) f += (double)grid_value<U>(j) * S <= ax;
+  const double vlo = (double)grid_value<U>(f), vhi = (double)grid_value<U>(f + 1u);
   if (vlo * S == ax) return f;
   const double lhs = (double)r24 * (vhi - vlo) * S;
   const double rhs = 16777216.0 * (ax - vlo * S);
@@ -269,7 +343,19 @@ __device__ __forceinline__ uint32_t sr_m3_exact(float axf, float Sf, uint32_t r2
 // exact arithmetic on y (Sterbenz subtraction, power-of-two scaling).  With
 // an approximate y, |t - T_exact| < 64, so a uniform within 128 of t is
 // flagged `amb` for the exact test.  Returns the chosen codeword value.
+template <bool U = false>
 __device__ __forceinline__ float sr_pick(float y, uint32_t r24, bool margin, bool& amb) {
+  if constexpr (U) {
+    // uniform grid: lo = floor(y), gap 1; y - lo is exact (Sterbenz), so
+    // t = 2^24 (y - lo) is exact arithmetic on y; |y - y_exact| < 2^-17.5
+    // for y < 7.5, so |t - T_exact| < 96
+    const float vlo = floorf(y);
+    const float t = __fmul_rn(__fsub_rn(y, vlo), 0x1p24f);
+    const float rf = __uint2float_rn(r24);
+    amb = margin && fabsf(rf - t) <= 128.0f;
+    const float v = rf < t ? __fadd_rn(vlo, 1.0f) : vlo;
+    return fminf(v, 7.0f);
+  }
   const uint32_t yb = __float_as_uint(y);
   const bool ge1 = y >= 1.0f;
   const float vlo = ge1 ? __uint_as_float(yb & 0xFFC00000u) : (y >= 0.5f ? 0.5f : 0.0f);
@@ -289,7 +375,7 @@ __device__ __forceinline__ float sr_pick(float y, uint32_t r24, bool margin, boo
 // hence exact and deterministic) into ws[seg].  The last CTA to finish
 // (ticket counter at ws[nseg]) turns the maxima into the outputs, then
 // resets ws to zero for the next call.
-template <class SEG>
+template <class SEG, bool U = false>
 __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, int64_t nblocks,
                                                    SEG seg, uint32_t* ws, float* s_t_out,
                                                    float* amax_out, int32_t* status) {
@@ -355,7 +441,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, 
       amax_out[k] = amax;
       if (!(amax <= 3.4028234663852886e38f) && status) atomicOr(status, TF4_DEV_NONFINITE);
     }
-    if (s_t_out) s_t_out[k] = tensor_scale(amax, status);
+    if (s_t_out) s_t_out[k] = tensor_scale<U>(amax, status);
   }
   if (tid == 0) ws[seg.count()] = 0u;
 }
@@ -392,12 +478,11 @@ constexpr int kCand = 9;
 // candidate k -> ulp offset 0, +1, -1, +2, -2, ...
 __device__ __forceinline__ int cand_offset(int k) { return (k & 1) ? ((k + 1) >> 1) : -(k >> 1); }
 
-// Decision points: E2M1 midpoints (i = 0..6, tie -> upper iff i odd) or the
-// nonzero codewords (i = 0..6 -> V[i+1]).
-template <bool MIDPOINTS>
+// Decision points: the grid's midpoints (i = 0..6, tie -> upper iff i odd)
+// or its nonzero codewords (i = 0..6 -> V[i+1]).
+template <bool U, bool MIDPOINTS>
 __device__ __forceinline__ float decision_point(int i) {
-  return MIDPOINTS ? 0.5f * (e2m1_value((uint32_t)i) + e2m1_value((uint32_t)i + 1u))
-                   : e2m1_value((uint32_t)i + 1u);
+  return MIDPOINTS ? grid_mid<U>(i) : grid_value<U>((uint32_t)i + 1u);
 }
 
 template <bool RZ>
@@ -411,21 +496,21 @@ __device__ __forceinline__ float mul(float a, float b) {
 // loop stays uniform: toward zero if every class has a safe multiplier in
 // that mode, else to nearest if every class has one there, else the mode
 // with more safe classes (the others take the exact path).
-template <bool MIDPOINTS, bool CODE_TABLE = MIDPOINTS>
+template <bool U, bool MIDPOINTS, bool CODE_TABLE = MIDPOINTS>
 __device__ void build_tables(float st, SegTables& t) {
   const int tid = threadIdx.x;
   __syncthreads();  // the previous piece is done with t
   const bool fast = st >= 0x1p-90f && st <= 0x1p100f;
   if (tid < 8) t.mask[tid] = (1u << (2 * kCand)) - 1u;
   if (CODE_TABLE) {
-    const int E0 = fast ? (int)((__float_as_uint(__fmul_rn(st, 2688.0f)) >> 23) & 0xFFu) - 2 : 0;
+    const int E0 = fast ? (int)((__float_as_uint(__fmul_rn(st, 448.0f * kGridMax<U>)) >> 23) & 0xFFu) - 2 : 0;
     if (tid == 0) {
       t.E0 = E0;
       t.fast = fast && E0 >= 4;
     }
     if (fast && E0 >= 4 && tid < 128) {
       const float bam = __uint_as_float(((uint32_t)E0 << 23) | ((uint32_t)tid << 16));
-      t.code[tid] = (uint8_t)e4m3_encode(__fdiv_rn(__fdiv_rn(bam, 6.0f), st));
+      t.code[tid] = (uint8_t)e4m3_encode(__fdiv_rn(__fdiv_rn(bam, kGridMax<U>), st));
     }
   } else if (tid == 0) {
     t.fast = fast;
@@ -434,7 +519,7 @@ __device__ void build_tables(float st, SegTables& t) {
   if (fast && tid < 8 * 28) {
     const int c = tid / 28, r = tid % 28, i = r >> 2, o = (r & 3) - 1;
     const float Sc = __fmul_rn(st, 1.0f + 0.125f * (float)c);
-    const float pt = decision_point<MIDPOINTS>(i);
+    const float pt = decision_point<U, MIDPOINTS>(i);
     const float P = __fmul_rn(pt, Sc);
     const float v = __uint_as_float((uint32_t)((int)(__float_as_uint(P) >> 16) + o) << 16);
     const float e = fmaf(-pt, Sc, v);  // exact sign: Sc >= 2^-96
@@ -478,10 +563,10 @@ __device__ __forceinline__ float block_rho(float rho_c, uint32_t e_b) {
   return __uint_as_float(__float_as_uint(rho_c) + (uint32_t)((7 - (int)e_b) << 23));
 }
 
-// Eight bf16 (four words) times rho -> eight E2M1 nibbles (signed, RNE).
-template <bool RZ = false>
+// Eight bf16 (four words) times rho -> eight grid nibbles (signed, RNE).
+template <bool RZ = false, bool U = false>
 __device__ __forceinline__ uint32_t cvt_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r) {
-  return cvt_e2m1x8(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r),
+  return cvt_grid_x8<U>(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r),
                     mul<RZ>(bf_hi(w1), r), mul<RZ>(bf_lo(w2), r), mul<RZ>(bf_hi(w2), r),
                     mul<RZ>(bf_lo(w3), r), mul<RZ>(bf_hi(w3), r));
 }
@@ -502,8 +587,9 @@ struct QuantArgs {
   int32_t* status;
 };
 
-// One NVFP4 block (16 bf16 in w[0..7]) -> code words, scale byte, flags.
-template <int MODE, bool RZ>
+// One block of an E4M3-scaled format (16 bf16 in w[0..7]; E2M1 grid for
+// NVFP4, uniform grid if U) -> code words, scale byte, flags.
+template <bool U, int MODE, bool RZ>
 __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, const SegTables& t,
                                             int64_t blk, uint64_t seed, uint32_t& c0, uint32_t& c1,
                                             uint32_t& sc, bool& bad) {
@@ -518,8 +604,8 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
       if (rho != 0.0f) {
         const float r = block_rho(rho, sc >> 3);
         if (MODE != kSR) {
-          c0 = cvt_words<RZ>(w[0], w[1], w[2], w[3], r);
-          c1 = cvt_words<RZ>(w[4], w[5], w[6], w[7], r);
+          c0 = cvt_words<RZ, U>(w[0], w[1], w[2], w[3], r);
+          c1 = cvt_words<RZ, U>(w[4], w[5], w[6], w[7], r);
           return;
         } else {
           // stochastic rounding on the codeword-safe product; rare
@@ -532,12 +618,12 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
             const float ax = __uint_as_float((h & 0x7FFFu) << 16);
             const uint32_t r24 = philox_w0((uint64_t)blk * 16u + k, seed) >> 8;
             bool amb;
-            float val = sr_pick(mul<RZ>(ax, r), r24, true, amb);
-            if (amb) val = e2m1_value(sr_m3_exact(ax, S, r24));
+            float val = sr_pick<U>(mul<RZ>(ax, r), r24, true, amb);
+            if (amb) val = grid_value<U>(sr_m3_exact<U>(ax, S, r24));
             v[k] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
           }
-          c0 = cvt_e2m1x8(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
-          c1 = cvt_e2m1x8(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+          c0 = cvt_grid_x8<U>(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+          c1 = cvt_grid_x8<U>(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
           return;
         }
       }
@@ -550,7 +636,7 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
   sc = 0;
   if (st > 0.0f) {  // st == 0: zero segment; NaN: non-finite segment
     const float bamax = __uint_as_float(mb << 16);
-    sc = e4m3_encode(__fdiv_rn(__fdiv_rn(bamax, 6.0f), st));
+    sc = e4m3_encode(__fdiv_rn(__fdiv_rn(bamax, kGridMax<U>), st));
     S = __fmul_rn(st, e4m3_decode(sc));
   }
   uint32_t out[2] = {0u, 0u};
@@ -561,9 +647,9 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
     uint32_t m3 = 0;
     if (S > 0.0f) {
       if (MODE == kSR)
-        m3 = sr_m3_exact(ax, S, philox_w0((uint64_t)blk * 16u + k, seed) >> 8);
+        m3 = sr_m3_exact<U>(ax, S, philox_w0((uint64_t)blk * 16u + k, seed) >> 8);
       else
-        m3 = rtn_m3_exact(ax, S);
+        m3 = rtn_m3_exact<U>(ax, S);
     }
     out[k >> 3] |= (((h >> 15) << 3) | m3) << (4 * (k & 7));
   }
@@ -622,23 +708,24 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
   const int64_t b0 = cta_begin(ci, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(ci + 1, gridDim.x, a.nblocks);
   const int tid = threadIdx.x;
-  if (FMT == TF4_NVFP4 && a.st_from_amax && blockIdx.x == 0 && a.s_t_out)
-    for (int k = tid; k < seg.count(); k += kThreads) a.s_t_out[k] = tensor_scale(a.st_src[k], a.status);
+  constexpr bool UG = kUni<FMT>;
+  if (kE4M3<FMT> && a.st_from_amax && blockIdx.x == 0 && a.s_t_out)
+    for (int k = tid; k < seg.count(); k += kThreads) a.s_t_out[k] = tensor_scale<UG>(a.st_src[k], a.status);
   int64_t hi = b1;
   while (hi > b0) {
     const int s = seg.find(hi - 1);
     const int64_t lo = max(b0, seg.start(s));
     float st = 0.0f;
-    if constexpr (FMT == TF4_NVFP4) {
-      st = a.st_from_amax ? tensor_scale(a.st_src[s], nullptr) : a.st_src[s];
-      if (MODE != kSR) build_tables<true>(st, tb);
-      else build_tables<false, true>(st, tb);
+    if constexpr (kE4M3<FMT>) {
+      st = a.st_from_amax ? tensor_scale<UG>(a.st_src[s], nullptr) : a.st_src[s];
+      if (MODE != kSR) build_tables<UG, true>(st, tb);
+      else build_tables<UG, false, true>(st, tb);
     }
     const uint4* xs = seg.xptr(s, a.x);
     uint8_t* bits = seg.bitsptr(s, a.bits);
     const int64_t n = hi - lo;
     for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
-      if constexpr (FMT == TF4_NVFP4) {
+      if constexpr (kE4M3<FMT>) {
         uint32_t w[U][8];
         int64_t blk[U];
 #pragma unroll
@@ -658,9 +745,9 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
           if (valid) {
             uint32_t c0, c1, sc;
             if (tb.rz)
-              nvfp4_block<MODE, true>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
+              nvfp4_block<UG, MODE, true>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
             else
-              nvfp4_block<MODE, false>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
+              nvfp4_block<UG, MODE, false>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
             reinterpret_cast<uint2*>(a.codes)[blk[u]] = make_uint2(c0, c1);
             a.scales[blk[u]] = (uint8_t)sc;
             if (MODE == kCAPTURE && bits)
@@ -738,7 +825,7 @@ __device__ __forceinline__ uint32_t spread_bits(uint32_t b) {
 // w0..w3) whose m3 & 1 differs from the recorded bit (mm: mismatch bits at
 // nibble bit 0): keep exact codewords and the saturated top, otherwise step
 // to the other neighbour.
-template <bool RZ>
+template <bool RZ, bool U = false>
 __device__ __forceinline__ uint32_t fix_mismatches(uint32_t c, uint32_t mm, uint32_t w0, uint32_t w1,
                                                    uint32_t w2, uint32_t w3, float r) {
   while (mm) {
@@ -748,8 +835,8 @@ __device__ __forceinline__ uint32_t fix_mismatches(uint32_t c, uint32_t mm, uint
     const uint32_t h = (e & 1) ? (wsel >> 16) : (wsel & 0xFFFFu);
     const float y = mul<RZ>(__uint_as_float((h & 0x7FFFu) << 16), r);
     const uint32_t n = (c >> (4 * e)) & 7u;
-    const float v = e2m1_value(n);
-    if (!(y == v || (n == 7u && y >= 6.0f))) {
+    const float v = grid_value<U>(n);
+    if (!(y == v || (n == 7u && y >= kGridMax<U>))) {
       const uint32_t n2 = y > v ? n + 1u : n - 1u;
       c = (c & ~(7u << (4 * e))) | (n2 << (4 * e));
     }
@@ -759,7 +846,8 @@ __device__ __forceinline__ uint32_t fix_mismatches(uint32_t c, uint32_t mm, uint
 
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
-  constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;  // elements per block
+  constexpr bool UG = kUni<FMT>;
+  constexpr int BE = kE4M3<FMT> ? 16 : 32;  // elements per block
   constexpr int NW = BE / 2;                       // bf16 pair words per block
   constexpr int NQ = BE / 8;                       // code words per block
   __shared__ SegTables tb;
@@ -771,9 +859,9 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
     const int s = seg.find(lo);
     const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
     float st = 0.0f;
-    if constexpr (FMT == TF4_NVFP4) {
+    if constexpr (kE4M3<FMT>) {
       st = a.rec_s_t[s];
-      build_tables<false>(st, tb);
+      build_tables<UG, false>(st, tb);
     }
     const int64_t n = hi - lo;
     constexpr int U = 2;  // blocks per lane per iteration
@@ -790,7 +878,7 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
             w[u][4 * q] = p.x; w[u][4 * q + 1] = p.y; w[u][4 * q + 2] = p.z; w[u][4 * q + 3] = p.w;
           }
           sc[u] = a.rec_scales[blk];
-          if constexpr (FMT == TF4_NVFP4) g[u] = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
+          if constexpr (kE4M3<FMT>) g[u] = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
           else g[u] = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
         }
       }
@@ -803,26 +891,27 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
           bad = block_absmax_bits(w[u]) >= 0x7F80u;
           uint32_t c[NQ];
           float r = 0.0f;
-          if constexpr (FMT == TF4_NVFP4) {
+          if constexpr (kE4M3<FMT>) {
             if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu) r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
             if (tb.rho[sc[u] & 7u] == 0.0f) r = 0.0f;
           } else {
             if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);  // 2^-(sc-127), exact
           }
           if (r != 0.0f) {
-            const bool rz = FMT == TF4_NVFP4 && tb.rz;
+            const bool rz = kE4M3<FMT> && tb.rz;
 #pragma unroll
             for (int q = 0; q < NQ; ++q) {
               const uint32_t* wq = &w[u][4 * q];
-              c[q] = rz ? cvt_words<true>(wq[0], wq[1], wq[2], wq[3], r) : cvt_words<false>(wq[0], wq[1], wq[2], wq[3], r);
+              c[q] = rz ? cvt_words<true, UG>(wq[0], wq[1], wq[2], wq[3], r)
+                        : cvt_words<false, UG>(wq[0], wq[1], wq[2], wq[3], r);
               const uint32_t mm = (c[q] ^ spread_bits(g[u] >> (8 * q))) & 0x11111111u;
               if (mm)
-                c[q] = rz ? fix_mismatches<true>(c[q], mm, wq[0], wq[1], wq[2], wq[3], r)
-                          : fix_mismatches<false>(c[q], mm, wq[0], wq[1], wq[2], wq[3], r);
+                c[q] = rz ? fix_mismatches<true, UG>(c[q], mm, wq[0], wq[1], wq[2], wq[3], r)
+                          : fix_mismatches<false, UG>(c[q], mm, wq[0], wq[1], wq[2], wq[3], r);
             }
           } else {
             float S;
-            if constexpr (FMT == TF4_NVFP4) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
+            if constexpr (kE4M3<FMT>) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
             else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
 #pragma unroll
             for (int q = 0; q < NQ; ++q) c[q] = 0u;
@@ -830,11 +919,11 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
             for (int e = 0; e < BE; ++e) {
               const uint32_t h = (e & 1) ? (w[u][e >> 1] >> 16) : (w[u][e >> 1] & 0xFFFFu);
               const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-              const uint32_t m3 = S > 0.0f ? guided_m3_exact(ax, S, (g[u] >> e) & 1u) : 0u;
+              const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
               c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
             }
           }
-          if constexpr (FMT == TF4_NVFP4) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
+          if constexpr (kE4M3<FMT>) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
           else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);
         }
         report_bad(bad, a.status);
@@ -861,9 +950,12 @@ struct GuidedFqArgs {
   int32_t* status;
 };
 
-// Four bf16 (two words) times r -> four E2M1 nibbles (16 bits).
-template <bool RZ>
+// Four bf16 (two words) times r -> four grid nibbles (16 bits).
+template <bool RZ, bool U = false>
 __device__ __forceinline__ uint32_t cvt_words4(uint32_t w0, uint32_t w1, float r) {
+  if constexpr (U)
+    return cvt_uni_x8(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r), mul<RZ>(bf_hi(w1), r),
+                      0.0f, 0.0f, 0.0f, 0.0f);
   uint32_t c;
   asm("{\n\t.reg .b8 q0, q1;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
@@ -877,7 +969,8 @@ __device__ __forceinline__ uint32_t cvt_words4(uint32_t w0, uint32_t w1, float r
 
 template <int FMT, class SEG, bool BF16>
 __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg) {
-  constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;
+  constexpr bool UG = kUni<FMT>;
+  constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int QPB = BE / 4;  // quads per block
   constexpr int U = 2;         // quads per lane per iteration
   __shared__ SegTables tb;
@@ -889,9 +982,9 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
     const int s = seg.find(lo);
     const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
     float st = 0.0f;
-    if constexpr (FMT == TF4_NVFP4) {
+    if constexpr (kE4M3<FMT>) {
       st = a.rec_s_t[s];
-      build_tables<false>(st, tb);
+      build_tables<UG, false>(st, tb);
     }
     const int64_t q0 = lo * QPB, q1 = hi * QPB;
     for (int64_t qb = q0; qb < q1; qb += (int64_t)U * kThreads) {
@@ -915,7 +1008,7 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
           bad = max(m & 0xFFFFu, m >> 16) >= 0x7F80u;
           float r = 0.0f, S;
           bool rz = false;
-          if constexpr (FMT == TF4_NVFP4) {
+          if constexpr (kE4M3<FMT>) {
             S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
             if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu && tb.rho[sc[u] & 7u] != 0.0f) {
               r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
@@ -928,22 +1021,23 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
           const uint32_t w0 = xv[u].x, w1 = xv[u].y;
           uint32_t c;
           if (r != 0.0f) {
-            c = rz ? cvt_words4<true>(w0, w1, r) : cvt_words4<false>(w0, w1, r);
+            c = rz ? cvt_words4<true, UG>(w0, w1, r) : cvt_words4<false, UG>(w0, w1, r);
             const uint32_t mm = (c ^ spread_bits(gq[u])) & 0x1111u;
             if (mm)
-              c = rz ? fix_mismatches<true>(c, mm, w0, w1, 0u, 0u, r) : fix_mismatches<false>(c, mm, w0, w1, 0u, 0u, r);
+              c = rz ? fix_mismatches<true, UG>(c, mm, w0, w1, 0u, 0u, r)
+                     : fix_mismatches<false, UG>(c, mm, w0, w1, 0u, 0u, r);
           } else {
             c = 0u;
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
               const uint32_t h = (e & 1) ? ((e & 2 ? w1 : w0) >> 16) : ((e & 2 ? w1 : w0) & 0xFFFFu);
               const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-              const uint32_t m3 = S > 0.0f ? guided_m3_exact(ax, S, (gq[u] >> e) & 1u) : 0u;
+              const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (gq[u] >> e) & 1u) : 0u;
               c |= (((h >> 15) << 3) | m3) << (4 * e);
             }
           }
           if (a.codes) reinterpret_cast<uint16_t*>(a.codes)[q] = (uint16_t)c;
-          const float4 v = decode4(c, S);
+          const float4 v = decode4_grid<UG>(c, S);
           if constexpr (BF16) {
             const __nv_bfloat162 p0 = __floats2bfloat162_rn(v.x, v.y), p1 = __floats2bfloat162_rn(v.z, v.w);
             reinterpret_cast<uint2*>(a.out)[q] =
@@ -986,7 +1080,8 @@ __device__ __forceinline__ int grid_index(uint32_t nib) {
 
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) {
-  constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;
+  constexpr bool UG = kUni<FMT>;
+  constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int NW = BE / 2;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
@@ -996,7 +1091,7 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
   while (lo < b1) {
     const int s = seg.find(lo);
     const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
-    const float st = FMT == TF4_NVFP4 ? a.rec_s_t[s] : 0.0f;
+    const float st = kE4M3<FMT> ? a.rec_s_t[s] : 0.0f;
     for (int64_t blk = lo + threadIdx.x; blk < hi; blk += kThreads) {
       uint32_t w[NW], cw[BE / 8];
 #pragma unroll
@@ -1004,7 +1099,7 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
         const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
         w[4 * q] = p.x; w[4 * q + 1] = p.y; w[4 * q + 2] = p.z; w[4 * q + 3] = p.w;
       }
-      if constexpr (FMT == TF4_NVFP4) {
+      if constexpr (kE4M3<FMT>) {
         const uint2 c = __ldg(reinterpret_cast<const uint2*>(a.rec_codes) + blk);
         cw[0] = c.x; cw[1] = c.y;
       } else {
@@ -1013,7 +1108,7 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
       }
       const uint32_t sc = a.rec_scales[blk];
       float S;
-      if constexpr (FMT == TF4_NVFP4) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
+      if constexpr (kE4M3<FMT>) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
       else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
       bad |= block_absmax_bits(w) >= 0x7F80u;
 #pragma unroll
@@ -1022,8 +1117,8 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
         const float ax = __uint_as_float((h & 0x7FFFu) << 16);
         const uint32_t no = (cw[e >> 3] >> (4 * (e & 7))) & 0xFu;
         const uint32_t sg = (h >> 15) << 3;
-        const uint32_t nr = sg | (S > 0.0f ? rtn_m3_exact(ax, S) : 0u);
-        const uint32_t ng = sg | (S > 0.0f ? guided_m3_exact(ax, S, no & 1u) : 0u);
+        const uint32_t nr = sg | (S > 0.0f ? rtn_m3_exact<UG>(ax, S) : 0u);
+        const uint32_t ng = sg | (S > 0.0f ? guided_m3_exact<UG>(ax, S, no & 1u) : 0u);
         const int d = abs(grid_index(nr) - grid_index(no));
         cnt[0] += d != 0;
         cnt[1] += d == 1;
@@ -1055,7 +1150,7 @@ struct DequantArgs {
 // store covers 512 contiguous bytes.  Segment pieces are whole blocks.
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
-  constexpr int BE = FMT == TF4_NVFP4 ? 16 : 32;
+  constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int QPB = BE / 4;  // quads per block
   constexpr int U = 4;         // quads per lane per iteration
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
@@ -1066,7 +1161,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
   while (lo < b1) {
     const int s = seg.find(lo);
     const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
-    const float st = FMT == TF4_NVFP4 ? a.s_t[s] : 0.0f;
+    const float st = kE4M3<FMT> ? a.s_t[s] : 0.0f;
     const int64_t q0 = lo * QPB, q1 = hi * QPB;
     for (int64_t qb = q0; qb < q1; qb += (int64_t)U * kThreads) {
       uint32_t cw[U], sc[U];
@@ -1083,9 +1178,9 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
         const int64_t q = qb + u * kThreads + tid;
         if (q < q1) {
           float S;
-          if constexpr (FMT == TF4_NVFP4) S = __fmul_rn(st, e4m3_decode(sc[u]));
+          if constexpr (kE4M3<FMT>) S = __fmul_rn(st, e4m3_decode(sc[u]));
           else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
-          a.out[q] = decode4(cw[u], S);
+          a.out[q] = decode4_grid<kUni<FMT>>(cw[u], S);
         }
       }
     }

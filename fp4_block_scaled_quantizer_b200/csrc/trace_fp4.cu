@@ -5,6 +5,7 @@
 #include <climits>
 #include <cstring>
 #include <mutex>
+#include <type_traits>
 
 #include "../../include/trace_fp4.h"
 #include "tf4_kernels.cuh"
@@ -23,10 +24,21 @@ struct Shape {
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Formats with an fp32 tensor scale (and hence segments and a workspace).
+bool has_tensor_scale(int fmt) { return fmt != TF4_MXFP4; }
+
+// Calls f with the format as a compile-time constant.
+template <class F>
+void by_format(int fmt, F&& f) {
+  if (fmt == TF4_NVFP4) f(std::integral_constant<int, TF4_NVFP4>{});
+  else if (fmt == TF4_UFP4) f(std::integral_constant<int, TF4_UFP4>{});
+  else f(std::integral_constant<int, TF4_MXFP4>{});
+}
+
 tf4_status check_desc(const tf4_desc* d, Shape* sh) {
   if (!d) return TF4_ERR_INVALID_ARG;
-  if (d->fmt != TF4_NVFP4 && d->fmt != TF4_MXFP4) return TF4_ERR_INVALID_ARG;
-  const int be = d->fmt == TF4_NVFP4 ? 16 : 32;
+  if (d->fmt != TF4_NVFP4 && d->fmt != TF4_MXFP4 && d->fmt != TF4_UFP4) return TF4_ERR_INVALID_ARG;
+  const int be = d->fmt == TF4_MXFP4 ? 32 : 16;
   if (d->rows < 0 || d->cols <= 0 || d->cols % be != 0) return TF4_ERR_SHAPE;
   if (d->rows > 0 && d->cols > (int64_t)(LLONG_MAX / 64) / d->rows) return TF4_ERR_SHAPE;
   const int nseg = d->num_segments;
@@ -112,30 +124,33 @@ tf4_status launched() {
 }
 
 size_t ws_bytes_for(const Shape& sh) {
-  if (sh.fmt != TF4_NVFP4) return 0;
+  if (!has_tensor_scale(sh.fmt)) return 0;
   return ((size_t)(sh.nseg + 1) * sizeof(uint32_t) + 255) & ~(size_t)255;
 }
 
-// NVFP4 quantize grid: shared by the amax pass and the quantize pass so
-// that both cover the same byte range per CTA.
-template <int MODE>
+// Quantize grid of the tensor-scale formats: shared by the amax pass and
+// the quantize pass so that both cover the same byte range per CTA.
+template <int FMT, int MODE>
 int64_t nvfp4_grid(const Shape& sh) {
-  return multi(sh) ? wave_grid(tf4::k_quant<TF4_NVFP4, MODE, tf4::SegN>, sh.nblocks)
-                   : wave_grid(tf4::k_quant<TF4_NVFP4, MODE, tf4::Seg1>, sh.nblocks);
+  return multi(sh) ? wave_grid(tf4::k_quant<FMT, MODE, tf4::SegN>, sh.nblocks)
+                   : wave_grid(tf4::k_quant<FMT, MODE, tf4::Seg1>, sh.nblocks);
 }
 
+// The amax pass; s_t_out (if not NULL) receives the tensor scale of FMT's grid.
+template <int FMT>
 tf4_status launch_amax(const Shape& sh, int64_t grid, const void* x, uint32_t* ws, float* s_t_out,
                        float* amax_out, int32_t* status, cudaStream_t st) {
+  constexpr bool U = tf4::kUni<FMT>;
   const uint4* x4 = static_cast<const uint4*>(x);
   // the amax pass works on 16-element blocks whatever the format
   const int64_t nb16 = sh.n / 16;
   if (multi(sh)) {
     tf4::SegN seg = make_segn(sh);
     seg.bpr = sh.cols / 16;
-    tf4::k_amax<tf4::SegN><<<(unsigned)grid, kThreads, 0, st>>>(x4, nb16, seg, ws, s_t_out, amax_out, status);
+    tf4::k_amax<tf4::SegN, U><<<(unsigned)grid, kThreads, 0, st>>>(x4, nb16, seg, ws, s_t_out, amax_out, status);
   } else {
-    tf4::k_amax<tf4::Seg1><<<(unsigned)grid, kThreads, 0, st>>>(x4, nb16, tf4::Seg1{}, ws, s_t_out, amax_out,
-                                                                 status);
+    tf4::k_amax<tf4::Seg1, U><<<(unsigned)grid, kThreads, 0, st>>>(x4, nb16, tf4::Seg1{}, ws, s_t_out, amax_out,
+                                                                    status);
   }
   return launched();
 }
@@ -148,7 +163,7 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
   tf4_status e = check_desc(d, &sh);
   if (e != TF4_OK) return e;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  const bool nv = sh.fmt == TF4_NVFP4;
+  const bool nv = has_tensor_scale(sh.fmt);
   if (nv && !s_t) return TF4_ERR_INVALID_ARG;
   if (nv && (!aligned(s_t, 4) || (amax_in && !aligned(amax_in, 4)))) return TF4_ERR_ALIGN;
   if (status && !aligned(status, 4)) return TF4_ERR_ALIGN;
@@ -173,20 +188,26 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
   a.status = status;
   a.s_t_out = s_t;
   if (nv) {
-    const int64_t grid = nvfp4_grid<MODE>(sh);
-    if (amax_in) {
-      a.st_src = amax_in;
-      a.st_from_amax = 1;
-    } else {
-      e = launch_amax(sh, grid, x, static_cast<uint32_t*>(ws), s_t, nullptr, status, st);
-      if (e != TF4_OK) return e;
-      a.st_src = s_t;
-      a.st_from_amax = 0;
-    }
-    if (multi(sh))
-      tf4::k_quant<TF4_NVFP4, MODE, tf4::SegN><<<(unsigned)grid, kThreads, 0, st>>>(a, make_segn(sh));
-    else
-      tf4::k_quant<TF4_NVFP4, MODE, tf4::Seg1><<<(unsigned)grid, kThreads, 0, st>>>(a, tf4::Seg1{});
+    by_format(sh.fmt, [&](auto f) {
+      constexpr int FMT = decltype(f)::value;
+      if constexpr (tf4::kE4M3<FMT>) {
+        const int64_t grid = nvfp4_grid<FMT, MODE>(sh);
+        if (amax_in) {
+          a.st_src = amax_in;
+          a.st_from_amax = 1;
+        } else {
+          e = launch_amax<FMT>(sh, grid, x, static_cast<uint32_t*>(ws), s_t, nullptr, status, st);
+          if (e != TF4_OK) return;
+          a.st_src = s_t;
+          a.st_from_amax = 0;
+        }
+        if (multi(sh))
+          tf4::k_quant<FMT, MODE, tf4::SegN><<<(unsigned)grid, kThreads, 0, st>>>(a, make_segn(sh));
+        else
+          tf4::k_quant<FMT, MODE, tf4::Seg1><<<(unsigned)grid, kThreads, 0, st>>>(a, tf4::Seg1{});
+      }
+    });
+    if (e != TF4_OK) return e;
   } else {
     a.st_src = nullptr;
     a.st_from_amax = 0;
@@ -254,7 +275,7 @@ size_t tf4_record_bytes(const tf4_desc* desc, int with_codes) {
   if (check_desc(desc, &sh) != TF4_OK) return 0;
   size_t b = with_codes ? (size_t)(sh.n / 2) : (size_t)(sh.n / 8);
   b += (size_t)sh.nblocks;
-  if (sh.fmt == TF4_NVFP4) b += sizeof(float) * (size_t)sh.nseg;
+  if (has_tensor_scale(sh.fmt)) b += sizeof(float) * (size_t)sh.nseg;
   return b;
 }
 
@@ -263,7 +284,7 @@ tf4_status tf4_segment_amax(const tf4_desc* desc, const void* x, float* amax, vo
   Shape sh;
   tf4_status e = check_desc(desc, &sh);
   if (e != TF4_OK) return e;
-  if (sh.fmt != TF4_NVFP4) return TF4_ERR_INVALID_ARG;
+  if (!has_tensor_scale(sh.fmt)) return TF4_ERR_INVALID_ARG;
   if (!amax) return TF4_ERR_INVALID_ARG;
   if (!aligned(amax, 4) || (status && !aligned(status, 4))) return TF4_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -274,7 +295,9 @@ tf4_status tf4_segment_amax(const tf4_desc* desc, const void* x, float* amax, vo
   if (!ws) return TF4_ERR_WORKSPACE;
   if (!aligned(ws, 4)) return TF4_ERR_ALIGN;
   if (ws_bytes < ws_bytes_for(sh)) return TF4_ERR_WORKSPACE;
-  return launch_amax(sh, nvfp4_grid<tf4::kRTN>(sh), x, static_cast<uint32_t*>(ws), nullptr, amax, status, st);
+  // the maxima do not depend on the grid; size the grid like NVFP4's quantize pass
+  return launch_amax<TF4_NVFP4>(sh, nvfp4_grid<TF4_NVFP4, tf4::kRTN>(sh), x, static_cast<uint32_t*>(ws), nullptr,
+                                amax, status, st);
 }
 
 tf4_status tf4_quantize_rtn(const tf4_desc* desc, const void* x, const float* amax_in, uint8_t* codes,
@@ -321,7 +344,7 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const 
   if (sh.nseg != 1) return TF4_ERR_INVALID_ARG;
   if (nl < 1 || nl > TF4_MAX_BATCH || !x) return TF4_ERR_INVALID_ARG;
   if (keep < 0 || keep > nl || ((keep > 0) != (info_bits != nullptr))) return TF4_ERR_INVALID_ARG;
-  const bool nv = sh.fmt == TF4_NVFP4;
+  const bool nv = has_tensor_scale(sh.fmt);
   if (nv && !s_t) return TF4_ERR_INVALID_ARG;
   if ((nv && !aligned(s_t, 4)) || (status && !aligned(status, 4))) return TF4_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -376,11 +399,17 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const 
   a.st_src = s_t;
   a.st_from_amax = 0;
   if (nv) {
-    const int64_t grid = wave_grid(tf4::k_quant<TF4_NVFP4, tf4::kCAPTURE, tf4::SegBatch>, total);
-    tf4::k_amax<tf4::SegBatch><<<(unsigned)grid, kThreads, 0, st>>>(nullptr, total, sb, static_cast<uint32_t*>(ws),
-                                                                    s_t, nullptr, status);
-    if ((e = launched()) != TF4_OK) return e;
-    tf4::k_quant<TF4_NVFP4, tf4::kCAPTURE, tf4::SegBatch><<<(unsigned)grid, kThreads, 0, st>>>(a, sb);
+    by_format(sh.fmt, [&](auto f) {
+      constexpr int FMT = decltype(f)::value;
+      if constexpr (tf4::kE4M3<FMT>) {
+        const int64_t grid = wave_grid(tf4::k_quant<FMT, tf4::kCAPTURE, tf4::SegBatch>, total);
+        tf4::k_amax<tf4::SegBatch, tf4::kUni<FMT>><<<(unsigned)grid, kThreads, 0, st>>>(
+            nullptr, total, sb, static_cast<uint32_t*>(ws), s_t, nullptr, status);
+        if ((e = launched()) != TF4_OK) return;
+        tf4::k_quant<FMT, tf4::kCAPTURE, tf4::SegBatch><<<(unsigned)grid, kThreads, 0, st>>>(a, sb);
+      }
+    });
+    if (e != TF4_OK) return e;
   } else {
     a.s_t_out = nullptr;
     a.st_src = nullptr;
@@ -397,7 +426,7 @@ tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_
   tf4_status e = check_desc(desc, &sh);
   if (e != TF4_OK) return e;
   if (sh.n == 0) return TF4_OK;
-  const bool nv = sh.fmt == TF4_NVFP4;
+  const bool nv = has_tensor_scale(sh.fmt);
   if (!x || !rec_scales || !rec_bits || !codes || (nv && !rec_s_t)) return TF4_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(rec_bits, 4) || (nv && !aligned(rec_s_t, 4)) ||
       (status && !aligned(status, 4)))
@@ -411,18 +440,18 @@ tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_
   a.rec_bits = rec_bits;
   a.codes = codes;
   a.status = status;
-  if (nv) {
-    if (multi(sh)) {
-      const int64_t g = wave_grid(tf4::k_guided<TF4_NVFP4, tf4::SegN>, sh.nblocks);
-      tf4::k_guided<TF4_NVFP4, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
-    } else {
-      const int64_t g = wave_grid(tf4::k_guided<TF4_NVFP4, tf4::Seg1>, sh.nblocks);
-      tf4::k_guided<TF4_NVFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  by_format(sh.fmt, [&](auto f) {
+    constexpr int FMT = decltype(f)::value;
+    if constexpr (tf4::kE4M3<FMT>) {
+      if (multi(sh)) {
+        const int64_t g = wave_grid(tf4::k_guided<FMT, tf4::SegN>, sh.nblocks);
+        tf4::k_guided<FMT, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+        return;
+      }
     }
-  } else {
-    const int64_t g = wave_grid(tf4::k_guided<TF4_MXFP4, tf4::Seg1>, sh.nblocks);
-    tf4::k_guided<TF4_MXFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
-  }
+    const int64_t g = wave_grid(tf4::k_guided<FMT, tf4::Seg1>, sh.nblocks);
+    tf4::k_guided<FMT, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  });
   return launched();
 }
 
@@ -433,7 +462,7 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
   tf4_status e = check_desc(desc, &sh);
   if (e != TF4_OK) return e;
   if (sh.n == 0) return TF4_OK;
-  const bool nv = sh.fmt == TF4_NVFP4;
+  const bool nv = has_tensor_scale(sh.fmt);
   if (!x || !rec_scales || !rec_bits || !out || (nv && !rec_s_t)) return TF4_ERR_INVALID_ARG;
   if (out_bf16 != 0 && out_bf16 != 1) return TF4_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(out, 16) || !aligned(rec_bits, 4) || (codes && !aligned(codes, 16)) ||
@@ -454,16 +483,18 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
     const int64_t g = wave_grid(tf4::k_guided_fq<FMT, SEG, BF>, sh.nblocks);          \
     tf4::k_guided_fq<FMT, SEG, BF><<<(unsigned)g, kThreads, 0, st>>>(a, segv);        \
   } while (0)
-  if (nv && multi(sh)) {
-    if (out_bf16) TF4_LAUNCH_FQ(TF4_NVFP4, tf4::SegN, true, make_segn(sh));
-    else TF4_LAUNCH_FQ(TF4_NVFP4, tf4::SegN, false, make_segn(sh));
-  } else if (nv) {
-    if (out_bf16) TF4_LAUNCH_FQ(TF4_NVFP4, tf4::Seg1, true, tf4::Seg1{});
-    else TF4_LAUNCH_FQ(TF4_NVFP4, tf4::Seg1, false, tf4::Seg1{});
-  } else {
-    if (out_bf16) TF4_LAUNCH_FQ(TF4_MXFP4, tf4::Seg1, true, tf4::Seg1{});
-    else TF4_LAUNCH_FQ(TF4_MXFP4, tf4::Seg1, false, tf4::Seg1{});
-  }
+  by_format(sh.fmt, [&](auto f) {
+    constexpr int FMT = decltype(f)::value;
+    if constexpr (tf4::kE4M3<FMT>) {
+      if (multi(sh)) {
+        if (out_bf16) TF4_LAUNCH_FQ(FMT, tf4::SegN, true, make_segn(sh));
+        else TF4_LAUNCH_FQ(FMT, tf4::SegN, false, make_segn(sh));
+        return;
+      }
+    }
+    if (out_bf16) TF4_LAUNCH_FQ(FMT, tf4::Seg1, true, tf4::Seg1{});
+    else TF4_LAUNCH_FQ(FMT, tf4::Seg1, false, tf4::Seg1{});
+  });
 #undef TF4_LAUNCH_FQ
   return launched();
 }
@@ -477,7 +508,7 @@ tf4_status tf4_mismatch_stats(const tf4_desc* desc, const void* x, const uint8_t
   if (!counts) return TF4_ERR_INVALID_ARG;
   if (!aligned(counts, 8) || (status && !aligned(status, 4))) return TF4_ERR_ALIGN;
   if (sh.n == 0) return TF4_OK;
-  const bool nv = sh.fmt == TF4_NVFP4;
+  const bool nv = has_tensor_scale(sh.fmt);
   if (!x || !rec_scales || !rec_codes || (nv && !rec_s_t)) return TF4_ERR_INVALID_ARG;
   if (!aligned(x, 16) || !aligned(rec_codes, 16) || (nv && !aligned(rec_s_t, 4))) return TF4_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -489,16 +520,18 @@ tf4_status tf4_mismatch_stats(const tf4_desc* desc, const void* x, const uint8_t
   a.rec_codes = rec_codes;
   a.counts = counts;
   a.status = status;
-  if (nv && multi(sh)) {
-    const int64_t g = wave_grid(tf4::k_mismatch<TF4_NVFP4, tf4::SegN>, sh.nblocks);
-    tf4::k_mismatch<TF4_NVFP4, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
-  } else if (nv) {
-    const int64_t g = wave_grid(tf4::k_mismatch<TF4_NVFP4, tf4::Seg1>, sh.nblocks);
-    tf4::k_mismatch<TF4_NVFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
-  } else {
-    const int64_t g = wave_grid(tf4::k_mismatch<TF4_MXFP4, tf4::Seg1>, sh.nblocks);
-    tf4::k_mismatch<TF4_MXFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
-  }
+  by_format(sh.fmt, [&](auto f) {
+    constexpr int FMT = decltype(f)::value;
+    if constexpr (tf4::kE4M3<FMT>) {
+      if (multi(sh)) {
+        const int64_t g = wave_grid(tf4::k_mismatch<FMT, tf4::SegN>, sh.nblocks);
+        tf4::k_mismatch<FMT, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+        return;
+      }
+    }
+    const int64_t g = wave_grid(tf4::k_mismatch<FMT, tf4::Seg1>, sh.nblocks);
+    tf4::k_mismatch<FMT, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  });
   return launched();
 }
 
@@ -508,7 +541,7 @@ tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint
   tf4_status e = check_desc(desc, &sh);
   if (e != TF4_OK) return e;
   if (sh.n == 0) return TF4_OK;
-  const bool nv = sh.fmt == TF4_NVFP4;
+  const bool nv = has_tensor_scale(sh.fmt);
   if (!codes || !scales || !out || (nv && !s_t)) return TF4_ERR_INVALID_ARG;
   if (!aligned(codes, 16) || !aligned(out, 16) || (nv && !aligned(s_t, 4))) return TF4_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -518,18 +551,18 @@ tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint
   a.s_t = s_t;
   a.out = reinterpret_cast<float4*>(out);
   a.nblocks = sh.nblocks;
-  if (nv) {
-    if (multi(sh)) {
-      const int64_t g = wave_grid(tf4::k_dequant<TF4_NVFP4, tf4::SegN>, sh.nblocks);
-      tf4::k_dequant<TF4_NVFP4, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
-    } else {
-      const int64_t g = wave_grid(tf4::k_dequant<TF4_NVFP4, tf4::Seg1>, sh.nblocks);
-      tf4::k_dequant<TF4_NVFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  by_format(sh.fmt, [&](auto f) {
+    constexpr int FMT = decltype(f)::value;
+    if constexpr (tf4::kE4M3<FMT>) {
+      if (multi(sh)) {
+        const int64_t g = wave_grid(tf4::k_dequant<FMT, tf4::SegN>, sh.nblocks);
+        tf4::k_dequant<FMT, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+        return;
+      }
     }
-  } else {
-    const int64_t g = wave_grid(tf4::k_dequant<TF4_MXFP4, tf4::Seg1>, sh.nblocks);
-    tf4::k_dequant<TF4_MXFP4, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
-  }
+    const int64_t g = wave_grid(tf4::k_dequant<FMT, tf4::Seg1>, sh.nblocks);
+    tf4::k_dequant<FMT, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+  });
   return launched();
 }
 
@@ -569,7 +602,7 @@ tf4_status tf4_quantize_capture_noalloc(const tf4_desc* desc, const void* x, uin
   uint32_t* scratch = noalloc_scratch();
   if (!scratch) return TF4_ERR_CUDA;
   const size_t need = sizeof(uint32_t) * (size_t)(sh.nseg + 1);
-  if (sh.fmt == TF4_NVFP4 && sh.n > 0 &&
+  if (has_tensor_scale(sh.fmt) && sh.n > 0 &&
       cudaMemsetAsync(scratch, 0, need, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return TF4_ERR_CUDA;
   return tf4_quantize_capture(desc, x, nullptr, codes, scales, s_t, bits, scratch, sizeof(tf4_noalloc_scratch),

@@ -18,6 +18,9 @@
  *     sharing one E4M3 scale; round-to-nearest forward, stochastic rounding
  *     for backward / weight updates.
  *   - aibr.jp/archives/132665 (TetraJet), section 3: MXFP4 per-group scale.
+ *   - "FP4学習の「収縮バイアス」問題を解決するUFP4レシピ" (gotosocial.
+ *     chinng-lab-srv.dev), section "UFP4 の設計と実装指針": a uniform 4-bit
+ *     grid (E1M2 / INT4) instead of E2M1's.
  *
  * Formats.  E2M1 magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} indexed by
  * m3 = exponent<<1 | mantissa; a code nibble is sign<<3 | m3.
@@ -29,6 +32,14 @@
  *   MXFP4: 32-element blocks; scale byte = e + 127 with
  *          e = clamp(floor(log2 bamax) - 2, -127, 127) (-127 for an
  *          all-zero block); S = 2^e.  No tensor scale.
+ *   UFP4:  the uniform grid {0, 1, ..., 7} (m3 = the magnitude itself) in
+ *          NVFP4's container: 16-element blocks, segments, s_t =
+ *          amax / (7*448), b = E4M3_rne_satfinite( fl32(fl32(bamax/7) / s_t) ),
+ *          S = fl32(s_t * E4M3(b)).  (E1M2's grid is this one / 4; with the
+ *          tensor scale taken from the grid maximum both give the same codes
+ *          and scale bytes.)  Every rule below reads "the grid maximum" (6 or
+ *          7) for 6, and everything the function descriptions say of NVFP4's
+ *          s_t, segments and workspace holds for UFP4 too.
  *   Rounding of y = |x| / S (the exact real quotient):
  *     RTN     nearest codeword, ties to even m3, saturating at 6;
  *     SR      between the two neighbours lo < y < hi, round up iff
@@ -43,13 +54,13 @@
  *             S == 0 gives signed zero.  The sign is always x's own.
  *
  * Layouts (all contiguous, row-major, flat element index i = r*cols + c):
- *   x         bf16 [rows, cols], cols % 16 == 0 (NVFP4) / % 32 (MXFP4)
+ *   x         bf16 [rows, cols], cols % 16 == 0 (NVFP4, UFP4) / % 32 (MXFP4)
  *   codes     uint8 [rows*cols/2]; element 2j in the low nibble of byte j
  *   scales    uint8 [rows, cols/block] (linear, not swizzled)
- *   s_t       float [num_segments] (NVFP4 only)
+ *   s_t       float [num_segments] (NVFP4 and UFP4 only)
  *   guidance  uint8 [rows*cols/8]; bit (i & 7) of byte (i >> 3) = m3_i & 1
  *
- * Segments.  NVFP4 may split the rows into num_segments groups (e.g. the
+ * Segments.  NVFP4 (and UFP4) may split the rows into num_segments groups (e.g. the
  * per-expert groups of a mixture-of-experts dispatch), each with its own
  * s_t.  seg_row_offsets is a HOST array of num_segments + 1 non-decreasing
  * row offsets, first 0, last rows; empty segments are allowed (their s_t is
@@ -98,7 +109,7 @@ typedef enum {
   TF4_ERR_CUDA = 7         /* a CUDA call failed                            */
 } tf4_status;
 
-typedef enum { TF4_NVFP4 = 0, TF4_MXFP4 = 1 } tf4_format;
+typedef enum { TF4_NVFP4 = 0, TF4_MXFP4 = 1, TF4_UFP4 = 2 } tf4_format;
 
 #define TF4_MAX_SEGMENTS 1024
 #define TF4_MAX_BATCH 64

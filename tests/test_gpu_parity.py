@@ -55,7 +55,7 @@ def check_quant(xb, fmt, mode=O.RTN, seg=None, seed=0, bits=True):
     assert r["status"] == 0
     assert_same("codes", host(q.codes), r["codes"])
     assert_same("scales", host(q.scales), r["scales"])
-    if fmt == O.NVFP4:
+    if O.HAS_TENSOR_SCALE[fmt]:
         assert_same("s_t", f32_bits(host(q.s_t)), f32_bits(r["s_t"]))
     if bits and mode != O.SR:
         assert_same("bits", host(q.bits), r["bits"])
@@ -78,14 +78,23 @@ def test_mxfp4_capture_shapes(shape):
     check_quant(xb, O.MXFP4)
 
 
-@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("shape", SHAPES_NV)
+def test_ufp4_capture_shapes(shape):
+    xb = W.random_bf16(shape, seed=sum(shape) + 2, device=DEV, outlier_frac=0.003)
+    check_quant(xb, O.UFP4)
+
+
+FMTS = [O.NVFP4, O.MXFP4, O.UFP4]
+
+
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("seed", [0, 4, 2**40 + 3])
 def test_sr_parity(fmt, seed):
     xb = W.random_bf16((67, 1024), seed=seed % 1000, device=DEV, outlier_frac=0.01)
     check_quant(xb, fmt, O.SR, seed=seed)
 
 
-@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("fmt", FMTS)
 def test_sr_full_compare_16m(fmt):
     """Every element of a 16.8M-element SR call against the oracle: enough
     elements for ~80 uniforms to fall within the fast path's safety margin
@@ -116,44 +125,66 @@ def test_e2m1_exhaustive_via_unit_scale():
     check_quant(xb, O.MXFP4)
 
 
-def test_e4m3_block_scale_sweep():
-    """NVFP4 with s_t = 1 (amax = 2688): every positive bf16 block max up to
-    2688 gives r = bamax/6, sweeping the device E4M3 rounding."""
+def test_uniform_grid_exhaustive_via_unit_scale():
+    """UFP4 with s_t = 1 (amax = 3136) and blocks whose max is 7.0 have
+    S = 1, so y = x: every bf16 value with |x| < 8 (both signs) goes through
+    the device's uniform-grid rounding as itself."""
+    b = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    v = ((b.astype(np.uint32) << 16).view(np.float32))
+    sel = b[np.isfinite(v) & (np.abs(v) < 7.0)]
+    per = 15
+    nblk = (len(sel) + per - 1) // per
+    pad = np.zeros(nblk * per, np.uint16)
+    pad[: len(sel)] = sel
+    blocks = np.concatenate([np.full((nblk, 1), 0x40E0, np.uint16), pad.reshape(nblk, per)], axis=1)  # 7.0
+    blocks = np.concatenate([blocks, np.full((1, 16), 0x4544, np.uint16)], axis=0)  # 3136.0
+    check_quant(W.from_bits(blocks, DEV), O.UFP4)
+
+
+@pytest.mark.parametrize("fmt,amax_bits,amax", [(O.NVFP4, 0x4528, 2688.0), (O.UFP4, 0x4544, 3136.0)])
+def test_e4m3_block_scale_sweep(fmt, amax_bits, amax):
+    """s_t = 1 (amax = 448 * grid max): every positive bf16 block max up to
+    amax gives r = bamax / grid max, sweeping the device E4M3 rounding."""
     b = np.arange(1, 0x7F80, dtype=np.uint32).astype(np.uint16)
     v = (b.astype(np.uint32) << 16).view(np.float32)
-    b = b[v <= 2688.0]
+    b = b[v <= amax]
     x = np.zeros((len(b) + 1, 16), np.uint16)
     x[:-1, 0] = b
     x[:-1, 1] = 0x8000 | b  # negative copy
     x[:-1, 2:] = (b[:, None] >> 1) & 0x7F7F
-    x[-1, 0] = 0x4528  # 2688.0
-    check_quant(W.from_bits(x, DEV), O.NVFP4)
+    x[-1, 0] = amax_bits
+    check_quant(W.from_bits(x, DEV), fmt)
 
 
-def _near_tie_tensor(rng, s_mant, rows=256):
-    """Rows whose per-tensor scale is 'nice' (amax = 2688 * s), so that many
-    midpoint * S are bf16 values; elements sit on and around those points."""
-    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, 0.5, 1, 1.5, 2, 3, 4, 6])
+def _near_tie_tensor(rng, s_mant, rows=256, fmt=O.NVFP4):
+    """Rows whose per-tensor scale is 'nice' (amax = 448 * grid max * s), so
+    that many midpoint * S are bf16 values; elements sit on and around those
+    points."""
+    if fmt == O.UFP4:
+        mids, top = np.concatenate([np.arange(7) + 0.5, np.arange(1, 8)]), 7.0
+    else:
+        mids, top = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5, 0.5, 1, 1.5, 2, 3, 4, 6]), 6.0
     out = np.zeros((rows, 16), np.float32)
     for r in range(rows):
         S = float(np.float32(rng.choice([0.5, 1.0, 1.25, 0.75, 1.5, 0.875]) * 2.0 ** rng.integers(-3, 3)))
         pts = rng.choice(mids, 15) * S
         out[r, 1:] = pts * (1 + rng.choice([-1, 0, 0, 1], 15) * 2.0 ** -8)
-        out[r, 0] = 6 * S
-    out[0, 0] = 2688.0 * s_mant
+        out[r, 0] = top * S
+    out[0, 0] = 448.0 * top * s_mant
     xb = torch.from_numpy(out).to(torch.bfloat16)
     return xb
 
 
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
 @pytest.mark.parametrize("s_mant", [1.0, 0.5, 3.0])
-def test_near_tie_blocks(s_mant):
+def test_near_tie_blocks(fmt, s_mant):
     rng = np.random.default_rng(int(s_mant * 10))
-    xb = _near_tie_tensor(rng, s_mant).to(DEV)
-    check_quant(xb, O.NVFP4)
-    check_quant(xb, O.NVFP4, O.SR, seed=11)
+    xb = _near_tie_tensor(rng, s_mant, fmt=fmt).to(DEV)
+    check_quant(xb, fmt)
+    check_quant(xb, fmt, O.SR, seed=11)
 
 
-@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("fmt", FMTS)
 def test_tiny_and_zero_scales(fmt):
     x = np.zeros((8, 64), np.uint16)
     x[1, :] = 0x0001          # smallest subnormals
@@ -163,31 +194,34 @@ def test_tiny_and_zero_scales(fmt):
     xb = W.from_bits(x, DEV)
     check_quant(xb, fmt)
     seg = [0, 2, 2, 4, 8]
-    if fmt == O.NVFP4:
+    if O.HAS_TENSOR_SCALE[fmt]:
         check_quant(xb, fmt, seg=seg)
 
 
-def test_segments_ragged_with_empties():
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
+def test_segments_ragged_with_empties(fmt):
     xb = W.random_bf16((300, 256), seed=9, device=DEV, outlier_frac=0.01)
     seg = [0, 0, 1, 1, 50, 51, 51, 299, 300, 300]
-    q, r = check_quant(xb, O.NVFP4, seg=seg)
-    check_quant(xb, O.NVFP4, O.SR, seg=seg, seed=5)
+    q, r = check_quant(xb, fmt, seg=seg)
+    check_quant(xb, fmt, O.SR, seg=seg, seed=5)
     xt = W.perturb(xb, 7, rel=0.02)
     g = B.tf4_quantize_guided(xt, q)
-    want, st = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], O.NVFP4, rec_s_t=r["s_t"], seg_off=seg)
+    want, st = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"], seg_off=seg)
     assert_same("guided", host(g), want)
 
 
-def test_segment_amax_and_amax_in():
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
+def test_segment_amax_and_amax_in(fmt):
     xb = W.random_bf16((200, 512), seed=12, device=DEV, outlier_frac=0.01)
     seg = [0, 20, 20, 150, 200]
     amax = B.tf4_segment_amax(xb, seg)
     want, _ = O.segment_amax(W.bf16_bits(xb), seg)
     assert_same("amax", f32_bits(host(amax)), f32_bits(want))
-    a = B.tf4_quantize_capture(xb, seg_off=seg)
-    b = B.tf4_quantize_capture(xb, seg_off=seg, amax_in=amax)
+    a = B.tf4_quantize_capture(xb, fmt=fmt, seg_off=seg)
+    b = B.tf4_quantize_capture(xb, fmt=fmt, seg_off=seg, amax_in=amax)
     for n in ("codes", "scales", "s_t", "bits"):
         assert torch.equal(getattr(a, n), getattr(b, n)), n
+    check_quant(xb, fmt, seg=seg)
 
 
 def test_workspace_returns_to_zero():
@@ -199,7 +233,7 @@ def test_workspace_returns_to_zero():
         assert int(ws.count_nonzero()) == 0
 
 
-@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("fmt", FMTS)
 @pytest.mark.parametrize("perturb", [0.0, 1e-3, 0.05])
 def test_guided_parity(fmt, perturb):
     xb = W.random_bf16((96, 1024), seed=17, device=DEV, outlier_frac=0.005)
@@ -214,7 +248,7 @@ def test_guided_parity(fmt, perturb):
         assert torch.equal(g, q.codes)
 
 
-@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("fmt", FMTS)
 def test_guided_unrelated_train_tensor(fmt):
     """Train-side values unrelated to the rollout's (about half the nibbles
     disagree with the recorded bit): every element still lands on the
@@ -227,7 +261,7 @@ def test_guided_unrelated_train_tensor(fmt):
     assert_same("guided", host(g), want)
 
 
-@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("fmt", FMTS)
 def test_guided_reproduces_sr_capture(fmt):
     xb = W.random_bf16((64, 512), seed=29, device=DEV)
     q = B.tf4_quantize_sr(xb, 77, fmt=fmt)
@@ -236,27 +270,29 @@ def test_guided_reproduces_sr_capture(fmt):
     assert torch.equal(g, q.codes)
 
 
-def test_guided_near_ties():
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
+def test_guided_near_ties(fmt):
     rng = np.random.default_rng(5)
-    xb = _near_tie_tensor(rng, 1.0).to(DEV)
-    q, r = check_quant(xb, O.NVFP4)
-    xt = _near_tie_tensor(np.random.default_rng(6), 1.0).to(DEV)
+    xb = _near_tie_tensor(rng, 1.0, fmt=fmt).to(DEV)
+    q, r = check_quant(xb, fmt)
+    xt = _near_tie_tensor(np.random.default_rng(6), 1.0, fmt=fmt).to(DEV)
     g = B.tf4_quantize_guided(xt, q)
-    want, _ = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], O.NVFP4, rec_s_t=r["s_t"])
+    want, _ = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"])
     assert_same("guided", host(g), want)
 
 
-@pytest.mark.parametrize("fmt", [O.NVFP4, O.MXFP4])
+@pytest.mark.parametrize("fmt", FMTS)
 def test_dequant_parity(fmt):
     xb = W.random_bf16((77, 2048), seed=31, device=DEV, outlier_frac=0.01)
-    seg = [0, 30, 77] if fmt == O.NVFP4 else None
+    seg = [0, 30, 77] if O.HAS_TENSOR_SCALE[fmt] else None
     q, r = check_quant(xb, fmt, seg=seg)
     d = B.tf4_dequantize(q)
     want = O.dequantize(r["codes"], r["scales"], 77, 2048, fmt, s_t=r["s_t"], seg_off=seg)
     assert_same("dequant", f32_bits(host(d)), f32_bits(want))
 
 
-@pytest.mark.parametrize("fmt,seg", [(O.NVFP4, None), (O.NVFP4, [0, 25, 25, 77]), (O.MXFP4, None)])
+@pytest.mark.parametrize("fmt,seg", [(O.NVFP4, None), (O.NVFP4, [0, 25, 25, 77]), (O.MXFP4, None), (O.UFP4, None),
+                                     (O.UFP4, [0, 25, 25, 77])])
 @pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
 def test_guided_fake_quant_parity(fmt, seg, dtype):
     """The fused train-side pass equals guided quantization followed by
@@ -275,7 +311,8 @@ def test_guided_fake_quant_parity(fmt, seg, dtype):
         assert_same("values", host(y.view(torch.int16)).view(np.uint16), O.f32_to_bf16(vals))
 
 
-@pytest.mark.parametrize("fmt,seg", [(O.NVFP4, None), (O.NVFP4, [0, 30, 30, 64]), (O.MXFP4, None)])
+@pytest.mark.parametrize("fmt,seg", [(O.NVFP4, None), (O.NVFP4, [0, 30, 30, 64]), (O.MXFP4, None), (O.UFP4, None),
+                                     (O.UFP4, [0, 30, 30, 64])])
 @pytest.mark.parametrize("rel", [1e-3, 0.05, None])
 def test_mismatch_stats_parity(fmt, seg, rel):
     """Mismatch diagnostics equal the oracle's counts (None: unrelated train tensor)."""
@@ -290,7 +327,8 @@ def test_mismatch_stats_parity(fmt, seg, rel):
         assert want[0] == want[1] + want[2]
 
 
-@pytest.mark.parametrize("fmt,L,keep", [(O.NVFP4, 5, 2), (O.NVFP4, 3, 3), (O.NVFP4, 1, 0), (O.MXFP4, 4, 1)])
+@pytest.mark.parametrize("fmt,L,keep", [(O.NVFP4, 5, 2), (O.NVFP4, 3, 3), (O.NVFP4, 1, 0), (O.MXFP4, 4, 1),
+                                        (O.UFP4, 4, 2)])
 def test_capture_batched_parity(fmt, L, keep):
     """One batched call = per-layer capture (oracle) for every layer; the
     deepest `keep` layers' guidance lands contiguously in the info cache."""
@@ -301,7 +339,7 @@ def test_capture_batched_parity(fmt, L, keep):
         r = O.quantize(W.bf16_bits(x), fmt, O.RTN, bits=True)
         assert_same(f"codes {i}", host(out.codes[i]), r["codes"])
         assert_same(f"scales {i}", host(out.scales[i]), r["scales"])
-        if fmt == O.NVFP4:
+        if O.HAS_TENSOR_SCALE[fmt]:
             assert_same(f"s_t {i}", f32_bits(host(out.s_t[i:i + 1])), f32_bits(r["s_t"]))
         if i >= L - keep:
             assert_same(f"bits {i}", host(out.info_bits[i - (L - keep)]), r["bits"])
@@ -397,8 +435,8 @@ def check_sampled(xb, q, fmt, seg=None, mode=O.RTN, seed=0, guided_x=None, g_cod
     rows, cols = xb.shape
     xs = W.bf16_bits(xb)
     s_t = None
-    if fmt == O.NVFP4:
-        s_t, st = O.segment_scales(xs, seg)
+    if O.HAS_TENSOR_SCALE[fmt]:
+        s_t, st = O.segment_scales(xs, seg, fmt)
         assert st == 0
         assert_same("s_t", f32_bits(host(q.s_t)), f32_bits(s_t))
     blk = O.BLOCK[fmt]
@@ -431,24 +469,25 @@ def test_activation_outliers_full():
         assert_same("guided", host(g), want)
 
 
-@pytest.mark.parametrize("layer", [0, 39])
-def test_layer_stack_layer_sampled(layer):
+@pytest.mark.parametrize("fmt,layer", [(O.NVFP4, 0), (O.NVFP4, 39), (O.UFP4, 39)])
+def test_layer_stack_layer_sampled(fmt, layer):
     x = W.layer_stack_layer(layer, DEV)
-    q = B.tf4_quantize_capture(x, guidance=layer >= 20)
+    q = B.tf4_quantize_capture(x, fmt=fmt, guidance=layer >= 20)
     g = B.tf4_quantize_guided(x, q) if layer >= 20 else None
     assert B.read_status(x.device) == 0
-    check_sampled(x, q, O.NVFP4, g_codes=g, guided_x=x if g is not None else None)
+    check_sampled(x, q, fmt, g_codes=g, guided_x=x if g is not None else None)
     if g is not None:
         assert torch.equal(g, q.codes)
 
 
-def test_moe_dispatch_sampled():
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
+def test_moe_dispatch_sampled(fmt):
     w = W.moe_dispatch(DEV)
     seg = w["seg_off"]
-    q = B.tf4_quantize_capture(w["x"], seg_off=seg)
+    q = B.tf4_quantize_capture(w["x"], fmt=fmt, seg_off=seg)
     g = B.tf4_quantize_guided(w["x_train"], q)
     assert B.read_status(w["x"].device) == 0
-    check_sampled(w["x"], q, O.NVFP4, seg=seg, guided_x=w["x_train"], g_codes=g)
+    check_sampled(w["x"], q, fmt, seg=seg, guided_x=w["x_train"], g_codes=g)
 
 
 def test_weights_sampled():
