@@ -36,6 +36,17 @@ constexpr bool kUni = FMT == TF4_UFP4;
 template <bool U>
 constexpr float kGridMax = U ? 7.0f : 6.0f;
 
+// Programmatic dependent launch.  The library launches its kernels with
+// programmatic stream serialization, so a kernel may be scheduled while the
+// grid before it in the stream is still finishing.  Every kernel therefore
+// first waits for that grid to complete and its memory to be visible
+// (before reading or writing anything), then lets the next grid begin
+// launching.  Without the launch attribute both instructions are no-ops.
+__device__ __forceinline__ void pdl_enter() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------------- segments
 // One per-tensor-scale segment covering everything (the common case).
 struct Seg1 {
@@ -379,6 +390,7 @@ template <class SEG, bool U = false>
 __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, int64_t nblocks,
                                                    SEG seg, uint32_t* ws, float* s_t_out,
                                                    float* amax_out, int32_t* status) {
+  pdl_enter();
   __shared__ uint32_t red[kThreads / 32];
   __shared__ int last;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, nblocks);
@@ -563,10 +575,41 @@ __device__ __forceinline__ float block_rho(float rho_c, uint32_t e_b) {
   return __uint_as_float(__float_as_uint(rho_c) + (uint32_t)((7 - (int)e_b) << 23));
 }
 
+// Uniform grid, 4 bf16 (two words) times r -> the 4 nibble bytes
+// [n0, n1, n2, n3] (byte i = sign<<3 | k_i).  k = round-half-even of |v|:
+// 2^23 + |v| is rounded once, to an integer, whose value sits in the low
+// mantissa bits (byte 0 of the fp32 pattern while k < 256).  CLAMP
+// saturates |v| at 7 first; without it the caller guarantees |v| < 7.5.
+// The signs are the bf16 sign bits (byte_perm picks the high byte of each
+// bf16; bit 7 of each byte moves to bit 3).
+template <bool RZ, bool CLAMP>
+__device__ __forceinline__ uint32_t uni_bytes4(uint32_t w0, uint32_t w1, float r) {
+  const float v[4] = {mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r), mul<RZ>(bf_hi(w1), r)};
+  uint32_t t[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    t[k] = __float_as_uint(__fadd_rn(CLAMP ? fminf(fabsf(v[k]), 7.0f) : fabsf(v[k]), 0x1p23f));
+  const uint32_t k4 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+  return k4 | ((__byte_perm(w0, w1, 0x7531) >> 4) & 0x08080808u);
+}
+
+// Nibble bytes [n0, n1, n2, n3] -> n0 | n1 << 4 in byte 0 and n2 | n3 << 4
+// in byte 2 (bytes 1 and 3 are don't-care).
+__device__ __forceinline__ uint32_t nib_pairs(uint32_t b) { return b | (b >> 4); }
+
+template <bool RZ, bool CLAMP>
+__device__ __forceinline__ uint32_t cvt_uni_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r) {
+  return __byte_perm(nib_pairs(uni_bytes4<RZ, CLAMP>(w0, w1, r)), nib_pairs(uni_bytes4<RZ, CLAMP>(w2, w3, r)),
+                     0x6420);
+}
+
 // Eight bf16 (four words) times rho -> eight grid nibbles (signed, RNE).
-template <bool RZ = false, bool U = false>
+// CLAMP (uniform grid only; E2M1's conversion always saturates): the
+// products may reach 7.5 or more.
+template <bool RZ = false, bool U = false, bool CLAMP = true>
 __device__ __forceinline__ uint32_t cvt_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r) {
-  return cvt_grid_x8<U>(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r),
+  if constexpr (U) return cvt_uni_words<RZ, CLAMP>(w0, w1, w2, w3, r);
+  return cvt_e2m1x8(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r),
                     mul<RZ>(bf_hi(w1), r), mul<RZ>(bf_lo(w2), r), mul<RZ>(bf_hi(w2), r),
                     mul<RZ>(bf_lo(w3), r), mul<RZ>(bf_hi(w3), r));
 }
@@ -604,8 +647,9 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
       if (rho != 0.0f) {
         const float r = block_rho(rho, sc >> 3);
         if (MODE != kSR) {
-          c0 = cvt_words<RZ, U>(w[0], w[1], w[2], w[3], r);
-          c1 = cvt_words<RZ, U>(w[4], w[5], w[6], w[7], r);
+          // normal E4M3 scale: y <= 7 (1 + 1/16) (1 + 2^-20) < 7.5, no clamp
+          c0 = cvt_words<RZ, U, false>(w[0], w[1], w[2], w[3], r);
+          c1 = cvt_words<RZ, U, false>(w[4], w[5], w[6], w[7], r);
           return;
         } else {
           // stochastic rounding on the codeword-safe product; rare
@@ -702,6 +746,7 @@ __device__ __forceinline__ void report_bad(bool bad, int32_t* status) {
 // are the ones the amax pass read last (still in L2).
 template <int FMT, int MODE, class SEG>
 __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
+  pdl_enter();
   constexpr int U = 2;  // blocks per lane per iteration
   __shared__ SegTables tb;
   const int64_t ci = (int64_t)gridDim.x - 1 - blockIdx.x;
@@ -846,6 +891,7 @@ __device__ __forceinline__ uint32_t fix_mismatches(uint32_t c, uint32_t mm, uint
 
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
+  pdl_enter();
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;  // elements per block
   constexpr int NW = BE / 2;                       // bf16 pair words per block
@@ -953,9 +999,7 @@ struct GuidedFqArgs {
 // Four bf16 (two words) times r -> four grid nibbles (16 bits).
 template <bool RZ, bool U = false>
 __device__ __forceinline__ uint32_t cvt_words4(uint32_t w0, uint32_t w1, float r) {
-  if constexpr (U)
-    return cvt_uni_x8(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r), mul<RZ>(bf_hi(w1), r),
-                      0.0f, 0.0f, 0.0f, 0.0f);
+  if constexpr (U) return __byte_perm(nib_pairs(uni_bytes4<RZ, true>(w0, w1, r)), 0u, 0x4420) & 0xFFFFu;
   uint32_t c;
   asm("{\n\t.reg .b8 q0, q1;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
@@ -969,6 +1013,7 @@ __device__ __forceinline__ uint32_t cvt_words4(uint32_t w0, uint32_t w1, float r
 
 template <int FMT, class SEG, bool BF16>
 __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg) {
+  pdl_enter();
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int QPB = BE / 4;  // quads per block
@@ -1080,6 +1125,7 @@ __device__ __forceinline__ int grid_index(uint32_t nib) {
 
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) {
+  pdl_enter();
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int NW = BE / 2;
@@ -1150,6 +1196,7 @@ struct DequantArgs {
 // store covers 512 contiguous bytes.  Segment pieces are whole blocks.
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
+  pdl_enter();
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int QPB = BE / 4;  // quads per block
   constexpr int U = 4;         // quads per lane per iteration
@@ -1193,6 +1240,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
 // unit (16 elements, when rows*cols % 32 == 16) is done by the last thread.
 __global__ void __launch_bounds__(kThreads) k_pack(const uint8_t* __restrict__ codes, uint8_t* bits,
                                                    int64_t nunits, int tail) {
+  pdl_enter();
   constexpr int U = 4;
   const int64_t u0 = cta_begin(blockIdx.x, gridDim.x, nunits);
   const int64_t u1 = cta_begin(blockIdx.x + 1, gridDim.x, nunits);
@@ -1233,6 +1281,7 @@ __device__ __forceinline__ uint2 spread8(uint32_t b) {
 // lanes on consecutive units, so every warp store covers 512 contiguous bytes.
 __global__ void __launch_bounds__(kThreads) k_unpack(const uint8_t* __restrict__ bits, uint8_t* mant,
                                                      int64_t nunits) {
+  pdl_enter();
   constexpr int U = 4;
   const int64_t u0 = cta_begin(blockIdx.x, gridDim.x, nunits);
   const int64_t u1 = cta_begin(blockIdx.x + 1, gridDim.x, nunits);

@@ -123,6 +123,26 @@ tf4_status launched() {
   return cudaGetLastError() == cudaSuccess ? TF4_OK : TF4_ERR_CUDA;
 }
 
+// Launch with programmatic stream serialization: the kernel may be
+// scheduled while the previous grid in the stream is finishing; every
+// kernel of the library waits for that grid (griddepcontrol.wait) before
+// touching memory, so ordering is as for a plain launch, minus the launch
+// gap.  Errors are left for launched().
+template <typename... KArgs, typename... Args>
+void launch_k(void (*kernel)(KArgs...), int64_t grid, cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
 size_t ws_bytes_for(const Shape& sh) {
   if (!has_tensor_scale(sh.fmt)) return 0;
   return ((size_t)(sh.nseg + 1) * sizeof(uint32_t) + 255) & ~(size_t)255;
@@ -147,10 +167,9 @@ tf4_status launch_amax(const Shape& sh, int64_t grid, const void* x, uint32_t* w
   if (multi(sh)) {
     tf4::SegN seg = make_segn(sh);
     seg.bpr = sh.cols / 16;
-    tf4::k_amax<tf4::SegN, U><<<(unsigned)grid, kThreads, 0, st>>>(x4, nb16, seg, ws, s_t_out, amax_out, status);
+    launch_k(tf4::k_amax<tf4::SegN, U>, grid, st, x4, nb16, seg, ws, s_t_out, amax_out, status);
   } else {
-    tf4::k_amax<tf4::Seg1, U><<<(unsigned)grid, kThreads, 0, st>>>(x4, nb16, tf4::Seg1{}, ws, s_t_out, amax_out,
-                                                                    status);
+    launch_k(tf4::k_amax<tf4::Seg1, U>, grid, st, x4, nb16, tf4::Seg1{}, ws, s_t_out, amax_out, status);
   }
   return launched();
 }
@@ -202,9 +221,9 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
           a.st_from_amax = 0;
         }
         if (multi(sh))
-          tf4::k_quant<FMT, MODE, tf4::SegN><<<(unsigned)grid, kThreads, 0, st>>>(a, make_segn(sh));
+          launch_k(tf4::k_quant<FMT, MODE, tf4::SegN>, grid, st, a, make_segn(sh));
         else
-          tf4::k_quant<FMT, MODE, tf4::Seg1><<<(unsigned)grid, kThreads, 0, st>>>(a, tf4::Seg1{});
+          launch_k(tf4::k_quant<FMT, MODE, tf4::Seg1>, grid, st, a, tf4::Seg1{});
       }
     });
     if (e != TF4_OK) return e;
@@ -213,7 +232,7 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
     a.st_from_amax = 0;
     a.s_t_out = nullptr;
     const int64_t grid = wave_grid(tf4::k_quant<TF4_MXFP4, MODE, tf4::Seg1>, sh.nblocks);
-    tf4::k_quant<TF4_MXFP4, MODE, tf4::Seg1><<<(unsigned)grid, kThreads, 0, st>>>(a, tf4::Seg1{});
+    launch_k(tf4::k_quant<TF4_MXFP4, MODE, tf4::Seg1>, grid, st, a, tf4::Seg1{});
   }
   return launched();
 }
@@ -403,10 +422,10 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const 
       constexpr int FMT = decltype(f)::value;
       if constexpr (tf4::kE4M3<FMT>) {
         const int64_t grid = wave_grid(tf4::k_quant<FMT, tf4::kCAPTURE, tf4::SegBatch>, total);
-        tf4::k_amax<tf4::SegBatch, tf4::kUni<FMT>><<<(unsigned)grid, kThreads, 0, st>>>(
-            nullptr, total, sb, static_cast<uint32_t*>(ws), s_t, nullptr, status);
+        launch_k(tf4::k_amax<tf4::SegBatch, tf4::kUni<FMT>>, grid, st, nullptr, total, sb,
+                 static_cast<uint32_t*>(ws), s_t, nullptr, status);
         if ((e = launched()) != TF4_OK) return;
-        tf4::k_quant<FMT, tf4::kCAPTURE, tf4::SegBatch><<<(unsigned)grid, kThreads, 0, st>>>(a, sb);
+        launch_k(tf4::k_quant<FMT, tf4::kCAPTURE, tf4::SegBatch>, grid, st, a, sb);
       }
     });
     if (e != TF4_OK) return e;
@@ -414,7 +433,7 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const 
     a.s_t_out = nullptr;
     a.st_src = nullptr;
     const int64_t grid = wave_grid(tf4::k_quant<TF4_MXFP4, tf4::kCAPTURE, tf4::SegBatch>, total);
-    tf4::k_quant<TF4_MXFP4, tf4::kCAPTURE, tf4::SegBatch><<<(unsigned)grid, kThreads, 0, st>>>(a, sb);
+    launch_k(tf4::k_quant<TF4_MXFP4, tf4::kCAPTURE, tf4::SegBatch>, grid, st, a, sb);
   }
   return launched();
 }
@@ -445,12 +464,12 @@ tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_
     if constexpr (tf4::kE4M3<FMT>) {
       if (multi(sh)) {
         const int64_t g = wave_grid(tf4::k_guided<FMT, tf4::SegN>, sh.nblocks);
-        tf4::k_guided<FMT, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+        launch_k(tf4::k_guided<FMT, tf4::SegN>, g, st, a, make_segn(sh));
         return;
       }
     }
     const int64_t g = wave_grid(tf4::k_guided<FMT, tf4::Seg1>, sh.nblocks);
-    tf4::k_guided<FMT, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+    launch_k(tf4::k_guided<FMT, tf4::Seg1>, g, st, a, tf4::Seg1{});
   });
   return launched();
 }
@@ -481,7 +500,7 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
 #define TF4_LAUNCH_FQ(FMT, SEG, BF, segv)                                             \
   do {                                                                                \
     const int64_t g = wave_grid(tf4::k_guided_fq<FMT, SEG, BF>, sh.nblocks);          \
-    tf4::k_guided_fq<FMT, SEG, BF><<<(unsigned)g, kThreads, 0, st>>>(a, segv);        \
+    launch_k(tf4::k_guided_fq<FMT, SEG, BF>, g, st, a, segv);                         \
   } while (0)
   by_format(sh.fmt, [&](auto f) {
     constexpr int FMT = decltype(f)::value;
@@ -525,12 +544,12 @@ tf4_status tf4_mismatch_stats(const tf4_desc* desc, const void* x, const uint8_t
     if constexpr (tf4::kE4M3<FMT>) {
       if (multi(sh)) {
         const int64_t g = wave_grid(tf4::k_mismatch<FMT, tf4::SegN>, sh.nblocks);
-        tf4::k_mismatch<FMT, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+        launch_k(tf4::k_mismatch<FMT, tf4::SegN>, g, st, a, make_segn(sh));
         return;
       }
     }
     const int64_t g = wave_grid(tf4::k_mismatch<FMT, tf4::Seg1>, sh.nblocks);
-    tf4::k_mismatch<FMT, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+    launch_k(tf4::k_mismatch<FMT, tf4::Seg1>, g, st, a, tf4::Seg1{});
   });
   return launched();
 }
@@ -556,12 +575,12 @@ tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint
     if constexpr (tf4::kE4M3<FMT>) {
       if (multi(sh)) {
         const int64_t g = wave_grid(tf4::k_dequant<FMT, tf4::SegN>, sh.nblocks);
-        tf4::k_dequant<FMT, tf4::SegN><<<(unsigned)g, kThreads, 0, st>>>(a, make_segn(sh));
+        launch_k(tf4::k_dequant<FMT, tf4::SegN>, g, st, a, make_segn(sh));
         return;
       }
     }
     const int64_t g = wave_grid(tf4::k_dequant<FMT, tf4::Seg1>, sh.nblocks);
-    tf4::k_dequant<FMT, tf4::Seg1><<<(unsigned)g, kThreads, 0, st>>>(a, tf4::Seg1{});
+    launch_k(tf4::k_dequant<FMT, tf4::Seg1>, g, st, a, tf4::Seg1{});
   });
   return launched();
 }
@@ -576,7 +595,7 @@ tf4_status tf4_pack_guidance(const tf4_desc* desc, const uint8_t* codes, uint8_t
   const int64_t units = sh.n / 32;
   const int tail = (sh.n % 32) != 0;
   const int64_t g = wave_grid(tf4::k_pack, units > 0 ? units : 1);
-  tf4::k_pack<<<(unsigned)g, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(codes, bits, units, tail);
+  launch_k(tf4::k_pack, g, reinterpret_cast<cudaStream_t>(stream), codes, bits, units, tail);
   return launched();
 }
 
@@ -589,7 +608,7 @@ tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_
   if (!aligned(bits, 4) || !aligned(mant, 16)) return TF4_ERR_ALIGN;
   const int64_t units = sh.n / 16;  // rows*cols is a multiple of 16
   const int64_t g = wave_grid(tf4::k_unpack, units);
-  tf4::k_unpack<<<(unsigned)g, kThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(bits, mant, units);
+  launch_k(tf4::k_unpack, g, reinterpret_cast<cudaStream_t>(stream), bits, mant, units);
   return launched();
 }
 
