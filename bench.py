@@ -57,12 +57,17 @@ def parse():
     p.add_argument("--rows", type=int, default=65536)
     p.add_argument("--cols", type=int, default=4096)
     p.add_argument("--e2e-steps", type=int, default=2)
+    p.add_argument("--event-every", type=int, default=10,
+                   help="per-kernel CUDA events on every n-th timed step (an event between two launches "
+                        "costs a few microseconds of idle GPU and stops the next launch from overlapping)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--cpu-rows", type=int, default=256, help="rows per layer in the oracle sample")
     p.add_argument("--ref-rows", type=int, default=48, help="rows per layer per reference step")
     p.add_argument("--suite", action="store_true",
                    help="time every call of the path on every workload (a table, not the bench line)")
+    p.add_argument("--only", action="append",
+                   help="with --suite: run only rows matching workload-prefix[:format[:call]] (repeatable)")
     return p.parse_args()
 
 
@@ -256,8 +261,11 @@ def run_ours(args, world, rank, local):
         step(None)
     torch.cuda.synchronize()
     assert B.read_status(dev) == 0, "non-finite input in the workload"
-    # per-kernel events for every timed step, read after the timed region
-    evs = [dict(amax=new_events(L), quant=new_events(L), guided=new_events(D)) for _ in range(args.steps)]
+    # per-kernel events on every event_every-th timed step, read after the timed region
+    every = max(1, args.event_every)
+    evs = [dict(amax=new_events(L), quant=new_events(L), guided=new_events(D)) if k % every == 0 else None
+           for k in range(args.steps)]
+    instrumented = [k for k in range(args.steps) if evs[k] is not None]
 
     clocks = Clocks(local)
     barrier(world)
@@ -273,7 +281,8 @@ def run_ours(args, world, rank, local):
     clk = clocks.stop()
     ms_total = t0.elapsed_time(t1)
     ms_step = max_over_ranks(ms_total / args.steps, world, dev)
-    times = {k: [[a.elapsed_time(b) for a, b in e[k]] for e in evs] for k in ("amax", "quant", "guided")}
+    times = {k: [[a.elapsed_time(b) for a, b in e[k]] for e in evs if e is not None]
+             for k in ("amax", "quant", "guided")}
 
     bytes_step, elems_step = step_bytes(args)
     value = world * bytes_step / (ms_step * 1e-3) / 1e9
@@ -315,7 +324,8 @@ def run_ours(args, world, rank, local):
                                     f"of those layers",
                            layers=L, deep_layers=D, rows=args.rows, cols=args.cols, format="NVFP4",
                            parallelism=f"dp{world} (independent stacks)",
-                           l2="inputs 512 MiB per layer > 126 MB L2; no flush"),
+                           l2="inputs 512 MiB per layer > 126 MB L2; no flush",
+                           per_kernel_events=f"timed steps {instrumented} of {args.steps}"),
                frac_of_peak=round(value / world / peak, 4),
                frac_of_datasheet=round(value / world / DATASHEET_HBM_GBS, 4),
                elements_per_s=round(world * elems_step / (ms_step * 1e-3), 1),
@@ -540,6 +550,19 @@ def run_suite(args):
         torch.cuda.synchronize()
         return a.elapsed_time(b) / reps * 1e3  # us
 
+    only = [tuple(f.split(":")) + ("", "", "") for f in (args.only or [])]
+
+    def sel(workload, fmt="", call=""):
+        """Is (workload, format, call) selected by --only (prefix match per field)?"""
+        if not only:
+            return True
+        return any(workload.startswith(w) and (not fmt or not f or fmt == f) and (not call or not c or call == c)
+                   for w, f, c, *_ in only)
+
+    def run(workload, fmt, call, n, fn, **extra):
+        if sel(workload, fmt, call):
+            record(workload, fmt, call, n, timed(fn), **extra)
+
     def record(workload, fmt, call, n, us, **extra):
         gbs = CALL_BYTES[(fmt, call)] * n / (us * 1e-6) / 1e9
         rows_out.append(dict(workload=workload, format=fmt, call=call, elements=n, us=round(us, 2),
@@ -549,8 +572,10 @@ def run_suite(args):
         n = x.numel()
         yf = torch.empty(x.shape, dtype=torch.float32, device=dev)
         yb = torch.empty(x.shape, dtype=torch.bfloat16, device=dev)
-        record(name, fmt, "guided_fq_f32", n, timed(lambda: B.tf4_guided_fake_quant(xt, q, out=yf)))
-        record(name, fmt, "guided_fq_bf16", n, timed(lambda: B.tf4_guided_fake_quant(xt, q, out=yb)))
+        run(name, fmt, "guided_fq_f32", n, lambda: B.tf4_guided_fake_quant(xt, q, out=yf))
+        run(name, fmt, "guided_fq_bf16", n, lambda: B.tf4_guided_fake_quant(xt, q, out=yb))
+        if not sel(name, fmt, "mismatch"):
+            return
         cnt = torch.zeros(4, dtype=torch.int64, device=dev)
         us = timed(lambda: B.tf4_mismatch_stats(xt, q, counts=cnt.zero_()))
         c = [int(v) for v in B.tf4_mismatch_stats(xt, q).tolist()]
@@ -566,15 +591,15 @@ def run_suite(args):
         bits = torch.empty(n // 8, dtype=torch.uint8, device=dev)
         mant = torch.empty(n, dtype=torch.uint8, device=dev)
         qr = B.tf4_quantize_rtn(x, seg_off=seg)
-        record(name, "nvfp4", "amax", n, timed(lambda: B.tf4_segment_amax(x, seg, out=amax)))
-        record(name, "nvfp4", "rtn", n, timed(lambda: B.tf4_quantize_rtn(x, seg_off=seg, out=qr)))
-        record(name, "nvfp4", "capture", n, timed(lambda: B.tf4_quantize_capture(x, seg_off=seg, out=q)))
-        record(name, "nvfp4", "guided", n, timed(lambda: B.tf4_quantize_guided(xt, q, out=g)))
-        record(name, "nvfp4", "sr", n, timed(lambda: B.tf4_quantize_sr(x, 4, seg_off=seg, out=qr)))
-        record(name, "nvfp4", "dequant", n, timed(lambda: B.tf4_dequantize(q, out=out)))
+        run(name, "nvfp4", "amax", n, lambda: B.tf4_segment_amax(x, seg, out=amax))
+        run(name, "nvfp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, seg_off=seg, out=qr))
+        run(name, "nvfp4", "capture", n, lambda: B.tf4_quantize_capture(x, seg_off=seg, out=q))
+        run(name, "nvfp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g))
+        run(name, "nvfp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, seg_off=seg, out=qr))
+        run(name, "nvfp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out))
         rows, cols = x.shape
-        record(name, "any", "pack", n, timed(lambda: B.tf4_pack_guidance(q.codes, rows, cols, out=bits)))
-        record(name, "any", "unpack", n, timed(lambda: B.tf4_unpack_guidance(bits, rows, cols, out=mant)))
+        run(name, "any", "pack", n, lambda: B.tf4_pack_guidance(q.codes, rows, cols, out=bits))
+        run(name, "any", "unpack", n, lambda: B.tf4_unpack_guidance(bits, rows, cols, out=mant))
         fq_and_diag(name, "nvfp4", q, x, xt)
         del q, g, out, bits, mant, qr
 
@@ -585,11 +610,11 @@ def run_suite(args):
         g = torch.empty_like(q.codes)
         out = torch.empty(x.shape, dtype=torch.float32, device=dev)
         qr = B.tf4_quantize_rtn(x, fmt=U, seg_off=seg)
-        record(name, "ufp4", "rtn", n, timed(lambda: B.tf4_quantize_rtn(x, fmt=U, seg_off=seg, out=qr)))
-        record(name, "ufp4", "capture", n, timed(lambda: B.tf4_quantize_capture(x, fmt=U, seg_off=seg, out=q)))
-        record(name, "ufp4", "guided", n, timed(lambda: B.tf4_quantize_guided(xt, q, out=g)))
-        record(name, "ufp4", "sr", n, timed(lambda: B.tf4_quantize_sr(x, 4, fmt=U, seg_off=seg, out=qr)))
-        record(name, "ufp4", "dequant", n, timed(lambda: B.tf4_dequantize(q, out=out)))
+        run(name, "ufp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, fmt=U, seg_off=seg, out=qr))
+        run(name, "ufp4", "capture", n, lambda: B.tf4_quantize_capture(x, fmt=U, seg_off=seg, out=q))
+        run(name, "ufp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g))
+        run(name, "ufp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, fmt=U, seg_off=seg, out=qr))
+        run(name, "ufp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out))
         fq_and_diag(name, "ufp4", q, x, xt)
         del q, g, out, qr
 
@@ -604,9 +629,9 @@ def run_suite(args):
         def per_layer():
             for i, x in enumerate(xs):
                 B.tf4_quantize_capture(x, fmt=fmt, guidance=i >= L - keep, out=per[i])
-        record(name, fname, "capture_stack_half_kept", n, timed(per_layer), launch="per_layer")
-        record(name, fname, "capture_stack_half_kept", n,
-               timed(lambda: B.tf4_quantize_capture_batched(xs, fmt=fmt, keep=keep, out=ob)), launch="batched")
+        run(name, fname, "capture_stack_half_kept", n, per_layer, launch="per_layer")
+        run(name, fname, "capture_stack_half_kept", n,
+            lambda: B.tf4_quantize_capture_batched(xs, fmt=fmt, keep=keep, out=ob), launch="batched")
         del ob, per
 
     def mx_calls(name, x, xt):
@@ -617,41 +642,55 @@ def run_suite(args):
         g = torch.empty_like(q.codes)
         out = torch.empty(x.shape, dtype=torch.float32, device=dev)
         qr = B.tf4_quantize_rtn(x, fmt=B.MXFP4)
-        record(name, "mxfp4", "rtn", n, timed(lambda: B.tf4_quantize_rtn(x, fmt=B.MXFP4, out=qr)))
-        record(name, "mxfp4", "capture", n, timed(lambda: B.tf4_quantize_capture(x, fmt=B.MXFP4, out=q)))
-        record(name, "mxfp4", "guided", n, timed(lambda: B.tf4_quantize_guided(xt, q, out=g)))
-        record(name, "mxfp4", "sr", n, timed(lambda: B.tf4_quantize_sr(x, 4, fmt=B.MXFP4, out=qr)))
-        record(name, "mxfp4", "dequant", n, timed(lambda: B.tf4_dequantize(q, out=out)))
+        run(name, "mxfp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, fmt=B.MXFP4, out=qr))
+        run(name, "mxfp4", "capture", n, lambda: B.tf4_quantize_capture(x, fmt=B.MXFP4, out=q))
+        run(name, "mxfp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g))
+        run(name, "mxfp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, fmt=B.MXFP4, out=qr))
+        run(name, "mxfp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out))
         fq_and_diag(name, "mxfp4", q, x, xt)
         del q, g, out, qr
 
-    w = W.activation_outliers(dev)
-    nv_calls("activation_outliers 4096x2048", w["x"], w["x_train"])
-    mx_calls("activation_outliers 4096x2048", w["x"], w["x_train"])
-    uf_calls("activation_outliers 4096x2048", w["x"], w["x_train"])
-    del w
-    xs = [W.random_bf16((4096, 2048), seed=300 + i, device=dev, outlier_frac=0.001) for i in range(40)]
-    stack_calls("40 layers of 4096x2048", xs, B.NVFP4, "nvfp4")
-    stack_calls("40 layers of 4096x2048", xs, B.MXFP4, "mxfp4")
-    del xs
-    x = W.layer_stack_layer(20, dev)
-    xt = W.perturb(x, 1020)
-    nv_calls("layer_stack layer 65536x4096", x, xt)
-    mx_calls("layer_stack layer 65536x4096", x, xt)
-    uf_calls("layer_stack layer 65536x4096", x, xt)
-    del x, xt
-    w = W.moe_dispatch(dev)
-    nv_calls("moe_dispatch 262144x2048, 128 experts", w["x"], w["x_train"], seg=w["seg_off"])
-    uf_calls("moe_dispatch 262144x2048, 128 experts", w["x"], w["x_train"], seg=w["seg_off"])
-    del w
-    x = W.weights(dev)
-    nv_calls("weights 8192x28672", x, W.perturb(x, 44))
-    mx_calls("weights 8192x28672", x, W.perturb(x, 44))
-    del x
-    w = W.kv_cache(dev)
-    nv_calls("kv_cache K 1048576x128", w["k"], w["k_train"])
-    mx_calls("kv_cache K 1048576x128", w["k"], w["k_train"])
-    del w
+    name = "activation_outliers 4096x2048"
+    if sel(name):
+        w = W.activation_outliers(dev)
+        nv_calls(name, w["x"], w["x_train"])
+        mx_calls(name, w["x"], w["x_train"])
+        uf_calls(name, w["x"], w["x_train"])
+        del w
+    name = "40 layers of 4096x2048"
+    if sel(name):
+        xs = [W.random_bf16((4096, 2048), seed=300 + i, device=dev, outlier_frac=0.001) for i in range(40)]
+        stack_calls(name, xs, B.NVFP4, "nvfp4")
+        stack_calls(name, xs, B.MXFP4, "mxfp4")
+        del xs
+    name = "layer_stack layer 65536x4096"
+    if sel(name):
+        x = W.layer_stack_layer(20, dev)
+        xt = W.perturb(x, 1020)
+        nv_calls(name, x, xt)
+        mx_calls(name, x, xt)
+        uf_calls(name, x, xt)
+        del x, xt
+    name = "moe_dispatch 262144x2048, 128 experts"
+    if sel(name):
+        w = W.moe_dispatch(dev)
+        nv_calls(name, w["x"], w["x_train"], seg=w["seg_off"])
+        uf_calls(name, w["x"], w["x_train"], seg=w["seg_off"])
+        del w
+    name = "weights 8192x28672"
+    if sel(name):
+        x = W.weights(dev)
+        nv_calls(name, x, W.perturb(x, 44))
+        mx_calls(name, x, W.perturb(x, 44))
+        uf_calls(name, x, W.perturb(x, 44))
+        del x
+    name = "kv_cache K 1048576x128"
+    if sel(name):
+        w = W.kv_cache(dev)
+        nv_calls(name, w["k"], w["k_train"])
+        mx_calls(name, w["k"], w["k_train"])
+        uf_calls(name, w["k"], w["k_train"])
+        del w
     torch.cuda.empty_cache()
     return dict(peak_gbs=peak, peak_kind=peak_kind, rows=rows_out)
 

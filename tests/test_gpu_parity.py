@@ -311,6 +311,23 @@ def test_guided_fake_quant_parity(fmt, seg, dtype):
         assert_same("values", host(y.view(torch.int16)).view(np.uint16), O.f32_to_bf16(vals))
 
 
+@pytest.mark.parametrize("fmt,shape", [(O.NVFP4, (1, 16)), (O.NVFP4, (3, 48)), (O.UFP4, (5, 16 * 33)), (O.MXFP4, (3, 64)),
+                                       (O.MXFP4, (1, 32))])
+def test_guided_fake_quant_small_shapes(fmt, shape):
+    """Single blocks and ragged block counts through the fused pass."""
+    xb = W.random_bf16(shape, seed=sum(shape) + 5, device=DEV, outlier_frac=0.05)
+    q, r = check_quant(xb, fmt)
+    xt = W.perturb(xb, 45, rel=0.05)
+    for dtype in (torch.float32, torch.bfloat16):
+        y, c = B.tf4_guided_fake_quant(xt, q, out_dtype=dtype, want_codes=True)
+        codes, vals, st = O.guided_fake_quant(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"])
+        assert_same("codes", host(c), codes)
+        if dtype == torch.float32:
+            assert_same("values", f32_bits(host(y)), f32_bits(vals))
+        else:
+            assert_same("values", host(y.view(torch.int16)).view(np.uint16), O.f32_to_bf16(vals))
+
+
 @pytest.mark.parametrize("fmt,seg", [(O.NVFP4, None), (O.NVFP4, [0, 30, 30, 64]), (O.MXFP4, None), (O.UFP4, None),
                                      (O.UFP4, [0, 30, 30, 64])])
 @pytest.mark.parametrize("rel", [1e-3, 0.05, None])
