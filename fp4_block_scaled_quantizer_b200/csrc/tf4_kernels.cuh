@@ -203,6 +203,13 @@ __device__ __forceinline__ float4 decode4_grid(uint32_t c, float S) {
   else return decode4(c, S);
 }
 
+// One 32-byte store (sm_100 256-bit vector store); p must be 32-B aligned.
+__device__ __forceinline__ void st_v8(float* p, const float4& a, const float4& b) {
+  asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(a.x), "f"(a.y), "f"(a.z),
+               "f"(a.w), "f"(b.x), "f"(b.y), "f"(b.z), "f"(b.w)
+               : "memory");
+}
+
 // m3 & 1 of eight nibbles -> eight bits (nibble k -> bit k).  The masked
 // bits sit at 4k; multiplying by 0x1248 (= 2^3 + 2^6 + 2^9 + 2^12) sends bit
 // 4k to 12 + k for k < 4 and to 24 + k for k >= 4, and every other partial
@@ -305,25 +312,80 @@ __device__ __forceinline__ uint32_t guided_m3_exact(float ax, float S, uint32_t 
   return f + ((f ^ g) & 1u);
 }
 
-// Philox4x32-10 (Salmon et al., SC'11), word 0 only, counter (idx, 0, 0),
-// key = seed.
-__device__ __forceinline__ uint32_t philox_w0(uint64_t idx, uint64_t seed) {
-  uint32_t c0 = (uint32_t)idx, c1 = (uint32_t)(idx >> 32), c2 = 0u, c3 = 0u;
-  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+// Philox4x32-10 (Salmon et al., SC'11), word 0 only, counter
+// (idx mod 2^32, idx >> 32, 0, 0), key = seed.  One round maps
+// (c0, c1, c2, c3) to (hi(M1 c2) ^ c1 ^ k0, lo(M1 c2), hi(M0 c0) ^ c3 ^ k1,
+// lo(M0 c0)); round j (0..9) uses the key (k0 + j W0, k1 + j W1).  The
+// quantize kernels take that schedule as kernel parameters (ks[2j],
+// ks[2j+1]) so the round keys are constant-bank operands.  Elements of one
+// quantization block share idx >> 32 (blocks of 16 or 32 never straddle a
+// multiple of 2^32), which makes round 2's M0 product the same for the
+// whole block (PhiloxBlk).  With the zero words of the counter, round 1 has
+// one product, and round 10 needs only hi(M1 c2) for word 0.
+constexpr uint32_t kPhiloxM0 = 0xD2511F53u, kPhiloxM1 = 0xCD9E8D57u;
+constexpr uint32_t kPhiloxW0 = 0x9E3779B9u, kPhiloxW1 = 0xBB67AE85u;
+constexpr int kPhiloxKeys = 20;
+
+__device__ __forceinline__ void mulhilo(uint32_t m, uint32_t c, uint32_t& hi, uint32_t& lo) {
+  const uint64_t p = (uint64_t)m * c;
+  hi = (uint32_t)(p >> 32);
+  lo = (uint32_t)p;
+}
+
+struct PhiloxBlk {
+  uint32_t c1;        // idx >> 32 of the block
+  uint32_t hi2, lo2;  // round 2: M0 * (c1 ^ k0)
+};
+
+__device__ __forceinline__ PhiloxBlk philox_block(uint64_t first_idx, const uint32_t* ks) {
+  PhiloxBlk b;
+  b.c1 = (uint32_t)(first_idx >> 32);
+  mulhilo(kPhiloxM0, b.c1 ^ ks[0], b.hi2, b.lo2);
+  return b;
+}
+
+// Word 0 for counter (lo32, b.c1, 0, 0) under key schedule ks.
+__device__ __forceinline__ uint32_t philox_w0_blk(uint32_t lo32, const PhiloxBlk& b, const uint32_t* ks) {
+  uint32_t hi0, lo0, hi1, lo1;
+  // round 1 (c2 = c3 = 0, so M1 c2 = 0): c0 <- c1_in ^ k0, whose M0 product
+  // is the block's (b.hi2, b.lo2); c1 <- 0; c2, c3 from M0 lo32
+  mulhilo(kPhiloxM0, lo32, hi0, lo0);
+  uint32_t c2 = hi0 ^ ks[1], c3 = lo0;
+  // round 2
+  mulhilo(kPhiloxM1, c2, hi1, lo1);
+  uint32_t c0 = hi1 ^ ks[2];  // ^ c1, which is 0
+  uint32_t c1 = lo1;
+  c2 = b.hi2 ^ c3 ^ ks[3];
+  c3 = b.lo2;
 #pragma unroll
-  for (int r = 0; r < 10; ++r) {
-    if (r) {
-      k0 += 0x9E3779B9u;
-      k1 += 0xBB67AE85u;
-    }
-    const uint32_t hi0 = __umulhi(0xD2511F53u, c0), lo0 = 0xD2511F53u * c0;
-    const uint32_t hi1 = __umulhi(0xCD9E8D57u, c2), lo1 = 0xCD9E8D57u * c2;
-    c0 = hi1 ^ c1 ^ k0;
+  for (int j = 2; j < 9; ++j) {
+    mulhilo(kPhiloxM0, c0, hi0, lo0);
+    mulhilo(kPhiloxM1, c2, hi1, lo1);
+    c0 = hi1 ^ c1 ^ ks[2 * j];
     c1 = lo1;
-    c2 = hi0 ^ c3 ^ k1;
+    c2 = hi0 ^ c3 ^ ks[2 * j + 1];
     c3 = lo0;
   }
-  return c0;
+  // round 10: word 0 only
+  return __umulhi(kPhiloxM1, c2) ^ c1 ^ ks[18];
+}
+
+// The key schedule of a seed (host and device).
+__host__ __device__ inline void philox_schedule(uint64_t seed, uint32_t (&ks)[kPhiloxKeys]) {
+  uint32_t k0 = (uint32_t)seed, k1 = (uint32_t)(seed >> 32);
+  for (int j = 0; j < 10; ++j) {
+    ks[2 * j] = k0;
+    ks[2 * j + 1] = k1;
+    k0 += kPhiloxW0;
+    k1 += kPhiloxW1;
+  }
+}
+
+// Word 0 for counter (idx mod 2^32, idx >> 32, 0, 0), key = seed.
+__device__ __forceinline__ uint32_t philox_w0(uint64_t idx, uint64_t seed) {
+  uint32_t ks[kPhiloxKeys];
+  philox_schedule(seed, ks);
+  return philox_w0_blk((uint32_t)idx, philox_block(idx, ks), ks);
 }
 
 // SR m3 of |x| on scale S > 0 with a 24-bit uniform r.  Every product of a
@@ -617,6 +679,13 @@ __device__ __forceinline__ uint32_t cvt_words(uint32_t w0, uint32_t w1, uint32_t
 // --------------------------------------------------------- quantize pass
 enum { kRTN = 0, kSR = 1, kCAPTURE = 2 };
 
+// Philox key schedule of the SR seed (philox_schedule), a kernel parameter
+// of its own: inside QuantArgs it raised every quantize variant's register
+// count (48 -> 57-64 for RTN/capture), costing a resident CTA per SM.
+struct PhiloxKeys {
+  uint32_t ks[kPhiloxKeys];
+};
+
 struct QuantArgs {
   const uint4* x;
   int64_t nblocks;
@@ -634,7 +703,7 @@ struct QuantArgs {
 // NVFP4, uniform grid if U) -> code words, scale byte, flags.
 template <bool U, int MODE, bool RZ>
 __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, const SegTables& t,
-                                            int64_t blk, uint64_t seed, uint32_t& c0, uint32_t& c1,
+                                            int64_t blk, const uint32_t* ks, uint32_t& c0, uint32_t& c1,
                                             uint32_t& sc, bool& bad) {
   const uint32_t mb = block_absmax_bits(w);
   bad = mb >= 0x7F80u;
@@ -655,19 +724,27 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
           // stochastic rounding on the codeword-safe product; rare
           // ambiguous thresholds are decided exactly
           const float S = __fmul_rn(st, e4m3_decode(sc));
-          float v[16];
+          const PhiloxBlk pb = philox_block((uint64_t)blk * 16u, ks);
+          const uint32_t lo32 = (uint32_t)((uint64_t)blk * 16u);
+          uint32_t c[2];
 #pragma unroll
-          for (int k = 0; k < 16; ++k) {
-            const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
-            const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-            const uint32_t r24 = philox_w0((uint64_t)blk * 16u + k, seed) >> 8;
-            bool amb;
-            float val = sr_pick<U>(mul<RZ>(ax, r), r24, true, amb);
-            if (amb) val = grid_value<U>(sr_m3_exact<U>(ax, S, r24));
-            v[k] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
+          for (int q = 0; q < 2; ++q) {  // 8 elements at a time
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const int k = 8 * q + e;
+              const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
+              const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+              const uint32_t r24 = philox_w0_blk(lo32 + (uint32_t)k, pb, ks) >> 8;
+              bool amb;
+              float val = sr_pick<U>(mul<RZ>(ax, r), r24, true, amb);
+              if (amb) val = grid_value<U>(sr_m3_exact<U>(ax, S, r24));
+              v[e] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
+            }
+            c[q] = cvt_grid_x8<U>(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
           }
-          c0 = cvt_grid_x8<U>(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
-          c1 = cvt_grid_x8<U>(v[8], v[9], v[10], v[11], v[12], v[13], v[14], v[15]);
+          c0 = c[0];
+          c1 = c[1];
           return;
         }
       }
@@ -690,8 +767,9 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
     const float ax = __uint_as_float((h & 0x7FFFu) << 16);
     uint32_t m3 = 0;
     if (S > 0.0f) {
-      if (MODE == kSR)
-        m3 = sr_m3_exact<U>(ax, S, philox_w0((uint64_t)blk * 16u + k, seed) >> 8);
+      if constexpr (MODE == kSR)
+        m3 = sr_m3_exact<U>(ax, S, philox_w0_blk((uint32_t)((uint64_t)blk * 16u) + (uint32_t)k,
+                                                 philox_block((uint64_t)blk * 16u, ks), ks) >> 8);
       else
         m3 = rtn_m3_exact<U>(ax, S);
     }
@@ -703,7 +781,7 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
 
 // One MXFP4 block (32 bf16 in w[0..15]) -> code words, scale byte, flags.
 template <int MODE>
-__device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk, uint64_t seed,
+__device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk, const uint32_t* ks,
                                             uint32_t (&c)[4], uint32_t& sc, bool& bad) {
   const uint32_t mb = block_absmax_bits(w);
   bad = mb >= 0x7F80u;
@@ -721,13 +799,15 @@ __device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk
   }
   // stochastic rounding on the exact quotient y = |x| * 2^-e
   const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
+  const PhiloxBlk pb = philox_block((uint64_t)blk * 32u, ks);
+  const uint32_t lo32 = (uint32_t)((uint64_t)blk * 32u);
   float v[32];
 #pragma unroll
   for (int k = 0; k < 32; ++k) {
     const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
     const float ax = __uint_as_float((h & 0x7FFFu) << 16);
     bool amb;
-    const float val = sr_pick(__fmul_rn(ax, inv), philox_w0((uint64_t)blk * 32u + k, seed) >> 8, false, amb);
+    const float val = sr_pick(__fmul_rn(ax, inv), philox_w0_blk(lo32 + (uint32_t)k, pb, ks) >> 8, false, amb);
     v[k] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
   }
 #pragma unroll
@@ -745,9 +825,12 @@ __device__ __forceinline__ void report_bad(bool bad, int32_t* status) {
 // gets range G-1-i) and walk them backwards, so that the first blocks read
 // are the ones the amax pass read last (still in L2).
 template <int FMT, int MODE, class SEG>
-__global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
+__global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg, PhiloxKeys pk) {
   pdl_enter();
-  constexpr int U = 2;  // blocks per lane per iteration
+  // blocks per lane per iteration: 2 keeps 64 B per lane in flight for the
+  // memory-bound modes; stochastic rounding is bound by the integer pipe
+  // and gains more from the registers (resident warps) one block saves
+  constexpr int U = MODE == kSR ? 1 : 2;
   __shared__ SegTables tb;
   const int64_t ci = (int64_t)gridDim.x - 1 - blockIdx.x;
   const int64_t b0 = cta_begin(ci, gridDim.x, a.nblocks);
@@ -790,9 +873,9 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
           if (valid) {
             uint32_t c0, c1, sc;
             if (tb.rz)
-              nvfp4_block<UG, MODE, true>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
+              nvfp4_block<UG, MODE, true>(w[u], st, tb, blk[u], pk.ks, c0, c1, sc, bad);
             else
-              nvfp4_block<UG, MODE, false>(w[u], st, tb, blk[u], a.seed, c0, c1, sc, bad);
+              nvfp4_block<UG, MODE, false>(w[u], st, tb, blk[u], pk.ks, c0, c1, sc, bad);
             reinterpret_cast<uint2*>(a.codes)[blk[u]] = make_uint2(c0, c1);
             a.scales[blk[u]] = (uint8_t)sc;
             if (MODE == kCAPTURE && bits)
@@ -822,7 +905,7 @@ __global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg) {
           bool bad = false;
           if (valid) {
             uint32_t c[4], sc;
-            mxfp4_block<MODE>(w[u], blk[u], a.seed, c, sc, bad);
+            mxfp4_block<MODE>(w[u], blk[u], pk.ks, c, sc, bad);
             reinterpret_cast<uint4*>(a.codes)[blk[u]] = make_uint4(c[0], c[1], c[2], c[3]);
             a.scales[blk[u]] = (uint8_t)sc;
             if (MODE == kCAPTURE && bits)
@@ -983,41 +1066,37 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
 // Train-side forward in one pass: guided quantization of x against the
 // rollout record, then dequantization of the chosen codes, written as fp32
 // or as bf16 (round-to-nearest-even of the fp32 value), and optionally the
-// codes.  Work unit = a quad of 4 consecutive elements (8 B of x in), so
-// consecutive lanes write consecutive 16-B (fp32) / 8-B (bf16) outputs.
+// codes.  Work unit = an oct of 8 consecutive elements (16 B of x in, one
+// guidance byte, one code word out), so consecutive lanes read 16-B and
+// write 16-B (bf16) / 2 x 16-B (fp32) pieces of one contiguous span.
 struct GuidedFqArgs {
-  const uint2* x;         // bf16 quads
+  const uint4* x;         // bf16 octs
   int64_t nblocks;
   const uint8_t* rec_scales;
   const float* rec_s_t;
   const uint8_t* rec_bits;
   uint8_t* codes;         // may be NULL
-  void* out;              // float4 (fp32) or uint2 (bf16) per quad
+  void* out;              // 2 x float4 (fp32) or uint4 (bf16) per oct
   int32_t* status;
 };
 
-// Four bf16 (two words) times r -> four grid nibbles (16 bits).
-template <bool RZ, bool U = false>
-__device__ __forceinline__ uint32_t cvt_words4(uint32_t w0, uint32_t w1, float r) {
-  if constexpr (U) return __byte_perm(nib_pairs(uni_bytes4<RZ, true>(w0, w1, r)), 0u, 0x4420) & 0xFFFFu;
-  uint32_t c;
-  asm("{\n\t.reg .b8 q0, q1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
-      "mov.b32 %0, {q0, q1, q1, q1};\n\t}"
-      : "=r"(c)
-      : "f"(mul<RZ>(bf_lo(w0), r)), "f"(mul<RZ>(bf_hi(w0), r)), "f"(mul<RZ>(bf_lo(w1), r)),
-        "f"(mul<RZ>(bf_hi(w1), r)));
-  return c & 0xFFFFu;
+__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
+  const __nv_bfloat162 p = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&p);
 }
 
-template <int FMT, class SEG, bool BF16>
+// Output modes of the fused pass.
+enum { kOutBf16 = 0, kOutF32 = 1, kOutF32V8 = 2 };
+
+// OUT: kOutBf16 (one 16-B store per oct), kOutF32 (two 16-B stores),
+// kOutF32V8 (one 32-B store; the host picks it only for a 32-B aligned out).
+template <int FMT, class SEG, int OUT>
 __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
-  constexpr int QPB = BE / 4;  // quads per block
-  constexpr int U = 2;         // quads per lane per iteration
+  constexpr int OPB = BE / 8;  // octs per block
+  constexpr int U = 2;         // octs per lane per iteration
   __shared__ SegTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
@@ -1031,26 +1110,26 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
       st = a.rec_s_t[s];
       build_tables<UG, false>(st, tb);
     }
-    const int64_t q0 = lo * QPB, q1 = hi * QPB;
-    for (int64_t qb = q0; qb < q1; qb += (int64_t)U * kThreads) {
-      uint2 xv[U];
-      uint32_t sc[U], gq[U];
+    const int64_t o0 = lo * OPB, o1 = hi * OPB;
+    for (int64_t ob = o0; ob < o1; ob += (int64_t)U * kThreads) {
+      uint4 xv[U];
+      uint32_t sc[U], g[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int64_t q = qb + u * kThreads + tid;
-        if (q < q1) {
-          xv[u] = __ldg(a.x + q);
-          sc[u] = __ldg(a.rec_scales + q / QPB);
-          gq[u] = (__ldg(a.rec_bits + (q >> 1)) >> (4 * (q & 1))) & 0xFu;  // 4 bits of this quad
+        const int64_t o = ob + u * kThreads + tid;
+        if (o < o1) {
+          xv[u] = __ldg(a.x + o);
+          sc[u] = __ldg(a.rec_scales + o / OPB);
+          g[u] = __ldg(a.rec_bits + o);
         }
       }
 #pragma unroll
       for (int u = 0; u < U; ++u) {
-        const int64_t q = qb + u * kThreads + tid;
+        const int64_t o = ob + u * kThreads + tid;
         bool bad = false;
-        if (q < q1) {
-          const uint32_t m = vmax_u16x2(xv[u].x & 0x7FFF7FFFu, xv[u].y & 0x7FFF7FFFu);
-          bad = max(m & 0xFFFFu, m >> 16) >= 0x7F80u;
+        if (o < o1) {
+          const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+          bad = block_absmax_bits(w) >= 0x7F80u;
           float r = 0.0f, S;
           bool rz = false;
           if constexpr (kE4M3<FMT>) {
@@ -1063,32 +1142,33 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
             S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
             if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);
           }
-          const uint32_t w0 = xv[u].x, w1 = xv[u].y;
           uint32_t c;
           if (r != 0.0f) {
-            c = rz ? cvt_words4<true, UG>(w0, w1, r) : cvt_words4<false, UG>(w0, w1, r);
-            const uint32_t mm = (c ^ spread_bits(gq[u])) & 0x1111u;
+            c = rz ? cvt_words<true, UG>(w[0], w[1], w[2], w[3], r) : cvt_words<false, UG>(w[0], w[1], w[2], w[3], r);
+            const uint32_t mm = (c ^ spread_bits(g[u])) & 0x11111111u;
             if (mm)
-              c = rz ? fix_mismatches<true, UG>(c, mm, w0, w1, 0u, 0u, r)
-                     : fix_mismatches<false, UG>(c, mm, w0, w1, 0u, 0u, r);
+              c = rz ? fix_mismatches<true, UG>(c, mm, w[0], w[1], w[2], w[3], r)
+                     : fix_mismatches<false, UG>(c, mm, w[0], w[1], w[2], w[3], r);
           } else {
             c = 0u;
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const uint32_t h = (e & 1) ? ((e & 2 ? w1 : w0) >> 16) : ((e & 2 ? w1 : w0) & 0xFFFFu);
+            for (int e = 0; e < 8; ++e) {
+              const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
               const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-              const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (gq[u] >> e) & 1u) : 0u;
+              const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
               c |= (((h >> 15) << 3) | m3) << (4 * e);
             }
           }
-          if (a.codes) reinterpret_cast<uint16_t*>(a.codes)[q] = (uint16_t)c;
-          const float4 v = decode4_grid<UG>(c, S);
-          if constexpr (BF16) {
-            const __nv_bfloat162 p0 = __floats2bfloat162_rn(v.x, v.y), p1 = __floats2bfloat162_rn(v.z, v.w);
-            reinterpret_cast<uint2*>(a.out)[q] =
-                make_uint2(*reinterpret_cast<const uint32_t*>(&p0), *reinterpret_cast<const uint32_t*>(&p1));
+          if (a.codes) reinterpret_cast<uint32_t*>(a.codes)[o] = c;
+          const float4 v0 = decode4_grid<UG>(c & 0xFFFFu, S), v1 = decode4_grid<UG>(c >> 16, S);
+          if constexpr (OUT == kOutBf16) {
+            reinterpret_cast<uint4*>(a.out)[o] = make_uint4(bf16x2_bits(v0.x, v0.y), bf16x2_bits(v0.z, v0.w),
+                                                            bf16x2_bits(v1.x, v1.y), bf16x2_bits(v1.z, v1.w));
+          } else if constexpr (OUT == kOutF32V8) {
+            st_v8(reinterpret_cast<float*>(a.out) + 8 * o, v0, v1);
           } else {
-            reinterpret_cast<float4*>(a.out)[q] = v;
+            reinterpret_cast<float4*>(a.out)[2 * o] = v0;
+            reinterpret_cast<float4*>(a.out)[2 * o + 1] = v1;
           }
         }
         report_bad(bad, a.status);
@@ -1228,6 +1308,51 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
           if constexpr (kE4M3<FMT>) S = __fmul_rn(st, e4m3_decode(sc[u]));
           else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
           a.out[q] = decode4_grid<kUni<FMT>>(cw[u], S);
+        }
+      }
+    }
+    lo = hi;
+  }
+}
+
+// Dequantize with 8 elements per lane (one code word in, one 32-byte store
+// out, so every warp store covers 1 KiB contiguous); the host picks it when
+// out is 32-B aligned.
+template <int FMT, class SEG>
+__global__ void __launch_bounds__(kThreads) k_dequant8(DequantArgs a, SEG seg) {
+  pdl_enter();
+  constexpr int BE = kE4M3<FMT> ? 16 : 32;
+  constexpr int OPB = BE / 8;  // octs per block
+  constexpr int U = 4;         // octs per lane per iteration
+  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
+  const int tid = threadIdx.x;
+  const uint32_t* codes4 = reinterpret_cast<const uint32_t*>(a.codes);
+  float* out = reinterpret_cast<float*>(a.out);
+  int64_t lo = b0;
+  while (lo < b1) {
+    const int s = seg.find(lo);
+    const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
+    const float st = kE4M3<FMT> ? a.s_t[s] : 0.0f;
+    const int64_t o0 = lo * OPB, o1 = hi * OPB;
+    for (int64_t ob = o0; ob < o1; ob += (int64_t)U * kThreads) {
+      uint32_t cw[U], sc[U];
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t o = ob + u * kThreads + tid;
+        if (o < o1) {
+          cw[u] = __ldg(codes4 + o);
+          sc[u] = __ldg(a.scales + o / OPB);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int64_t o = ob + u * kThreads + tid;
+        if (o < o1) {
+          float S;
+          if constexpr (kE4M3<FMT>) S = __fmul_rn(st, e4m3_decode(sc[u]));
+          else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
+          st_v8(out + 8 * o, decode4_grid<kUni<FMT>>(cw[u] & 0xFFFFu, S), decode4_grid<kUni<FMT>>(cw[u] >> 16, S));
         }
       }
     }

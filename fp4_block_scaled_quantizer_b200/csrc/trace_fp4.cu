@@ -204,6 +204,8 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
   a.scales = scales;
   a.bits = bits;
   a.seed = seed;
+  tf4::PhiloxKeys pk;
+  tf4::philox_schedule(seed, pk.ks);
   a.status = status;
   a.s_t_out = s_t;
   if (nv) {
@@ -221,9 +223,9 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
           a.st_from_amax = 0;
         }
         if (multi(sh))
-          launch_k(tf4::k_quant<FMT, MODE, tf4::SegN>, grid, st, a, make_segn(sh));
+          launch_k(tf4::k_quant<FMT, MODE, tf4::SegN>, grid, st, a, make_segn(sh), pk);
         else
-          launch_k(tf4::k_quant<FMT, MODE, tf4::Seg1>, grid, st, a, tf4::Seg1{});
+          launch_k(tf4::k_quant<FMT, MODE, tf4::Seg1>, grid, st, a, tf4::Seg1{}, pk);
       }
     });
     if (e != TF4_OK) return e;
@@ -232,7 +234,7 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
     a.st_from_amax = 0;
     a.s_t_out = nullptr;
     const int64_t grid = wave_grid(tf4::k_quant<TF4_MXFP4, MODE, tf4::Seg1>, sh.nblocks);
-    launch_k(tf4::k_quant<TF4_MXFP4, MODE, tf4::Seg1>, grid, st, a, tf4::Seg1{});
+    launch_k(tf4::k_quant<TF4_MXFP4, MODE, tf4::Seg1>, grid, st, a, tf4::Seg1{}, pk);
   }
   return launched();
 }
@@ -413,6 +415,8 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const 
   a.scales = scales;
   a.bits = info_bits;
   a.seed = 0;
+  tf4::PhiloxKeys pk;
+  tf4::philox_schedule(0, pk.ks);
   a.status = status;
   a.s_t_out = s_t;
   a.st_src = s_t;
@@ -425,7 +429,7 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const 
         launch_k(tf4::k_amax<tf4::SegBatch, tf4::kUni<FMT>>, grid, st, nullptr, total, sb,
                  static_cast<uint32_t*>(ws), s_t, nullptr, status);
         if ((e = launched()) != TF4_OK) return;
-        launch_k(tf4::k_quant<FMT, tf4::kCAPTURE, tf4::SegBatch>, grid, st, a, sb);
+        launch_k(tf4::k_quant<FMT, tf4::kCAPTURE, tf4::SegBatch>, grid, st, a, sb, pk);
       }
     });
     if (e != TF4_OK) return e;
@@ -433,7 +437,7 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t nl, const 
     a.s_t_out = nullptr;
     a.st_src = nullptr;
     const int64_t grid = wave_grid(tf4::k_quant<TF4_MXFP4, tf4::kCAPTURE, tf4::SegBatch>, total);
-    launch_k(tf4::k_quant<TF4_MXFP4, tf4::kCAPTURE, tf4::SegBatch>, grid, st, a, sb);
+    launch_k(tf4::k_quant<TF4_MXFP4, tf4::kCAPTURE, tf4::SegBatch>, grid, st, a, sb, pk);
   }
   return launched();
 }
@@ -489,7 +493,7 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
     return TF4_ERR_ALIGN;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   tf4::GuidedFqArgs a;
-  a.x = static_cast<const uint2*>(x);
+  a.x = static_cast<const uint4*>(x);
   a.nblocks = sh.nblocks;
   a.rec_scales = rec_scales;
   a.rec_s_t = rec_s_t;
@@ -497,22 +501,26 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
   a.codes = codes;
   a.out = out;
   a.status = status;
-#define TF4_LAUNCH_FQ(FMT, SEG, BF, segv)                                             \
+#define TF4_LAUNCH_FQ(FMT, SEG, OUT, segv)                                            \
   do {                                                                                \
-    const int64_t g = wave_grid(tf4::k_guided_fq<FMT, SEG, BF>, sh.nblocks);          \
-    launch_k(tf4::k_guided_fq<FMT, SEG, BF>, g, st, a, segv);                         \
+    const int64_t g = wave_grid(tf4::k_guided_fq<FMT, SEG, OUT>, sh.nblocks);         \
+    launch_k(tf4::k_guided_fq<FMT, SEG, OUT>, g, st, a, segv);                        \
   } while (0)
+  // fp32 output: one 32-byte store per 8 elements when out allows it
+  const int mode = out_bf16 ? tf4::kOutBf16 : (aligned(out, 32) ? tf4::kOutF32V8 : tf4::kOutF32);
   by_format(sh.fmt, [&](auto f) {
     constexpr int FMT = decltype(f)::value;
     if constexpr (tf4::kE4M3<FMT>) {
       if (multi(sh)) {
-        if (out_bf16) TF4_LAUNCH_FQ(FMT, tf4::SegN, true, make_segn(sh));
-        else TF4_LAUNCH_FQ(FMT, tf4::SegN, false, make_segn(sh));
+        if (mode == tf4::kOutBf16) TF4_LAUNCH_FQ(FMT, tf4::SegN, tf4::kOutBf16, make_segn(sh));
+        else if (mode == tf4::kOutF32V8) TF4_LAUNCH_FQ(FMT, tf4::SegN, tf4::kOutF32V8, make_segn(sh));
+        else TF4_LAUNCH_FQ(FMT, tf4::SegN, tf4::kOutF32, make_segn(sh));
         return;
       }
     }
-    if (out_bf16) TF4_LAUNCH_FQ(FMT, tf4::Seg1, true, tf4::Seg1{});
-    else TF4_LAUNCH_FQ(FMT, tf4::Seg1, false, tf4::Seg1{});
+    if (mode == tf4::kOutBf16) TF4_LAUNCH_FQ(FMT, tf4::Seg1, tf4::kOutBf16, tf4::Seg1{});
+    else if (mode == tf4::kOutF32V8) TF4_LAUNCH_FQ(FMT, tf4::Seg1, tf4::kOutF32V8, tf4::Seg1{});
+    else TF4_LAUNCH_FQ(FMT, tf4::Seg1, tf4::kOutF32, tf4::Seg1{});
   });
 #undef TF4_LAUNCH_FQ
   return launched();
@@ -570,17 +578,29 @@ tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint
   a.s_t = s_t;
   a.out = reinterpret_cast<float4*>(out);
   a.nblocks = sh.nblocks;
+  // 8 elements and one 32-byte store per lane when out allows it
+  const bool v8 = aligned(out, 32);
   by_format(sh.fmt, [&](auto f) {
     constexpr int FMT = decltype(f)::value;
     if constexpr (tf4::kE4M3<FMT>) {
       if (multi(sh)) {
-        const int64_t g = wave_grid(tf4::k_dequant<FMT, tf4::SegN>, sh.nblocks);
-        launch_k(tf4::k_dequant<FMT, tf4::SegN>, g, st, a, make_segn(sh));
+        if (v8) {
+          const int64_t g = wave_grid(tf4::k_dequant8<FMT, tf4::SegN>, sh.nblocks);
+          launch_k(tf4::k_dequant8<FMT, tf4::SegN>, g, st, a, make_segn(sh));
+        } else {
+          const int64_t g = wave_grid(tf4::k_dequant<FMT, tf4::SegN>, sh.nblocks);
+          launch_k(tf4::k_dequant<FMT, tf4::SegN>, g, st, a, make_segn(sh));
+        }
         return;
       }
     }
-    const int64_t g = wave_grid(tf4::k_dequant<FMT, tf4::Seg1>, sh.nblocks);
-    launch_k(tf4::k_dequant<FMT, tf4::Seg1>, g, st, a, tf4::Seg1{});
+    if (v8) {
+      const int64_t g = wave_grid(tf4::k_dequant8<FMT, tf4::Seg1>, sh.nblocks);
+      launch_k(tf4::k_dequant8<FMT, tf4::Seg1>, g, st, a, tf4::Seg1{});
+    } else {
+      const int64_t g = wave_grid(tf4::k_dequant<FMT, tf4::Seg1>, sh.nblocks);
+      launch_k(tf4::k_dequant<FMT, tf4::Seg1>, g, st, a, tf4::Seg1{});
+    }
   });
   return launched();
 }

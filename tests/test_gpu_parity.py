@@ -311,6 +311,25 @@ def test_guided_fake_quant_parity(fmt, seg, dtype):
         assert_same("values", host(y.view(torch.int16)).view(np.uint16), O.f32_to_bf16(vals))
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+def test_fp32_outputs_only_16_byte_aligned(fmt):
+    """Outputs 16-B but not 32-B aligned take the 16-byte-store kernels
+    (dequantize, fused fp32 fake-quant): same values."""
+    rows, cols = 37, 1024
+    xb = W.random_bf16((rows, cols), seed=47, device=DEV, outlier_frac=0.01)
+    q, r = check_quant(xb, fmt)
+    buf = torch.empty(rows * cols + 8, dtype=torch.float32, device=DEV)
+    view = buf[4:4 + rows * cols].view(rows, cols)
+    assert view.data_ptr() % 32 == 16
+    d = B.tf4_dequantize(q, out=view)
+    want = O.dequantize(r["codes"], r["scales"], rows, cols, fmt, s_t=r["s_t"])
+    assert_same("dequant", f32_bits(host(d)), f32_bits(want))
+    xt = W.perturb(xb, 48, rel=0.05)
+    y, _ = B.tf4_guided_fake_quant(xt, q, out=view)
+    _, vals, _ = O.guided_fake_quant(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"])
+    assert_same("fake-quant", f32_bits(host(y)), f32_bits(vals))
+
+
 @pytest.mark.parametrize("fmt,shape", [(O.NVFP4, (1, 16)), (O.NVFP4, (3, 48)), (O.UFP4, (5, 16 * 33)), (O.MXFP4, (3, 64)),
                                        (O.MXFP4, (1, 32))])
 def test_guided_fake_quant_small_shapes(fmt, shape):
