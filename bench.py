@@ -62,8 +62,10 @@ def parse():
                         "costs a few microseconds of idle GPU and stops the next launch from overlapping)")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--cpu-rows", type=int, default=256, help="rows per layer in the oracle sample")
-    p.add_argument("--ref-rows", type=int, default=48, help="rows per layer per reference step")
+    p.add_argument("--cpu-rows", type=int, default=256, help="rows per layer in the single-core oracle sample")
+    p.add_argument("--cpu-mc-factor", type=int, default=8,
+                   help="the all-core oracle sample is this many times the single-core one")
+    p.add_argument("--ref-rows", type=int, default=256, help="rows per layer per reference step")
     p.add_argument("--suite", action="store_true",
                    help="time every call of the path on every workload (a table, not the bench line)")
     p.add_argument("--only", action="append",
@@ -463,47 +465,67 @@ def sample_host(args, rows):
 
 
 def cpu_baseline(args, rows):
+    """The oracle on a row sample of the workload: on every host core (one
+    spawned process per layer task) and, for reference, on one core."""
     import oracle as O
+    from oracle.pool import OraclePool
 
     O.lib()
     xs, xts = sample_host(args, rows)
     t = time.perf_counter()
     oracle_sample_step(args, rows, xs, xts)
-    dt = time.perf_counter() - t
-    sample_args = argparse.Namespace(**{**vars(args), "rows": rows})
-    b, _ = step_bytes(sample_args)
-    return dict(value=round(b / dt / 1e9, 4), unit="GB/s", cores=1, kind="oracle",
-                sample=f"first {rows} of {args.rows} rows of each of the {args.layers} layers "
-                       f"(capture) and of the {args.deep} perturbed deep layers (guided); "
-                       f"{dt:.1f} s single-threaded C oracle")
+    dt1 = time.perf_counter() - t
+    b1, _ = step_bytes(argparse.Namespace(**{**vars(args), "rows": rows}))
+    rows_mc = rows * args.cpu_mc_factor
+    xs, xts = sample_host(args, rows_mc)
+    pool = OraclePool()
+    try:
+        t = time.perf_counter()
+        pool.run(xs, xts, args.layers - args.deep)
+        dtm = time.perf_counter() - t
+    finally:
+        pool.close()
+    bm, _ = step_bytes(argparse.Namespace(**{**vars(args), "rows": rows_mc}))
+    return dict(value=round(bm / dtm / 1e9, 4), unit="GB/s", cores=pool.workers, kind="oracle",
+                sample=f"first {rows_mc} of {args.rows} rows of each of the {args.layers} layers "
+                       f"(capture) and of the {args.deep} perturbed deep layers (guided), one process per "
+                       f"layer on {pool.workers} host cores, {dtm:.1f} s",
+                value_1core=round(b1 / dt1 / 1e9, 4),
+                sample_1core=f"first {rows} rows of each layer, single-threaded, {dt1:.1f} s")
 
 
 def run_reference(args, world, rank):
     if rank != 0:
         return None
     import oracle as O
+    from oracle.pool import OraclePool
 
     O.lib()
     rows = args.ref_rows
     xs, xts = sample_host(args, rows)
-    for _ in range(args.warmup):
-        oracle_sample_step(args, rows, xs, xts)
-    t = time.perf_counter()
-    for _ in range(args.steps):
-        oracle_sample_step(args, rows, xs, xts)
-    dt = (time.perf_counter() - t) / args.steps
+    pool = OraclePool()
+    try:
+        for _ in range(args.warmup):
+            pool.run(xs, xts, args.layers - args.deep)
+        t = time.perf_counter()
+        for _ in range(args.steps):
+            pool.run(xs, xts, args.layers - args.deep)
+        dt = (time.perf_counter() - t) / args.steps
+    finally:
+        pool.close()
     sample_args = argparse.Namespace(**{**vars(args), "rows": rows})
     b, _ = step_bytes(sample_args)
     v = round(b / dt / 1e9, 4)
     sample = (f"first {rows} of {args.rows} rows of each of the {args.layers} layers (capture) and of the "
-              f"{args.deep} perturbed deep layers (guided) per step")
+              f"{args.deep} perturbed deep layers (guided) per step, one process per layer on {pool.workers} "
+              f"host cores")
     return dict(impl="reference", metric=METRIC, value=v, unit="GB/s", n_gpus=world, steps=args.steps,
                 warmup=args.warmup, ms_per_step=round(dt * 1e3, 2), higher_is_better=True, scaling="weak",
                 vs_baseline=None, dtype="f64", data="synthetic",
                 config=dict(workload=f"layer_stack: {args.layers} layers x {args.rows}x{args.cols} bf16, "
                                      f"NVFP4 capture + guided (row sample)", layers=args.layers,
                             rows=args.rows, cols=args.cols, format="NVFP4"),
-                cpu_baseline=dict(value=v, unit="GB/s", cores=1, kind="oracle", sample=sample),
+                cpu_baseline=dict(value=v, unit="GB/s", cores=pool.workers, kind="oracle", sample=sample),
                 e2e=dict(value=v, unit="GB/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
 
 
