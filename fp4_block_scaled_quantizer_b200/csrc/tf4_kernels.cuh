@@ -197,9 +197,26 @@ __device__ __forceinline__ float4 decode4_uni(uint32_t c, float S) {
   return make_float4(v[0], v[1], v[2], v[3]);
 }
 
+// The same through CUDA's E4M3 -> half conversion: magnitude k (0..7) as an
+// E4M3 byte is the subnormal k * 2^-9 (exact in f16), the nibble's sign
+// goes to the byte's sign bit, and (k 2^-9) (S 2^9) = k S is rounded once.
+// Needs S 2^9 finite: the caller checks S <= 2^100.
+__device__ __forceinline__ float4 decode4_uni_e4m3(uint32_t c, float S) {
+  uint32_t t = c & 0xFFFFu;
+  t = (t | (t << 8)) & 0x00FF00FFu;   // n0|n1<<4 in byte 0, n2|n3<<4 in byte 2
+  t = (t | (t << 4)) & 0x0F0F0F0Fu;   // n0..n3 in bytes 0..3
+  t = (t & 0x07070707u) | ((t & 0x08080808u) << 4);
+  const float S9 = S * 512.0f;        // exact
+  const __half2_raw h0 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(t & 0xFFFFu), __NV_E4M3);
+  const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(t >> 16), __NV_E4M3);
+  const float2 f0 = __half22float2(__half2(h0));
+  const float2 f1 = __half22float2(__half2(h1));
+  return make_float4(__fmul_rn(f0.x, S9), __fmul_rn(f0.y, S9), __fmul_rn(f1.x, S9), __fmul_rn(f1.y, S9));
+}
+
 template <bool U>
 __device__ __forceinline__ float4 decode4_grid(uint32_t c, float S) {
-  if constexpr (U) return decode4_uni(c, S);
+  if constexpr (U) return S <= 0x1p100f ? decode4_uni_e4m3(c, S) : decode4_uni(c, S);
   else return decode4(c, S);
 }
 
@@ -1017,7 +1034,8 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
         bool bad = false;
         if (k < n) {
           const int64_t blk = lo + k;
-          bad = block_absmax_bits(w[u]) >= 0x7F80u;
+          const uint32_t mb = block_absmax_bits(w[u]);
+          bad = mb >= 0x7F80u;
           uint32_t c[NQ];
           float r = 0.0f;
           if constexpr (kE4M3<FMT>) {
@@ -1129,7 +1147,8 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
         bool bad = false;
         if (o < o1) {
           const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
-          bad = block_absmax_bits(w) >= 0x7F80u;
+          const uint32_t mb = block_absmax_bits(w);
+          bad = mb >= 0x7F80u;
           float r = 0.0f, S;
           bool rz = false;
           if constexpr (kE4M3<FMT>) {
@@ -1144,7 +1163,8 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
           }
           uint32_t c;
           if (r != 0.0f) {
-            c = rz ? cvt_words<true, UG>(w[0], w[1], w[2], w[3], r) : cvt_words<false, UG>(w[0], w[1], w[2], w[3], r);
+            c = rz ? cvt_words<true, UG>(w[0], w[1], w[2], w[3], r)
+                   : cvt_words<false, UG>(w[0], w[1], w[2], w[3], r);
             const uint32_t mm = (c ^ spread_bits(g[u])) & 0x11111111u;
             if (mm)
               c = rz ? fix_mismatches<true, UG>(c, mm, w[0], w[1], w[2], w[3], r)
@@ -1187,7 +1207,6 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
 // grid index (sign ? -m3 : m3, so +0 and -0 are equal).  Accumulates
 // counts[0] += #(n_r != n_o), counts[1] += #(|n_r - n_o| == 1),
 // counts[2] += #(|n_r - n_o| >= 2), counts[3] += #(n_g != n_o).
-// Exact per-element comparisons (a diagnostic; not on the hot path).
 struct MismatchArgs {
   const uint4* x;
   int64_t nblocks;
@@ -1203,12 +1222,40 @@ __device__ __forceinline__ int grid_index(uint32_t nib) {
   return (nib & 8u) ? -m : m;
 }
 
+// Counts over the nibbles where code word cx differs from the rollout's co:
+// with d = |index(cx) - index(co)|, cnt[0..2] += (d != 0, d == 1, d >= 2)
+// (NEAREST) or cnt[3] += (d != 0) (guided).  Equal nibbles count nothing.
+template <bool NEAREST>
+__device__ __forceinline__ void count_diffs(uint32_t cx, uint32_t co, uint32_t (&cnt)[4]) {
+  uint32_t d = cx ^ co;
+  while (d) {
+    const int e = (__ffs(d) - 1) >> 2;
+    d &= ~(0xFu << (4 * e));
+    const int dd = abs(grid_index((cx >> (4 * e)) & 0xFu) - grid_index((co >> (4 * e)) & 0xFu));
+    if (NEAREST) {
+      cnt[0] += dd != 0;
+      cnt[1] += dd == 1;
+      cnt[2] += dd >= 2;
+    } else {
+      cnt[3] += dd != 0;
+    }
+  }
+}
+
+// Per block, nearest and guided rounding of the train values on the
+// recorded grid take the quantize / guided fast paths (per-segment tables
+// verified against the grid's midpoints and codewords respectively; MXFP4's
+// quotient is exact), falling back to exact per-element comparisons where
+// no verified multiplier exists; the code words are then compared with the
+// rollout's nibble-wise, and only differing nibbles are classified.
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int NW = BE / 2;
+  constexpr int NQ = BE / 8;
+  __shared__ SegTables tmid, tcw;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   uint32_t cnt[4] = {0u, 0u, 0u, 0u};
@@ -1218,8 +1265,12 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
     const int s = seg.find(lo);
     const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
     const float st = kE4M3<FMT> ? a.rec_s_t[s] : 0.0f;
+    if constexpr (kE4M3<FMT>) {
+      build_tables<UG, true, false>(st, tmid);
+      build_tables<UG, false>(st, tcw);
+    }
     for (int64_t blk = lo + threadIdx.x; blk < hi; blk += kThreads) {
-      uint32_t w[NW], cw[BE / 8];
+      uint32_t w[NW], cw[NQ];
 #pragma unroll
       for (int q = 0; q < NW / 4; ++q) {
         const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
@@ -1233,23 +1284,60 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
         cw[0] = c.x; cw[1] = c.y; cw[2] = c.z; cw[3] = c.w;
       }
       const uint32_t sc = a.rec_scales[blk];
-      float S;
-      if constexpr (kE4M3<FMT>) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
-      else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
-      bad |= block_absmax_bits(w) >= 0x7F80u;
+      float S, rm = 0.0f, rc = 0.0f;
+      bool rzm = false, rzc = false;
+      if constexpr (kE4M3<FMT>) {
+        S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
+        if ((sc >> 3) >= 1u && sc < 0x7Fu) {
+          if (tmid.fast && tmid.rho[sc & 7u] != 0.0f) {
+            rm = block_rho(tmid.rho[sc & 7u], sc >> 3);
+            rzm = tmid.rz;
+          }
+          if (tcw.fast && tcw.rho[sc & 7u] != 0.0f) {
+            rc = block_rho(tcw.rho[sc & 7u], sc >> 3);
+            rzc = tcw.rz;
+          }
+        }
+      } else {
+        S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
+        if (sc >= 1u && sc <= 252u) rm = rc = __uint_as_float((254u - sc) << 23);  // 2^-(sc-127), exact
+      }
+      const uint32_t mb = block_absmax_bits(w);
+      bad |= mb >= 0x7F80u;
 #pragma unroll
-      for (int e = 0; e < BE; ++e) {
-        const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-        const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-        const uint32_t no = (cw[e >> 3] >> (4 * (e & 7))) & 0xFu;
-        const uint32_t sg = (h >> 15) << 3;
-        const uint32_t nr = sg | (S > 0.0f ? rtn_m3_exact<UG>(ax, S) : 0u);
-        const uint32_t ng = sg | (S > 0.0f ? guided_m3_exact<UG>(ax, S, no & 1u) : 0u);
-        const int d = abs(grid_index(nr) - grid_index(no));
-        cnt[0] += d != 0;
-        cnt[1] += d == 1;
-        cnt[2] += d >= 2;
-        cnt[3] += grid_index(ng) != grid_index(no);
+      for (int q = 0; q < NQ; ++q) {
+        const uint32_t* wq = &w[4 * q];
+        const uint32_t co = cw[q];
+        uint32_t cr = 0u, cg = 0u;
+        if (rm != 0.0f) {
+          cr = rzm ? cvt_words<true, UG>(wq[0], wq[1], wq[2], wq[3], rm)
+                   : cvt_words<false, UG>(wq[0], wq[1], wq[2], wq[3], rm);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t h = (e & 1) ? (wq[e >> 1] >> 16) : (wq[e >> 1] & 0xFFFFu);
+            const uint32_t m3 = S > 0.0f ? rtn_m3_exact<UG>(__uint_as_float((h & 0x7FFFu) << 16), S) : 0u;
+            cr |= (((h >> 15) << 3) | m3) << (4 * e);
+          }
+        }
+        if (rc != 0.0f) {
+          cg = rzc ? cvt_words<true, UG>(wq[0], wq[1], wq[2], wq[3], rc)
+                   : cvt_words<false, UG>(wq[0], wq[1], wq[2], wq[3], rc);
+          const uint32_t mm = (cg ^ co) & 0x11111111u;  // mantissa bit vs the rollout's
+          if (mm)
+            cg = rzc ? fix_mismatches<true, UG>(cg, mm, wq[0], wq[1], wq[2], wq[3], rc)
+                     : fix_mismatches<false, UG>(cg, mm, wq[0], wq[1], wq[2], wq[3], rc);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t h = (e & 1) ? (wq[e >> 1] >> 16) : (wq[e >> 1] & 0xFFFFu);
+            const uint32_t g = (co >> (4 * e)) & 1u;
+            const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(__uint_as_float((h & 0x7FFFu) << 16), S, g) : 0u;
+            cg |= (((h >> 15) << 3) | m3) << (4 * e);
+          }
+        }
+        count_diffs<true>(cr, co, cnt);
+        count_diffs<false>(cg, co, cnt);
       }
     }
     lo = hi;

@@ -363,6 +363,18 @@ def test_mismatch_stats_parity(fmt, seg, rel):
         assert want[0] == want[1] + want[2]
 
 
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
+def test_mismatch_stats_near_ties(fmt):
+    """Train values on and around the recorded grid's midpoints and codewords:
+    the fast nearest / guided paths of the diagnostics agree with the oracle."""
+    xb = _near_tie_tensor(np.random.default_rng(15), 1.0, fmt=fmt).to(DEV)
+    q, r = check_quant(xb, fmt)
+    xt = _near_tie_tensor(np.random.default_rng(16), 1.0, fmt=fmt).to(DEV)
+    c = B.tf4_mismatch_stats(xt, q)
+    want = O.mismatch_stats(W.bf16_bits(xt), r["scales"], r["codes"], fmt, rec_s_t=r["s_t"])
+    assert host(c).tolist() == want.tolist()
+
+
 @pytest.mark.parametrize("fmt,L,keep", [(O.NVFP4, 5, 2), (O.NVFP4, 3, 3), (O.NVFP4, 1, 0), (O.MXFP4, 4, 1),
                                         (O.UFP4, 4, 2)])
 def test_capture_batched_parity(fmt, L, keep):
@@ -558,6 +570,37 @@ def test_sr_counter_beyond_2_32():
         want = _oracle_row_with_offset(W.bf16_bits(x[r:r + 1])[0], r * cols, 2**33 + 5)
         assert_same(f"row {r}", host(q.codes[r * cols // 2:(r + 1) * cols // 2]), want)
     del x, q
+    torch.cuda.empty_cache()
+
+
+def test_nvfp4_capture_beyond_2_32_elements():
+    """NVFP4 capture + guided on a (2^32 + 2^20)-element tensor: 64-bit
+    block indices through amax, quantize, guided and pack; the tensor scale
+    against the oracle's full amax pass, sampled rows (across the 2^32
+    boundary) against the oracle given that scale."""
+    cols = 4096
+    rows = (2**32 + 2**20) // cols
+    g = torch.Generator(device=DEV).manual_seed(9)
+    x = torch.randn((rows, cols), generator=g, device=DEV, dtype=torch.bfloat16)
+    q = B.tf4_quantize_capture(x)
+    gq = B.tf4_quantize_guided(x, q)
+    assert B.read_status(x.device) == 0
+    assert torch.equal(gq, q.codes)
+    del gq
+    bits = B.tf4_pack_guidance(q.codes, rows, cols)
+    assert torch.equal(bits, q.bits)
+    del bits
+    xs = W.bf16_bits(x)
+    st, status = O.segment_scales(xs)
+    assert status == 0
+    assert_same("s_t", f32_bits(host(q.s_t)), f32_bits(st))
+    r0 = 2**32 // cols
+    for r in (0, r0 - 1, r0, r0 + 1, rows - 1):
+        want = O.quantize(xs[r:r + 1], O.NVFP4, s_t=st, bits=True)
+        assert_same(f"codes row {r}", host(q.codes[r * cols // 2:(r + 1) * cols // 2]), want["codes"])
+        assert_same(f"scales row {r}", host(q.scales[r]), want["scales"])
+        assert_same(f"bits row {r}", host(q.bits[r * cols // 8:(r + 1) * cols // 8]), want["bits"])
+    del x, q, xs
     torch.cuda.empty_cache()
 
 
