@@ -581,14 +581,58 @@ def run_suite(args):
         return any(workload.startswith(w) and (not fmt or not f or fmt == f) and (not call or not c or call == c)
                    for w, f, c, *_ in only)
 
-    def run(workload, fmt, call, n, fn, **extra):
-        if sel(workload, fmt, call):
-            record(workload, fmt, call, n, timed(fn), **extra)
+    flush_buf = []
 
-    def record(workload, fmt, call, n, us, **extra):
+    def timed_cold(fn, reps=10):
+        """Mean time of fn with L2 flushed before each rep (a 512 MiB memset,
+        outside the events)."""
+        if not flush_buf:
+            flush_buf.append(torch.empty(512 << 20, dtype=torch.uint8, device=dev))
+        for _ in range(3):
+            fn()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            flush_buf[0].zero_()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in ev) / reps * 1e3
+
+    def timed_graph(fn, reps=10):
+        """Mean time of fn over reps calls captured in one CUDA graph and
+        replayed (back to back on the GPU, no host launch pacing)."""
+        for _ in range(3):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            for _ in range(reps):
+                fn()
+        g.replay()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        g.replay()
+        b.record()
+        torch.cuda.synchronize()
+        del g
+        return a.elapsed_time(b) / reps * 1e3
+
+    def run(workload, fmt, call, n, fn, cold=False, **extra):
+        if sel(workload, fmt, call):
+            record(workload, fmt, call, n, timed(fn), l2="warm" if cold else None, **extra)
+            if cold:
+                record(workload, fmt, call, n, timed_graph(fn), l2="warm, CUDA graph", **extra)
+                record(workload, fmt, call, n, timed_cold(fn), l2="cold", **extra)
+
+    def record(workload, fmt, call, n, us, l2=None, **extra):
         gbs = CALL_BYTES[(fmt, call)] * n / (us * 1e-6) / 1e9
+        if l2:
+            extra["l2"] = l2
         rows_out.append(dict(workload=workload, format=fmt, call=call, elements=n, us=round(us, 2),
-                             gbs=round(gbs, 1), frac=round(gbs / peak, 4), **extra))
+                             gbs=round(gbs, 1), frac=round(gbs / peak, 4),
+                             elements_per_s=round(n / (us * 1e-6), 1), **extra))
 
     def fq_and_diag(name, fmt, q, x, xt):
         n = x.numel()
@@ -604,7 +648,7 @@ def run_suite(args):
         record(name, fmt, "mismatch", n, us, counts=dict(mismatch=c[0], adjacent=c[1], far=c[2], after_guidance=c[3]),
                adjacent_fraction=(round(c[1] / c[0], 6) if c[0] else None))
 
-    def nv_calls(name, x, xt, seg=None):
+    def nv_calls(name, x, xt, seg=None, cold=False):
         n = x.numel()
         q = B.tf4_quantize_capture(x, seg_off=seg)
         amax = B.tf4_segment_amax(x, seg)
@@ -613,30 +657,30 @@ def run_suite(args):
         bits = torch.empty(n // 8, dtype=torch.uint8, device=dev)
         mant = torch.empty(n, dtype=torch.uint8, device=dev)
         qr = B.tf4_quantize_rtn(x, seg_off=seg)
-        run(name, "nvfp4", "amax", n, lambda: B.tf4_segment_amax(x, seg, out=amax))
-        run(name, "nvfp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, seg_off=seg, out=qr))
-        run(name, "nvfp4", "capture", n, lambda: B.tf4_quantize_capture(x, seg_off=seg, out=q))
-        run(name, "nvfp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g))
-        run(name, "nvfp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, seg_off=seg, out=qr))
-        run(name, "nvfp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out))
+        run(name, "nvfp4", "amax", n, lambda: B.tf4_segment_amax(x, seg, out=amax), cold=cold)
+        run(name, "nvfp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, seg_off=seg, out=qr), cold=cold)
+        run(name, "nvfp4", "capture", n, lambda: B.tf4_quantize_capture(x, seg_off=seg, out=q), cold=cold)
+        run(name, "nvfp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g), cold=cold)
+        run(name, "nvfp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, seg_off=seg, out=qr), cold=cold)
+        run(name, "nvfp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out), cold=cold)
         rows, cols = x.shape
-        run(name, "any", "pack", n, lambda: B.tf4_pack_guidance(q.codes, rows, cols, out=bits))
-        run(name, "any", "unpack", n, lambda: B.tf4_unpack_guidance(bits, rows, cols, out=mant))
+        run(name, "any", "pack", n, lambda: B.tf4_pack_guidance(q.codes, rows, cols, out=bits), cold=cold)
+        run(name, "any", "unpack", n, lambda: B.tf4_unpack_guidance(bits, rows, cols, out=mant), cold=cold)
         fq_and_diag(name, "nvfp4", q, x, xt)
         del q, g, out, bits, mant, qr
 
-    def uf_calls(name, x, xt, seg=None):
+    def uf_calls(name, x, xt, seg=None, cold=False):
         n = x.numel()
         U = B.UFP4
         q = B.tf4_quantize_capture(x, fmt=U, seg_off=seg)
         g = torch.empty_like(q.codes)
         out = torch.empty(x.shape, dtype=torch.float32, device=dev)
         qr = B.tf4_quantize_rtn(x, fmt=U, seg_off=seg)
-        run(name, "ufp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, fmt=U, seg_off=seg, out=qr))
-        run(name, "ufp4", "capture", n, lambda: B.tf4_quantize_capture(x, fmt=U, seg_off=seg, out=q))
-        run(name, "ufp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g))
-        run(name, "ufp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, fmt=U, seg_off=seg, out=qr))
-        run(name, "ufp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out))
+        run(name, "ufp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, fmt=U, seg_off=seg, out=qr), cold=cold)
+        run(name, "ufp4", "capture", n, lambda: B.tf4_quantize_capture(x, fmt=U, seg_off=seg, out=q), cold=cold)
+        run(name, "ufp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g), cold=cold)
+        run(name, "ufp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, fmt=U, seg_off=seg, out=qr), cold=cold)
+        run(name, "ufp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out), cold=cold)
         fq_and_diag(name, "ufp4", q, x, xt)
         del q, g, out, qr
 
@@ -656,7 +700,7 @@ def run_suite(args):
             lambda: B.tf4_quantize_capture_batched(xs, fmt=fmt, keep=keep, out=ob), launch="batched")
         del ob, per
 
-    def mx_calls(name, x, xt):
+    def mx_calls(name, x, xt, cold=False):
         if x.shape[1] % 32:
             return
         n = x.numel()
@@ -664,20 +708,20 @@ def run_suite(args):
         g = torch.empty_like(q.codes)
         out = torch.empty(x.shape, dtype=torch.float32, device=dev)
         qr = B.tf4_quantize_rtn(x, fmt=B.MXFP4)
-        run(name, "mxfp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, fmt=B.MXFP4, out=qr))
-        run(name, "mxfp4", "capture", n, lambda: B.tf4_quantize_capture(x, fmt=B.MXFP4, out=q))
-        run(name, "mxfp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g))
-        run(name, "mxfp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, fmt=B.MXFP4, out=qr))
-        run(name, "mxfp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out))
+        run(name, "mxfp4", "rtn", n, lambda: B.tf4_quantize_rtn(x, fmt=B.MXFP4, out=qr), cold=cold)
+        run(name, "mxfp4", "capture", n, lambda: B.tf4_quantize_capture(x, fmt=B.MXFP4, out=q), cold=cold)
+        run(name, "mxfp4", "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g), cold=cold)
+        run(name, "mxfp4", "sr", n, lambda: B.tf4_quantize_sr(x, 4, fmt=B.MXFP4, out=qr), cold=cold)
+        run(name, "mxfp4", "dequant", n, lambda: B.tf4_dequantize(q, out=out), cold=cold)
         fq_and_diag(name, "mxfp4", q, x, xt)
         del q, g, out, qr
 
     name = "activation_outliers 4096x2048"
     if sel(name):
         w = W.activation_outliers(dev)
-        nv_calls(name, w["x"], w["x_train"])
-        mx_calls(name, w["x"], w["x_train"])
-        uf_calls(name, w["x"], w["x_train"])
+        nv_calls(name, w["x"], w["x_train"], cold=True)
+        mx_calls(name, w["x"], w["x_train"], cold=True)
+        uf_calls(name, w["x"], w["x_train"], cold=True)
         del w
     name = "40 layers of 4096x2048"
     if sel(name):

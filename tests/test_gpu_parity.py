@@ -455,6 +455,39 @@ def test_empty_tensor():
     assert q.s_t.shape == (2,) and not q.s_t.any()
 
 
+def test_cuda_graph_capture_and_replay():
+    """The calls launch only kernels on the given stream (no allocation, no
+    host synchronisation), so a rollout capture + train-side fake-quant step
+    can be captured in a CUDA graph and replayed on new data in the same
+    buffers, with the results of direct calls."""
+    rows, cols = 96, 2048
+    x = W.random_bf16((rows, cols), seed=81, device=DEV, outlier_frac=0.01)
+    xt = W.perturb(x, 82, rel=0.01)
+    y = torch.empty((rows, cols), dtype=torch.bfloat16, device=DEV)
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):  # warm-up on the capture stream: its workspace exists before capture
+        q = B.tf4_quantize_capture(x)
+        B.tf4_guided_fake_quant(xt, q, out=y)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        B.tf4_quantize_capture(x, out=q)
+        B.tf4_guided_fake_quant(xt, q, out=y)
+    for seed in (83, 84):
+        x.copy_(W.random_bf16((rows, cols), seed=seed, device=DEV, outlier_frac=0.02))
+        xt.copy_(W.perturb(x, seed + 10, rel=0.01))
+        g.replay()
+        torch.cuda.synchronize()
+        q2 = B.tf4_quantize_capture(x)
+        y2, _ = B.tf4_guided_fake_quant(xt, q2, out_dtype=torch.bfloat16)
+        for name in ("codes", "scales", "s_t", "bits"):
+            assert torch.equal(getattr(q, name), getattr(q2, name)), name
+        assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
+    assert B.read_status(x.device) == 0
+    del g
+
+
 def test_ste_identity_backward():
     from fp4_block_scaled_quantizer_b200 import ste
     xb = W.random_bf16((16, 256), seed=41, device=DEV).requires_grad_(True)
