@@ -149,3 +149,16 @@ def test_batched_capture_rejects_bad_arguments(L):
     assert call(d, 2, ptrs, 0, None, wsb=4) == 4                # workspace too small
     assert call(d, 2, ptrs, 0, None, s_t=None) == 1
     assert L.tf4_workspace_bytes_batched(3) == 256 and L.tf4_workspace_bytes_batched(0) == 0
+
+
+def test_uniform_grid_format_arguments(L):
+    """UFP4 uses NVFP4's container: 16-element blocks, segments and a
+    workspace; unknown format numbers are refused."""
+    assert _rtn(L, B.Desc(B.UFP4, 4, 24)) == 2                       # cols % 16
+    assert L.tf4_workspace_bytes(B.Desc(B.UFP4, 4, 32).ptr) >= 8
+    assert L.tf4_workspace_bytes(B.Desc(B.UFP4, 10, 32, [0, 5, 10]).ptr) >= 12
+    assert _rtn(L, B.Desc(B.UFP4, 10, 16, [0, 5, 4, 10])) == 1       # decreasing offsets
+    assert _rtn(L, B.Desc(B.UFP4, 4, 32), s_t=None) == 1             # tensor scale required
+    assert _rtn(L, B.Desc(3, 4, 32)) == 1
+    s = B.sizes(B.UFP4, 64, 128)
+    assert s["scales"] == 64 * 128 // 16 and s["record_full"] == 64 * 128 // 2 + 64 * 128 // 16 + 4
