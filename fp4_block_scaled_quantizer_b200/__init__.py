@@ -9,5 +9,5 @@ from .binding import (  # noqa: F401
     MXFP4, NVFP4, UFP4, Desc, Quantized, Tf4Error, capture_layers, lib, read_status, sizes,
     tf4_dequantize, tf4_guided_fake_quant, tf4_mismatch_stats, tf4_pack_guidance, tf4_quantize_capture,
     tf4_quantize_capture_batched, tf4_quantize_guided, tf4_quantize_rtn, tf4_quantize_sr, tf4_segment_amax,
-    tf4_unpack_guidance,
+    tf4_swizzle_scales, tf4_unpack_guidance,
 )

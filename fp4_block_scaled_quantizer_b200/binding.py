@@ -43,7 +43,7 @@ EXPORTS = (
     "tf4_record_bytes", "tf4_segment_amax", "tf4_quantize_rtn", "tf4_quantize_sr",
     "tf4_quantize_capture", "tf4_quantize_guided", "tf4_dequantize", "tf4_pack_guidance",
     "tf4_unpack_guidance", "tf4_guided_fake_quant", "tf4_mismatch_stats", "tf4_workspace_bytes_batched",
-    "tf4_quantize_capture_batched", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
+    "tf4_quantize_capture_batched", "tf4_blocked_scales_bytes", "tf4_swizzle_scales", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
     "tf4_version",
 )
 
@@ -99,6 +99,8 @@ def lib():
                     "tf4_guided_fake_quant": (st, [dp, vp, vp, vp, vp, vp, vp, ctypes.c_int, i32p, vp]),
                     "tf4_mismatch_stats": (st, [dp, vp, vp, vp, vp, vp, i32p, vp]),
                     "tf4_workspace_bytes_batched": (sz, [ctypes.c_int32]),
+                    "tf4_blocked_scales_bytes": (sz, [dp]),
+                    "tf4_swizzle_scales": (st, [dp, vp, vp, vp]),
                     "tf4_quantize_capture_batched": (st, [dp, ctypes.c_int32, vp, vp, vp, vp, ctypes.c_int32, vp,
                                                           vp, sz, i32p, vp]),
                     "tf4_read_status": (st, [i32p, vp]),
@@ -375,6 +377,19 @@ def tf4_dequantize(q: Quantized, codes=None, stream=None, out=None) -> torch.Ten
     o = out if out is not None else torch.empty((q.rows, q.cols), dtype=torch.float32, device=c.device)
     _check(lib().tf4_dequantize(d.ptr, _ptr(c), _ptr(q.scales), _ptr(q.s_t), _ptr(o), _stream(stream, c.device)),
            "tf4_dequantize")
+    return o
+
+
+def tf4_swizzle_scales(q: Quantized, stream=None, out=None) -> torch.Tensor:
+    """The record's block scales in the tiled layout block-scaled FP4 GEMMs
+    read (uint8 [ceil(rows/128)*128, ceil(nb/4)*4] as laid out in memory)."""
+    d = Desc(q.fmt, q.rows, q.cols, q.seg_off)
+    nb = q.cols // BLOCK[q.fmt]
+    shape = ((q.rows + 127) // 128 * 128, (nb + 3) // 4 * 4)
+    assert lib().tf4_blocked_scales_bytes(d.ptr) == shape[0] * shape[1]
+    o = out if out is not None else torch.empty(shape, dtype=torch.uint8, device=q.scales.device)
+    _check(lib().tf4_swizzle_scales(d.ptr, _ptr(q.scales), _ptr(o), _stream(stream, q.scales.device)),
+           "tf4_swizzle_scales")
     return o
 
 

@@ -1518,4 +1518,32 @@ __global__ void __launch_bounds__(kThreads) k_unpack(const uint8_t* __restrict__
   }
 }
 
+// ------------------------------------------------- tiled scale layout
+// Block scales rearranged for block-scaled FP4 GEMMs (the cuBLAS
+// documentation's "1D Block Scaling Factors Layout"): the [rows, nb] scale
+// matrix, zero-padded to 128-row x 4-column tiles, tiles in row-major
+// order, 512 bytes each, entry (r, c) of a tile at byte (r % 32) * 16 +
+// (r / 32) * 4 + c.  One lane writes one 16-byte line of a tile: row
+// i = r % 32 of its four 32-row groups, 4 columns each.
+__global__ void __launch_bounds__(kThreads) k_swizzle(const uint8_t* __restrict__ scales, int64_t rows, int64_t nb,
+                                                      int64_t ntc, int64_t nlines, uint4* out) {
+  pdl_enter();
+  for (int64_t l = (int64_t)blockIdx.x * kThreads + threadIdx.x; l < nlines; l += (int64_t)gridDim.x * kThreads) {
+    const int64_t tile = l >> 5;
+    const int64_t i = l & 31;
+    const int64_t r0 = (tile / ntc) * 128 + i, c0 = (tile % ntc) * 4;
+    uint32_t word[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t r = r0 + 32 * j;
+      uint32_t v = 0u;
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        if (r < rows && c0 + c < nb) v |= (uint32_t)__ldg(scales + r * nb + c0 + c) << (8 * c);
+      word[j] = v;
+    }
+    out[l] = make_uint4(word[0], word[1], word[2], word[3]);
+  }
+}
+
 }  // namespace tf4

@@ -632,6 +632,30 @@ tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_
   return launched();
 }
 
+size_t tf4_blocked_scales_bytes(const tf4_desc* desc) {
+  Shape sh;
+  if (check_desc(desc, &sh) != TF4_OK) return 0;
+  const int64_t nb = sh.cols / sh.be;
+  return (size_t)((sh.rows + 127) / 128 * 128) * (size_t)((nb + 3) / 4 * 4);
+}
+
+tf4_status tf4_swizzle_scales(const tf4_desc* desc, const uint8_t* scales, uint8_t* blocked, tf4_stream_t stream) {
+  Shape sh;
+  tf4_status e = check_desc(desc, &sh);
+  if (e != TF4_OK) return e;
+  if (sh.n == 0) return TF4_OK;
+  if (!scales || !blocked) return TF4_ERR_INVALID_ARG;
+  if (!aligned(blocked, 16)) return TF4_ERR_ALIGN;
+  const int64_t nb = sh.cols / sh.be;
+  const int64_t ntc = (nb + 3) / 4;
+  const int64_t nlines = (sh.rows + 127) / 128 * ntc * 32;  // 16-byte lines, 32 per tile
+  const int64_t wave = (int64_t)sm_count() * occupancy(reinterpret_cast<const void*>(tf4::k_swizzle));
+  const int64_t need = (nlines + kThreads - 1) / kThreads;
+  launch_k(tf4::k_swizzle, need < wave ? need : wave, reinterpret_cast<cudaStream_t>(stream), scales, sh.rows, nb,
+           ntc, nlines, reinterpret_cast<uint4*>(blocked));
+  return launched();
+}
+
 tf4_status tf4_quantize_capture_noalloc(const tf4_desc* desc, const void* x, uint8_t* codes, uint8_t* scales,
                                         float* s_t, uint8_t* bits, int32_t* status, tf4_stream_t stream) {
   Shape sh;

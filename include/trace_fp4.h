@@ -189,6 +189,21 @@ tf4_status tf4_quantize_capture_batched(const tf4_desc* desc, int32_t num_layers
                                         void* workspace, size_t workspace_bytes,
                                         int32_t* dev_status, tf4_stream_t stream);
 
+/* Block scales in the tiled layout block-scaled FP4 GEMMs take for their
+ * scale operands (NVIDIA cuBLAS documentation, "1D Block Scaling Factors
+ * Layout"; the same bytes a tcgen05 block-scaled MMA's scale tensor holds):
+ * the [rows, cols/block] scale matrix, zero-padded to a multiple of 128 rows
+ * and 4 columns, as 128 x 4 tiles in row-major tile order, 512 bytes each,
+ * entry (r, c) of a tile at byte (r % 32) * 16 + (r / 32) * 4 + c.  NVFP4 /
+ * UFP4 scale bytes are the E4M3 block scales (the per-segment s_t stays a
+ * separate factor), MXFP4 ones the E8M0 exponents.  The TRACE pages do not
+ * define this layout; it lets a captured record feed an FP4 GEMM directly.
+ *   scales   device [rows, cols/block] (any alignment)
+ *   blocked  device, tf4_blocked_scales_bytes(desc) bytes, 16-byte aligned */
+size_t tf4_blocked_scales_bytes(const tf4_desc* desc);
+tf4_status tf4_swizzle_scales(const tf4_desc* desc, const uint8_t* scales, uint8_t* blocked,
+                              tf4_stream_t stream);
+
 /* Train-side guided quantization of x (the trainer's value) with the
  * rollout's recorded scale bytes, recorded s_t (NVFP4; NULL for MXFP4) and
  * recorded guidance bits.  One pass over x, no workspace. */

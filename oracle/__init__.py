@@ -68,6 +68,7 @@ def lib():
             "orc_unpack_guidance": (None, [u8p, i64, u8p]),
             "orc_rtn_with_scales_rows": (None, [ctypes.c_int, u16p, i64, i64, i32, i64p, u8p, f32p, i64, i64,
                                                 u8p]),
+            "orc_swizzle_scales": (None, [u8p, i64, i64, u8p]),
             "orc_f32_to_bf16": (ctypes.c_uint16, [ctypes.c_float]),
             "orc_f32_to_bf16_array": (None, [f32p, i64, u16p]),
         }
@@ -256,6 +257,16 @@ def unpack_codes(codes, n):
     out[0::2] = c & 0xF
     out[1::2] = c >> 4
     return out[:n]
+
+
+def swizzle_scales(scales2d):
+    """The [rows, nb] scale bytes in the 128 x 4 tiled layout of block-scaled
+    GEMMs (flat uint8 array, zero-padded)."""
+    sc = np.ascontiguousarray(scales2d, dtype=np.uint8)
+    rows, nb = sc.shape
+    out = np.zeros(((rows + 127) // 128 * 128) * ((nb + 3) // 4 * 4), dtype=np.uint8)
+    lib().orc_swizzle_scales(_p(sc, ctypes.c_uint8), rows, nb, _p(out, ctypes.c_uint8))
+    return out
 
 
 def f32_to_bf16(v):

@@ -459,3 +459,21 @@ void orc_rtn_with_scales_rows(int fmt, const uint16_t* x, int64_t rows, int64_t 
     }
   }
 }
+
+/* Block scales in the tiled layout block-scaled FP4 GEMMs read (NVIDIA cuBLAS
+ * documentation, "1D Block Scaling Factors Layout"): the [rows, nb] scale
+ * matrix, zero-padded to a multiple of 128 rows and 4 columns, is cut into
+ * 128 x 4 tiles stored one after another in row-major tile order, 512 bytes
+ * each; inside a tile, entry (r, c) sits at byte (r % 32) * 16 + (r / 32) * 4
+ * + c. */
+void orc_swizzle_scales(const uint8_t* scales, int64_t rows, int64_t nb, uint8_t* out) {
+  const int64_t prow = (rows + 127) / 128 * 128, pcol = (nb + 3) / 4 * 4;
+  const int64_t ntc = pcol / 4;
+  for (int64_t r = 0; r < prow; ++r)
+    for (int64_t c = 0; c < pcol; ++c) {
+      const int64_t tile = (r / 128) * ntc + c / 4;
+      const int64_t rr = r % 128, cc = c % 4;
+      const int64_t off = tile * 512 + (rr % 32) * 16 + (rr / 32) * 4 + cc;
+      out[off] = (r < rows && c < nb) ? scales[r * nb + c] : 0;
+    }
+}

@@ -100,6 +100,7 @@ void orc_unpack_guidance(const uint8_t* bits, int64_t n, uint8_t* mant);
 void orc_rtn_with_scales_rows(int fmt, const uint16_t* x, int64_t rows, int64_t cols, int32_t nseg,
                               const int64_t* seg_off, const uint8_t* scales, const float* s_t,
                               int64_t row_begin, int64_t row_end, uint8_t* codes);
+void orc_swizzle_scales(const uint8_t* scales, int64_t rows, int64_t nb, uint8_t* out);
 uint16_t orc_f32_to_bf16(float v);
 void orc_f32_to_bf16_array(const float* v, int64_t n, uint16_t* out);
 

@@ -455,6 +455,39 @@ def test_empty_tensor():
     assert q.s_t.shape == (2,) and not q.s_t.any()
 
 
+@pytest.mark.parametrize("fmt,shape", [(O.NVFP4, (1, 16)), (O.NVFP4, (130, 80)), (O.MXFP4, (300, 2048)),
+                                       (O.UFP4, (77, 48)), (O.NVFP4, (256, 4096))])
+def test_swizzled_scales_parity(fmt, shape):
+    """Scale bytes in the tiled layout of block-scaled GEMMs: the oracle's
+    index map, zero padding included."""
+    xb = W.random_bf16(shape, seed=sum(shape) + 9, device=DEV, outlier_frac=0.01)
+    q, r = check_quant(xb, fmt)
+    blk = B.tf4_swizzle_scales(q)
+    want = O.swizzle_scales(r["scales"].reshape(shape[0], -1))
+    assert_same("blocked scales", host(blk), want)
+
+
+def test_block_scaled_gemm_consumes_the_record():
+    """An NVFP4 record (codes + tiled E4M3 scales) fed to the block-scaled
+    FP4 GEMM behind torch._scaled_mm gives the product of the dequantized
+    matrices times the two tensor scales (which the GEMM leaves out), within
+    the bf16 output's rounding.  (torch's FP4 GEMM takes E4M3 block scales
+    only; the MXFP4 layout is checked against the oracle above.)"""
+    fmt = O.NVFP4
+    m, n, k = 256, 384, 1024
+    a = W.random_bf16((m, k), seed=91, device=DEV, outlier_frac=0.01)
+    b = W.random_bf16((n, k), seed=92, device=DEV, outlier_frac=0.01)
+    qa, qb = B.tf4_quantize_capture(a, fmt=fmt), B.tf4_quantize_capture(b, fmt=fmt)
+    sdt = torch.float8_e4m3fn
+    sa, sb = B.tf4_swizzle_scales(qa).view(sdt).reshape(-1), B.tf4_swizzle_scales(qb).view(sdt).reshape(-1)
+    fa = qa.codes.view(m, k // 2).view(torch.float4_e2m1fn_x2)
+    fb = qb.codes.view(n, k // 2).view(torch.float4_e2m1fn_x2)
+    c = torch._scaled_mm(fa, fb.t(), sa, sb, out_dtype=torch.bfloat16).float() * (qa.s_t * qb.s_t)
+    ref = B.tf4_dequantize(qa) @ B.tf4_dequantize(qb).t()
+    err = (c - ref).abs().max().item()
+    assert err <= 2.0 ** -7 * ref.abs().max().item(), (err, ref.abs().max().item())
+
+
 def test_cuda_graph_capture_and_replay():
     """The calls launch only kernels on the given stream (no allocation, no
     host synchronisation), so a rollout capture + train-side fake-quant step

@@ -512,3 +512,33 @@ def test_mismatch_stats_closed_form(orc):
     xt[0] = W.bf16_bits(torch.from_numpy(vt).to(torch.bfloat16).reshape(1, 32))[0]
     st = orc.mismatch_stats(xt, r["scales"], r["codes"], orc.MXFP4)
     assert st.tolist() == [2, 1, 1, 1]
+
+
+def _torch_to_blocked():
+    """torch's rearrangement helper, taken from its testing module by
+    compiling just that function (the module itself needs packages this
+    image lacks)."""
+    import ast
+    import torch.testing._internal as ti
+    path = os.path.join(os.path.dirname(ti.__file__), "common_quantized.py")
+    tree = ast.parse(open(path).read())
+    keep = [n for n in tree.body if isinstance(n, ast.FunctionDef) and n.name in ("to_blocked", "ceil_div")]
+    ns = {"torch": torch, "math": math}
+    exec(compile(ast.Module(body=keep, type_ignores=[]), path, "exec"), ns)
+    if "ceil_div" not in ns:
+        ns["ceil_div"] = lambda a, b: (a + b - 1) // b
+    return ns["to_blocked"]
+
+
+def test_swizzled_scales_vs_torch_to_blocked(orc):
+    """The tiled scale layout of block-scaled GEMMs: the oracle's index map
+    against torch's own rearrangement helper (an independent implementation
+    of the same documented layout), with ragged row and column counts."""
+    to_blocked = _torch_to_blocked()
+    rng = np.random.default_rng(21)
+    for rows, nb in [(1, 1), (128, 4), (130, 5), (300, 64), (77, 3), (256, 896)]:
+        sc = rng.integers(1, 255, size=(rows, nb), dtype=np.uint8)
+        want = to_blocked(torch.from_numpy(sc)).reshape(-1).numpy()
+        got = orc.swizzle_scales(sc)
+        assert got.shape == want.shape and np.array_equal(got, want), (rows, nb)
+        assert np.count_nonzero(got) == rows * nb  # a permutation of the entries, zero padding
