@@ -716,6 +716,17 @@ def run_suite(args):
         fq_and_diag(name, "mxfp4", q, x, xt)
         del q, g, out, qr
 
+    name = "reference streams (torch, 1 GiB)"
+    if sel(name):
+        # the measured-peak cross-check, not the library: a device copy
+        buf = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+        src = torch.empty(1 << 30, dtype=torch.uint8, device=dev)
+        for call, fn, bpb in (("copy (read + write)", lambda: buf.copy_(src), 2.0),):
+            us = timed(fn)
+            gbs = bpb * (1 << 30) / (us * 1e-6) / 1e9
+            rows_out.append(dict(workload=name, format="-", call=call, elements=1 << 30, us=round(us, 2),
+                                 gbs=round(gbs, 1), frac=round(gbs / peak, 4), elements_per_s=None))
+        del buf, src
     name = "activation_outliers 4096x2048"
     if sel(name):
         w = W.activation_outliers(dev)
