@@ -23,6 +23,9 @@
  *               uniform 4-bit grid (E1M2 / INT4) in place of E2M1.
  *   [PHILOX]    Salmon, Moraes, Dror, Shaw, "Parallel random numbers: as
  *               easy as 1, 2, 3", SC'11 -- the Philox4x32-10 generator.
+ *   [CUBLAS]    NVIDIA cuBLAS documentation, "1D Block Scaling Factors
+ *               Layout" -- the tiled scale layout of block-scaled GEMMs
+ *               (not on the TRACE pages; used by orc_swizzle_scales).
  *
  * Layouts (identical to the library's public layouts, restated here):
  *   x        bf16 bit patterns, row-major [rows, cols], cols % block == 0
