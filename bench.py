@@ -348,17 +348,35 @@ def run_ours(args, world, rank, local):
 def run_e2e(args, world, dev, xs, xts, recs, amax, gcodes):
     """Same step through the public API with host buffers: every step copies
     the layers' inputs from pinned host memory (double-buffered on a copy
-    stream) and reads every result back to pinned host memory."""
+    stream) and reads every result back to pinned host memory.  With several
+    ranks on one host each rank takes a 1/world share of the stack (half of
+    it deep layers), so the pinned host memory stays that of one stack."""
     import psutil
 
     from fp4_block_scaled_quantizer_b200 import binding as B
 
+    if world > 1:
+        Lf, Df = args.layers, args.deep
+        L = max(2, Lf // world)
+        D = min(Df, L // 2)
+        keep = list(range(L - D)) + list(range(Lf - D, Lf))  # some shallow layers, then the deepest D
+        xs, recs, amax = [xs[i] for i in keep], [recs[i] for i in keep], [amax[i] for i in keep]
+        xts, gcodes = xts[Df - D:], gcodes[Df - D:]
+        args = argparse.Namespace(**{**vars(args), "layers": L, "deep": D})
     L, D = args.layers, args.deep
     first_deep = L - D
     n = args.rows * args.cols
     in_bytes = (L + D) * n * 2
     out_bytes = L * (n // 2 + n // 16 + 4) + D * (n // 8 + n // 2)
-    if psutil.virtual_memory().available < 1.6 * (in_bytes + out_bytes):
+    local = int(os.environ.get("LOCAL_WORLD_SIZE", "1"))
+    ok = psutil.virtual_memory().available >= 1.6 * (in_bytes + out_bytes) * local
+    if world > 1:  # every rank takes the same branch
+        import torch.distributed as dist
+
+        f = torch.tensor([1 if ok else 0], dtype=torch.int32, device=dev)
+        dist.all_reduce(f, op=dist.ReduceOp.MIN)
+        ok = bool(f.item())
+    if not ok:
         return dict(value=None, unit="GB/s", skipped="not enough host memory for pinned buffers")
     hx = [torch.empty_like(x, device="cpu").pin_memory() for x in xs]
     hxt = [torch.empty_like(x, device="cpu").pin_memory() for x in xts]
@@ -431,6 +449,7 @@ def run_e2e(args, world, dev, xs, xts, recs, amax, gcodes):
     bytes_step, _ = step_bytes(args)
     return dict(value=round(world * bytes_step / (ms * 1e-3) / 1e9, 2), unit="GB/s", ms_per_step=round(ms, 2),
                 h2d_bytes_per_step=in_bytes, d2h_bytes_per_step=out_bytes, steps=args.e2e_steps,
+                layers_per_rank=L, deep_layers_per_rank=D,
                 overlap="double-buffered H2D on a copy stream, D2H on a third stream")
 
 
