@@ -193,9 +193,11 @@ def test_tiny_and_zero_scales(fmt):
     x[4, 5] = 0x0C00          # ~1e-35
     xb = W.from_bits(x, DEV)
     check_quant(xb, fmt)
+    check_quant(xb, fmt, O.SR, seed=3)  # E4M3-subnormal and zero scales take the exact SR path
     seg = [0, 2, 2, 4, 8]
     if O.HAS_TENSOR_SCALE[fmt]:
         check_quant(xb, fmt, seg=seg)
+        check_quant(xb, fmt, O.SR, seg=seg, seed=4)
 
 
 @pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
