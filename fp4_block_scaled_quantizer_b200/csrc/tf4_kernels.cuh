@@ -2,10 +2,13 @@
 //
 // Streaming, elementwise + reduction work: no tensor cores.  Every kernel
 // splits its flat array of quantization blocks into one contiguous range
-// per CTA (grid = SMs x resident CTAs, one wave), and lanes of a warp take
-// consecutive blocks so that each warp instruction moves a contiguous span.
-// NVFP4: one lane owns one 16-element block (32 B of bf16, two 16-B loads);
-// MXFP4: one lane owns one 32-element block (four 16-B loads).
+// per CTA (grid = 1 to 4 waves of SMs x resident CTAs, chosen on the host),
+// and lanes of a warp take consecutive work units so that each warp
+// instruction moves a contiguous span.  Quantize / guided passes: one lane
+// owns one block per unit (NVFP4 / UFP4: 16 elements, 32 B of bf16, two
+// 16-B loads; MXFP4: 32 elements, four loads); the fused fake-quant and the
+// wide-store dequantize take 8 elements per lane, the narrow-store
+// dequantize 4.
 //
 // Definitions followed are stated in include/trace_fp4.h (and the pages
 // cited there); the notes below only explain how each kernel reaches the
