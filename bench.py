@@ -745,7 +745,26 @@ def run_suite(args):
             gbs = bpb * (1 << 30) / (us * 1e-6) / 1e9
             rows_out.append(dict(workload=name, format="-", call=call, elements=1 << 30, us=round(us, 2),
                                  gbs=round(gbs, 1), frac=round(gbs / peak, 4), elements_per_s=None))
-        del buf, src
+        # the host link that bounds the end-to-end figure: pinned host <-> device copies (frac: none, not HBM)
+        hsrc = torch.empty(1 << 30, dtype=torch.uint8).pin_memory()
+        hdst = torch.empty(1 << 30, dtype=torch.uint8).pin_memory()
+        side = torch.cuda.Stream(dev)
+
+        def both():
+            side.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(side):
+                hdst.copy_(src, non_blocking=True)
+            buf.copy_(hsrc, non_blocking=True)
+            torch.cuda.current_stream(dev).wait_stream(side)
+
+        for call, fn, bpb in (("pinned host -> device copy", lambda: buf.copy_(hsrc, non_blocking=True), 1.0),
+                              ("device -> pinned host copy", lambda: hdst.copy_(src, non_blocking=True), 1.0),
+                              ("both directions at once (2 x 1 GiB)", both, 2.0)):
+            us = timed(fn, reps=5)
+            gbs = bpb * (1 << 30) / (us * 1e-6) / 1e9
+            rows_out.append(dict(workload=name, format="-", call=call, elements=1 << 30, us=round(us, 2),
+                                 gbs=round(gbs, 1), frac=None, elements_per_s=None))
+        del buf, src, hsrc, hdst
     name = "activation_outliers 4096x2048"
     if sel(name):
         w = W.activation_outliers(dev)

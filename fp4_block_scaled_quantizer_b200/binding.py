@@ -149,8 +149,28 @@ class Desc:
 def _ptr(t: Optional[torch.Tensor]):
     if t is None:
         return None
-    assert t.is_cuda and t.is_contiguous(), "expected a contiguous CUDA tensor"
+    if not (t.is_cuda and t.is_contiguous()):
+        raise ValueError(f"expected a contiguous CUDA tensor, got one on {t.device}"
+                         f"{'' if t.is_contiguous() else ' (not contiguous)'}")
     return ctypes.c_void_p(t.data_ptr())
+
+
+def _buf(t: Optional[torch.Tensor], name: str, numel: int, dtype: torch.dtype, device: torch.device):
+    """Check a caller-supplied buffer before its pointer is handed to the
+    library, which cannot see sizes: a CUDA tensor on `device`, contiguous,
+    of `dtype`, with at least `numel` elements (the kernels read or write
+    exactly `numel`; a shorter buffer would be overrun)."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name}: expected a torch.Tensor, got {type(t).__name__}")
+    if not t.is_cuda or t.device != device:
+        raise ValueError(f"{name}: expected a CUDA tensor on {device}, got one on {t.device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: expected a contiguous tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: expected dtype {dtype}, got {t.dtype}")
+    if t.numel() < numel:
+        raise ValueError(f"{name}: needs {numel} elements, has {t.numel()}")
+    return t
 
 
 def _stream(stream: Optional[torch.cuda.Stream], device) -> ctypes.c_void_p:
@@ -164,9 +184,27 @@ def _check(status: int, what: str):
 
 
 def _as_2d(x: torch.Tensor):
-    assert x.dtype == torch.bfloat16, "input must be bf16"
-    assert x.is_cuda and x.is_contiguous()
+    if not isinstance(x, torch.Tensor):
+        raise TypeError(f"expected a torch.Tensor, got {type(x).__name__}")
+    if x.dtype != torch.bfloat16:
+        raise TypeError(f"input must be bf16, got {x.dtype}")
+    if not (x.is_cuda and x.is_contiguous()):
+        raise ValueError(f"input must be a contiguous CUDA tensor (got one on {x.device})")
+    if x.dim() == 0:
+        raise ValueError("input must have at least one dimension")
     return x.reshape(-1, x.shape[-1]) if x.dim() != 2 else x
+
+
+def _check_record(rec, desc: "Desc", device, name: str, bits=None, codes=False):
+    """Sizes of a rollout record's buffers against the shape they are used with."""
+    nb = desc.n // BLOCK[desc.fmt]
+    _buf(rec.scales, f"{name}: record scales", nb, torch.uint8, device)
+    if HAS_TENSOR_SCALE[desc.fmt]:
+        _buf(rec.s_t, f"{name}: record s_t", desc.num_segments, torch.float32, device)
+    if bits is not None:
+        _buf(bits, f"{name}: guidance bits", desc.n // 8, torch.uint8, device)
+    if codes:
+        _buf(rec.codes, f"{name}: record codes", desc.n // 2, torch.uint8, device)
 
 
 _ws_cache: dict = {}
@@ -227,6 +265,14 @@ class Quantized:
 
 def _outputs(desc: Desc, device, want_bits: bool, out: Optional[Quantized]):
     if out is not None:
+        _buf(out.codes, "out.codes", desc.n // 2, torch.uint8, device)
+        _buf(out.scales, "out.scales", desc.n // BLOCK[desc.fmt], torch.uint8, device)
+        if HAS_TENSOR_SCALE[desc.fmt]:
+            _buf(out.s_t, "out.s_t", desc.num_segments, torch.float32, device)
+        if want_bits:
+            _buf(out.bits, "out.bits", desc.n // 8, torch.uint8, device)
+        # the record describes what this call wrote
+        out.fmt, out.rows, out.cols, out.seg_off = desc.fmt, desc.rows, desc.cols, desc.seg_off
         return out
     codes = torch.empty(desc.n // 2, dtype=torch.uint8, device=device)
     scales = torch.empty((desc.rows, desc.cols // BLOCK[desc.fmt]), dtype=torch.uint8, device=device)
@@ -236,10 +282,16 @@ def _outputs(desc: Desc, device, want_bits: bool, out: Optional[Quantized]):
     return Quantized(codes, scales, s_t, bits, desc.fmt, desc.rows, desc.cols, desc.seg_off)
 
 
+def _amax_in(amax_in, desc: Desc, device):
+    if amax_in is not None:
+        _buf(amax_in, "amax_in", desc.num_segments, torch.float32, device)
+
+
 def tf4_segment_amax(x: torch.Tensor, seg_off=None, stream=None, out=None) -> torch.Tensor:
     x2 = _as_2d(x)
     d = Desc(NVFP4, x2.shape[0], x2.shape[1], seg_off)
-    amax = out if out is not None else torch.empty(d.num_segments, dtype=torch.float32, device=x.device)
+    amax = (_buf(out, "out", d.num_segments, torch.float32, x.device) if out is not None
+            else torch.empty(d.num_segments, dtype=torch.float32, device=x.device))
     ws = workspace(d, x.device, stream)
     _check(lib().tf4_segment_amax(d.ptr, _ptr(x2), _ptr(amax), _ptr(ws), ws.numel(),
                                   _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_segment_amax")
@@ -250,6 +302,7 @@ def tf4_quantize_rtn(x, fmt=NVFP4, seg_off=None, amax_in=None, stream=None, out=
     x2 = _as_2d(x)
     d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
     q = _outputs(d, x.device, False, out)
+    _amax_in(amax_in, d, x.device)
     ws = workspace(d, x.device, stream)
     _check(lib().tf4_quantize_rtn(d.ptr, _ptr(x2), _ptr(amax_in), _ptr(q.codes), _ptr(q.scales), _ptr(q.s_t),
                                   _ptr(ws), ws.numel(), _ptr(status_word(x.device)), _stream(stream, x.device)),
@@ -261,6 +314,7 @@ def tf4_quantize_sr(x, seed: int, fmt=NVFP4, seg_off=None, amax_in=None, stream=
     x2 = _as_2d(x)
     d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
     q = _outputs(d, x.device, False, out)
+    _amax_in(amax_in, d, x.device)
     ws = workspace(d, x.device, stream)
     _check(lib().tf4_quantize_sr(d.ptr, _ptr(x2), ctypes.c_uint64(seed & (2**64 - 1)), _ptr(amax_in),
                                  _ptr(q.codes), _ptr(q.scales), _ptr(q.s_t), _ptr(ws), ws.numel(),
@@ -275,6 +329,7 @@ def tf4_quantize_capture(x, fmt=NVFP4, seg_off=None, guidance=True, amax_in=None
     x2 = _as_2d(x)
     d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
     q = _outputs(d, x.device, guidance, out)
+    _amax_in(amax_in, d, x.device)
     ws = workspace(d, x.device, stream)
     _check(lib().tf4_quantize_capture(d.ptr, _ptr(x2), _ptr(amax_in), _ptr(q.codes), _ptr(q.scales),
                                       _ptr(q.s_t), _ptr(q.bits if guidance else None), _ptr(ws), ws.numel(),
@@ -306,12 +361,25 @@ def tf4_quantize_capture_batched(xs, fmt=NVFP4, keep=0, stream=None, out: Option
     """Capture a list of same-shaped bf16 tensors (layers) in two launches;
     guidance is kept for the last `keep` layers, in one contiguous buffer."""
     L = len(xs)
+    if L == 0:
+        raise ValueError("tf4_quantize_capture_batched: no layers")
     x2 = [_as_2d(x) for x in xs]
     rows, cols = x2[0].shape
-    assert all(t.shape == (rows, cols) for t in x2)
     dev = x2[0].device
+    if any(t.shape != (rows, cols) or t.device != dev for t in x2):
+        raise ValueError("tf4_quantize_capture_batched: layers must share one shape and one device")
+    if not 0 <= keep <= L:
+        raise ValueError(f"tf4_quantize_capture_batched: keep={keep} outside [0, {L}]")
     d = Desc(fmt, rows, cols)
-    if out is None:
+    if out is not None:
+        n = rows * cols
+        _buf(out.codes, "out.codes", L * (n // 2), torch.uint8, dev)
+        _buf(out.scales, "out.scales", L * (n // BLOCK[fmt]), torch.uint8, dev)
+        if HAS_TENSOR_SCALE[fmt]:
+            _buf(out.s_t, "out.s_t", L, torch.float32, dev)
+        if keep:
+            _buf(out.info_bits, "out.info_bits", keep * (n // 8), torch.uint8, dev)
+    else:
         n = rows * cols
         out = BatchedCapture(torch.empty((L, n // 2), dtype=torch.uint8, device=dev),
                              torch.empty((L, rows, cols // BLOCK[fmt]), dtype=torch.uint8, device=dev),
@@ -332,8 +400,11 @@ def tf4_quantize_guided(x, rec: Quantized, stream=None, out=None, rec_bits=None)
     x2 = _as_2d(x)
     d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
     bits = rec_bits if rec_bits is not None else rec.bits
-    assert bits is not None, "the record holds no guidance bits"
-    codes = out if out is not None else torch.empty(d.n // 2, dtype=torch.uint8, device=x.device)
+    if bits is None:
+        raise ValueError("tf4_quantize_guided: the record holds no guidance bits")
+    _check_record(rec, d, x.device, "tf4_quantize_guided", bits=bits)
+    codes = (_buf(out, "out", d.n // 2, torch.uint8, x.device) if out is not None
+             else torch.empty(d.n // 2, dtype=torch.uint8, device=x.device))
     _check(lib().tf4_quantize_guided(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(bits), _ptr(codes),
                                      _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_quantize_guided")
     return codes
@@ -344,14 +415,24 @@ def tf4_guided_fake_quant(x, rec: Quantized, out_dtype=torch.float32, want_codes
     """Guided quantization + dequantization in one pass.  Returns (values,
     codes): values [rows, cols] in out_dtype (float32, or bfloat16 = RNE of
     the fp32 value); codes only if want_codes (else None)."""
-    assert out_dtype in (torch.float32, torch.bfloat16)
+    if out_dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError(f"tf4_guided_fake_quant: out_dtype must be float32 or bfloat16, got {out_dtype}")
     x2 = _as_2d(x)
     d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
     bits = rec_bits if rec_bits is not None else rec.bits
-    assert bits is not None, "the record holds no guidance bits"
-    o = out if out is not None else torch.empty(x2.shape, dtype=out_dtype, device=x.device)
-    c = codes if codes is not None else (
-        torch.empty(d.n // 2, dtype=torch.uint8, device=x.device) if want_codes else None)
+    if bits is None:
+        raise ValueError("tf4_guided_fake_quant: the record holds no guidance bits")
+    _check_record(rec, d, x.device, "tf4_guided_fake_quant", bits=bits)
+    if out is not None:
+        if not isinstance(out, torch.Tensor) or out.dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError("tf4_guided_fake_quant: out must be a float32 or bfloat16 tensor")
+        o = _buf(out, "out", d.n, out.dtype, x.device)
+    else:
+        o = torch.empty(x2.shape, dtype=out_dtype, device=x.device)
+    if codes is not None:
+        c = _buf(codes, "codes", d.n // 2, torch.uint8, x.device)
+    else:
+        c = torch.empty(d.n // 2, dtype=torch.uint8, device=x.device) if want_codes else None
     _check(lib().tf4_guided_fake_quant(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(bits), _ptr(c),
                                        _ptr(o), 1 if o.dtype == torch.bfloat16 else 0,
                                        _ptr(status_word(x.device)), _stream(stream, x.device)),
@@ -365,7 +446,9 @@ def tf4_mismatch_stats(x, rec: Quantized, counts=None, stream=None) -> torch.Ten
     `counts` (int64 [4], zero-initialised if not given) and returns it."""
     x2 = _as_2d(x)
     d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
-    c = counts if counts is not None else torch.zeros(4, dtype=torch.int64, device=x.device)
+    _check_record(rec, d, x.device, "tf4_mismatch_stats", codes=True)
+    c = (_buf(counts, "counts", 4, torch.int64, x.device) if counts is not None
+         else torch.zeros(4, dtype=torch.int64, device=x.device))
     _check(lib().tf4_mismatch_stats(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(rec.codes), _ptr(c),
                                     _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_mismatch_stats")
     return c
@@ -374,7 +457,12 @@ def tf4_mismatch_stats(x, rec: Quantized, counts=None, stream=None) -> torch.Ten
 def tf4_dequantize(q: Quantized, codes=None, stream=None, out=None) -> torch.Tensor:
     d = Desc(q.fmt, q.rows, q.cols, q.seg_off)
     c = codes if codes is not None else q.codes
-    o = out if out is not None else torch.empty((q.rows, q.cols), dtype=torch.float32, device=c.device)
+    if not isinstance(c, torch.Tensor) or not c.is_cuda:
+        raise ValueError("tf4_dequantize: codes must be a CUDA tensor")
+    _buf(c, "codes", d.n // 2, torch.uint8, c.device)
+    _check_record(q, d, c.device, "tf4_dequantize")
+    o = (_buf(out, "out", d.n, torch.float32, c.device) if out is not None
+         else torch.empty((q.rows, q.cols), dtype=torch.float32, device=c.device))
     _check(lib().tf4_dequantize(d.ptr, _ptr(c), _ptr(q.scales), _ptr(q.s_t), _ptr(o), _stream(stream, c.device)),
            "tf4_dequantize")
     return o
@@ -386,8 +474,12 @@ def tf4_swizzle_scales(q: Quantized, stream=None, out=None) -> torch.Tensor:
     d = Desc(q.fmt, q.rows, q.cols, q.seg_off)
     nb = q.cols // BLOCK[q.fmt]
     shape = ((q.rows + 127) // 128 * 128, (nb + 3) // 4 * 4)
-    assert lib().tf4_blocked_scales_bytes(d.ptr) == shape[0] * shape[1]
-    o = out if out is not None else torch.empty(shape, dtype=torch.uint8, device=q.scales.device)
+    if not isinstance(q.scales, torch.Tensor) or not q.scales.is_cuda:
+        raise ValueError("tf4_swizzle_scales: the record's scales must be a CUDA tensor")
+    dev = q.scales.device
+    _buf(q.scales, "record scales", q.rows * nb, torch.uint8, dev)
+    o = (_buf(out, "out", shape[0] * shape[1], torch.uint8, dev) if out is not None
+         else torch.empty(shape, dtype=torch.uint8, device=dev))
     _check(lib().tf4_swizzle_scales(d.ptr, _ptr(q.scales), _ptr(o), _stream(stream, q.scales.device)),
            "tf4_swizzle_scales")
     return o
@@ -395,7 +487,11 @@ def tf4_swizzle_scales(q: Quantized, stream=None, out=None) -> torch.Tensor:
 
 def tf4_pack_guidance(codes: torch.Tensor, rows: int, cols: int, fmt=NVFP4, stream=None, out=None):
     d = Desc(fmt, rows, cols)
-    o = out if out is not None else torch.empty(d.n // 8, dtype=torch.uint8, device=codes.device)
+    if not isinstance(codes, torch.Tensor) or not codes.is_cuda:
+        raise ValueError("tf4_pack_guidance: codes must be a CUDA tensor")
+    _buf(codes, "codes", d.n // 2, torch.uint8, codes.device)
+    o = (_buf(out, "out", d.n // 8, torch.uint8, codes.device) if out is not None
+         else torch.empty(d.n // 8, dtype=torch.uint8, device=codes.device))
     _check(lib().tf4_pack_guidance(d.ptr, _ptr(codes), _ptr(o), _stream(stream, codes.device)),
            "tf4_pack_guidance")
     return o
@@ -403,7 +499,11 @@ def tf4_pack_guidance(codes: torch.Tensor, rows: int, cols: int, fmt=NVFP4, stre
 
 def tf4_unpack_guidance(bits: torch.Tensor, rows: int, cols: int, fmt=NVFP4, stream=None, out=None):
     d = Desc(fmt, rows, cols)
-    o = out if out is not None else torch.empty(d.n, dtype=torch.uint8, device=bits.device)
+    if not isinstance(bits, torch.Tensor) or not bits.is_cuda:
+        raise ValueError("tf4_unpack_guidance: bits must be a CUDA tensor")
+    _buf(bits, "bits", d.n // 8, torch.uint8, bits.device)
+    o = (_buf(out, "out", d.n, torch.uint8, bits.device) if out is not None
+         else torch.empty(d.n, dtype=torch.uint8, device=bits.device))
     _check(lib().tf4_unpack_guidance(d.ptr, _ptr(bits), _ptr(o), _stream(stream, bits.device)),
            "tf4_unpack_guidance")
     return o

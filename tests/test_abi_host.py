@@ -162,3 +162,25 @@ def test_uniform_grid_format_arguments(L):
     assert _rtn(L, B.Desc(3, 4, 32)) == 1
     s = B.sizes(B.UFP4, 64, 128)
     assert s["scales"] == 64 * 128 // 16 and s["record_full"] == 64 * 128 // 2 + 64 * 128 // 16 + 4
+
+
+def test_binding_rejects_bad_tensors_before_the_library():
+    """The binding checks dtype, device and layout of its inputs and the
+    size of caller-supplied buffers (the C ABI sees only pointers); on a
+    CPU-only host every such call is refused before any pointer is passed."""
+    import torch
+
+    with pytest.raises(TypeError):
+        B.tf4_quantize_capture(torch.zeros(4, 16, dtype=torch.float32))
+    with pytest.raises(ValueError):
+        B.tf4_quantize_capture(torch.zeros(4, 16, dtype=torch.bfloat16))  # host tensor
+    with pytest.raises(ValueError):
+        B.tf4_quantize_capture(torch.zeros(16, 4, dtype=torch.bfloat16).t())  # not contiguous
+    with pytest.raises(ValueError):
+        B._buf(torch.zeros(8, dtype=torch.uint8), "out", 8, torch.uint8, torch.device("cuda", 0))
+    with pytest.raises(TypeError):
+        B._buf(None, "out", 8, torch.uint8, torch.device("cuda", 0))
+    with pytest.raises(ValueError):
+        B.tf4_quantize_capture_batched([])
+    with pytest.raises(ValueError):
+        B.tf4_pack_guidance(torch.zeros(8, dtype=torch.uint8), 1, 16)

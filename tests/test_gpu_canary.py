@@ -102,3 +102,36 @@ def test_batched_capture_outputs_stay_inside(fmt):
     B.tf4_quantize_capture_batched(xs, fmt=fmt, keep=keep, out=out)
     assert B.read_status(xs[0].device) == 0
     g.check(f"batched fmt {fmt}")
+
+
+def test_short_or_mistyped_buffers_are_refused_before_launch():
+    """Buffers the library would overrun (or misread) are refused by the
+    binding with nothing launched: the caller's buffer keeps its bytes."""
+    rows, cols = 64, 256
+    n = rows * cols
+    x = W.random_bf16((rows, cols), seed=5, device=DEV)
+    q = B.tf4_quantize_capture(x)
+    short = torch.full((n // 2 - 1,), CANARY, dtype=torch.uint8, device=DEV)
+    with pytest.raises(ValueError):
+        B.tf4_quantize_guided(x, q, out=short)
+    with pytest.raises(ValueError):
+        B.tf4_quantize_guided(W.random_bf16((2 * rows, cols), seed=6, device=DEV), q)  # record too small
+    with pytest.raises(ValueError):
+        B.tf4_pack_guidance(q.codes, rows, cols, out=short[: n // 8 - 1])
+    with pytest.raises(ValueError):
+        B.tf4_unpack_guidance(q.bits, rows, cols, out=short)  # needs n bytes
+    bad = B.Quantized(torch.empty(n // 2, dtype=torch.uint8, device=DEV), torch.empty(10, dtype=torch.uint8, device=DEV),
+                      torch.empty(1, dtype=torch.float32, device=DEV), torch.empty(n // 8, dtype=torch.uint8, device=DEV))
+    with pytest.raises(ValueError):
+        B.tf4_quantize_capture(x, out=bad)
+    with pytest.raises(ValueError):
+        B.tf4_quantize_rtn(x, seg_off=[0, 32, 64], amax_in=torch.ones(1, device=DEV))
+    with pytest.raises(TypeError):
+        B.tf4_dequantize(q, out=torch.empty((rows, cols), dtype=torch.float16, device=DEV))
+    with pytest.raises(TypeError):
+        B.tf4_mismatch_stats(x, q, counts=torch.zeros(4, dtype=torch.int32, device=DEV))
+    with pytest.raises(TypeError):
+        B.tf4_guided_fake_quant(x, q, out=torch.empty((rows, cols), dtype=torch.float16, device=DEV))
+    torch.cuda.synchronize()
+    assert bool((short == CANARY).all())
+    assert B.read_status(x.device) == 0
