@@ -213,6 +213,35 @@ def test_segments_ragged_with_empties(fmt):
 
 
 @pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
+def test_maximum_segment_count(fmt):
+    """TF4_MAX_SEGMENTS (1024) ragged segments, about a fifth of them empty,
+    each with its own tensor scale (values scaled per segment over 2^-20 ..
+    2^20): capture, SR, guided, dequantize and fused fake-quant = oracle."""
+    rng = np.random.default_rng(21)
+    rows, cols, nseg = 3000, 64, B.MAX_SEGMENTS
+    cuts = np.sort(rng.integers(0, rows + 1, size=nseg - 1))
+    cuts[rng.random(nseg - 1) < 0.2] = cuts[0]  # repeated offsets: empty segments
+    seg = [0] + sorted(int(c) for c in cuts) + [rows]
+    row_scale = np.ones(rows, np.float32)
+    for s in range(nseg):
+        row_scale[seg[s]:seg[s + 1]] = 2.0 ** rng.integers(-20, 21)
+    x = W.random_bf16((rows, cols), seed=22, device=DEV, outlier_frac=0.01)
+    xb = (x.float() * torch.from_numpy(row_scale).to(DEV)[:, None]).to(torch.bfloat16)
+    q, r = check_quant(xb, fmt, seg=seg)
+    check_quant(xb, fmt, O.SR, seg=seg, seed=23)
+    xt = W.perturb(xb, 24, rel=0.02)
+    xts = W.bf16_bits(xt)
+    want, _ = O.quantize_guided(xts, r["scales"], r["bits"], fmt, rec_s_t=r["s_t"], seg_off=seg)
+    assert_same("guided", host(B.tf4_quantize_guided(xt, q)), want)
+    rd = O.dequantize(r["codes"], r["scales"], rows, cols, fmt, s_t=r["s_t"], seg_off=seg)
+    assert_same("dequant", f32_bits(host(B.tf4_dequantize(q))), f32_bits(rd))
+    y, _ = B.tf4_guided_fake_quant(xt, q)
+    _, rv, _ = O.guided_fake_quant(xts, r["scales"], r["bits"], fmt, rec_s_t=r["s_t"], seg_off=seg)
+    assert_same("fake-quant", f32_bits(host(y)), f32_bits(rv))
+    assert B.read_status(xb.device) == 0
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
 def test_segment_amax_and_amax_in(fmt):
     xb = W.random_bf16((200, 512), seed=12, device=DEV, outlier_frac=0.01)
     seg = [0, 20, 20, 150, 200]
@@ -396,6 +425,25 @@ def test_capture_batched_parity(fmt, L, keep):
     if keep:
         g = B.tf4_quantize_guided(xs[-1], out.layer(L - 1))
         assert torch.equal(g, out.codes[L - 1])
+
+
+@pytest.mark.parametrize("fmt,keep", [(O.NVFP4, 64), (O.MXFP4, 1), (O.UFP4, 33)])
+def test_capture_batched_maximum_layer_count(fmt, keep):
+    """TF4_MAX_BATCH (64) layers in one call, each with its own scale range."""
+    L = 64
+    blk = O.BLOCK[fmt]
+    xs = [(W.random_bf16((7, 3 * blk), seed=200 + i, device=DEV, outlier_frac=0.05).float() * 2.0 ** (i - 32)
+           ).to(torch.bfloat16) for i in range(L)]
+    out = B.tf4_quantize_capture_batched(xs, fmt=fmt, keep=keep)
+    assert B.read_status(xs[0].device) == 0
+    for i, x in enumerate(xs):
+        r = O.quantize(W.bf16_bits(x), fmt, O.RTN, bits=True)
+        assert_same(f"codes {i}", host(out.codes[i]), r["codes"])
+        assert_same(f"scales {i}", host(out.scales[i]), r["scales"])
+        if O.HAS_TENSOR_SCALE[fmt]:
+            assert_same(f"s_t {i}", f32_bits(host(out.s_t[i:i + 1])), f32_bits(r["s_t"]))
+        if i >= L - keep:
+            assert_same(f"bits {i}", host(out.info_bits[i - (L - keep)]), r["bits"])
 
 
 def test_capture_batched_large_layers_per_layer_path():
