@@ -67,7 +67,10 @@
  * 0).  NULL means one segment.  MXFP4 requires num_segments == 1.
  *
  * Ownership, streams, errors.  The caller owns every buffer (device memory
- * unless stated).  The library never allocates, frees or synchronizes,
+ * unless stated) and sizes it as the Layouts above say: the library sees
+ * pointers only and cannot check a buffer's extent (the Python binding
+ * checks every tensor's size, dtype and device before passing its pointer).
+ * The library never allocates, frees or synchronizes,
  * except tf4_read_status, which synchronizes its stream.  Every call is
  * asynchronous on `stream` and launches on the current CUDA device.
  * Argument, shape and alignment problems are returned before anything is
