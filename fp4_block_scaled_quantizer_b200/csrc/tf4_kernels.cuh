@@ -844,8 +844,20 @@ __device__ __forceinline__ void report_bad(bool bad, int32_t* status) {
 // Quantize pass.  CTAs take the amax pass's ranges in reverse order (CTA i
 // gets range G-1-i) and walk them backwards, so that the first blocks read
 // are the ones the amax pass read last (still in L2).
+// Resident CTAs per SM asked of the compiler (0: its own choice).  The
+// ragged-segment nearest / capture variants are held to 5 (48 registers,
+// a few loop invariants spilled), which measured 2-3% faster on the MoE
+// dispatch workload than the 64 registers / 4 CTAs they take otherwise;
+// the batched variants lost that way (MXFP4: 140 -> 175 us for 40 layers
+// of 4096x2048), and a bound of 1 lets the compiler take far more
+// registers, so every other variant keeps the compiler's choice.
+template <int MODE, class SEG>
+constexpr int quant_min_ctas() {
+  return (MODE != kSR && std::is_same<SEG, SegN>::value) ? 5 : 0;
+}
+
 template <int FMT, int MODE, class SEG>
-__global__ void __launch_bounds__(kThreads) k_quant(QuantArgs a, SEG seg, PhiloxKeys pk) {
+__global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant(QuantArgs a, SEG seg, PhiloxKeys pk) {
   pdl_enter();
   // blocks per lane per iteration: 2 keeps 64 B per lane in flight for the
   // memory-bound modes; stochastic rounding is bound by the integer pipe
