@@ -720,6 +720,45 @@ def test_nvfp4_capture_beyond_2_32_elements():
     torch.cuda.empty_cache()
 
 
+def test_dequant_fake_quant_unpack_diagnostics_beyond_2_32_elements():
+    """The other 64-bit paths on a (2^32 + 2^20)-element NVFP4 record:
+    dequantize (32-byte stores), bf16 fused fake-quant, unpack and the
+    mismatch diagnostics; rows across the 2^32 boundary against the oracle."""
+    cols = 4096
+    rows = (2**32 + 2**20) // cols
+    g = torch.Generator(device=DEV).manual_seed(10)
+    x = torch.randn((rows, cols), generator=g, device=DEV, dtype=torch.bfloat16)
+    q = B.tf4_quantize_capture(x)
+    cnt = B.tf4_mismatch_stats(x, q)
+    assert cnt.tolist() == [0, 0, 0, 0]
+    r0 = 2**32 // cols
+    sample = (0, r0 - 1, r0, r0 + 1, rows - 1)
+    st = host(q.s_t)
+    got = {}
+    d = B.tf4_dequantize(q)
+    got["dequant"] = {r: host(d[r]) for r in sample}
+    del d
+    y, _ = B.tf4_guided_fake_quant(x, q, out_dtype=torch.bfloat16)
+    got["fq"] = {r: host(y[r].view(torch.int16)).view(np.uint16) for r in sample}
+    del y
+    mant = B.tf4_unpack_guidance(q.bits, rows, cols)
+    got["unpack"] = {r: host(mant[r * cols:(r + 1) * cols]) for r in sample}
+    del mant
+    assert B.read_status(x.device) == 0
+    for r in sample:
+        xs = W.bf16_bits(x[r:r + 1])
+        codes = host(q.codes[r * cols // 2:(r + 1) * cols // 2])
+        scales = host(q.scales[r])
+        bits = host(q.bits[r * cols // 8:(r + 1) * cols // 8])
+        rd = O.dequantize(codes, scales, 1, cols, O.NVFP4, s_t=st)
+        assert_same(f"dequant row {r}", f32_bits(got["dequant"][r]), f32_bits(rd))
+        _, rv, _ = O.guided_fake_quant(xs, scales, bits, O.NVFP4, rec_s_t=st)
+        assert_same(f"fake-quant row {r}", got["fq"][r], O.f32_to_bf16(rv))
+        assert_same(f"unpack row {r}", got["unpack"][r], O.unpack_guidance(bits, cols))
+    del x, q
+    torch.cuda.empty_cache()
+
+
 def _oracle_row_with_offset(row_bits, base_index, seed):
     """Oracle SR codes of one MXFP4 row whose first element has flat index
     base_index (element-level oracle calls)."""
