@@ -14,6 +14,7 @@ the same names take tensors.
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -24,6 +25,7 @@ import torch
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libtrace_fp4.so")
+DEBUG_LIB_PATH = os.path.join(HERE, "libtrace_fp4_debug.so")  # built with --debug-bounds
 
 NVFP4, MXFP4, UFP4 = 0, 1, 2
 BLOCK = {NVFP4: 16, MXFP4: 32, UFP4: 16}
@@ -44,7 +46,7 @@ EXPORTS = (
     "tf4_quantize_capture", "tf4_quantize_guided", "tf4_dequantize", "tf4_pack_guidance",
     "tf4_unpack_guidance", "tf4_guided_fake_quant", "tf4_mismatch_stats", "tf4_workspace_bytes_batched",
     "tf4_quantize_capture_batched", "tf4_blocked_scales_bytes", "tf4_swizzle_scales", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
-    "tf4_version",
+    "tf4_version", "tf4_debug_bounds_enabled", "tf4_debug_bounds_violations",
 )
 
 
@@ -106,6 +108,8 @@ def lib():
                     "tf4_read_status": (st, [i32p, vp]),
                     "tf4_status_string": (ctypes.c_char_p, [st]),
                     "tf4_version": (ctypes.c_int, []),
+                    "tf4_debug_bounds_enabled": (ctypes.c_int, []),
+                    "tf4_debug_bounds_violations": (st, [ctypes.POINTER(ctypes.c_uint64), vp]),
                 }
                 for name, (res, args) in sig.items():
                     fn = getattr(L, name)
@@ -234,6 +238,31 @@ def status_word(device) -> torch.Tensor:
         t = torch.zeros(1, dtype=torch.int32, device=device)
         _status_cache[key] = t
     return t
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Route this module's calls through the library at `path` (for example
+    the bounds-checking build, DEBUG_LIB_PATH) inside the `with` block."""
+    global _lib, LIB_PATH
+    with _lock:
+        saved = (_lib, LIB_PATH)
+        _lib, LIB_PATH = None, path
+    try:
+        yield lib()
+    finally:
+        with _lock:
+            _lib, LIB_PATH = saved
+
+
+def debug_bounds_violations(device=None, stream=None) -> int:
+    """Synchronize and return (and reset) the number of work units the
+    kernels skipped as out of range; always 0 unless the loaded library is
+    the bounds-checking build."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    n = ctypes.c_uint64(0)
+    _check(lib().tf4_debug_bounds_violations(ctypes.byref(n), _stream(stream, dev)), "tf4_debug_bounds_violations")
+    return int(n.value)
 
 
 def read_status(device, stream=None) -> int:

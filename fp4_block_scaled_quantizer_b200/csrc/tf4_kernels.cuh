@@ -116,6 +116,26 @@ __device__ __forceinline__ int64_t cta_begin(int64_t i, int64_t grid, int64_t n)
   return i * q + (i < r ? i : r);
 }
 
+// ------------------------------------------------------- debug bounds
+// Builds with TF4_DEBUG_BOUNDS check every work unit a kernel is about to
+// read or write: its index must lie in the range [lo, hi) the CTA is
+// working on and in [0, n), the extent of the buffers in those units.  A
+// unit outside is skipped (not read, not written) and counted in
+// g_tf4_bounds, which tf4_debug_bounds_violations reads and clears.  In
+// other builds the check is the constant true and compiles away.
+__device__ unsigned long long g_tf4_bounds;
+
+__device__ __forceinline__ bool unit_ok(int64_t i, int64_t lo, int64_t hi, int64_t n) {
+#ifdef TF4_DEBUG_BOUNDS
+  if (i >= lo && i < hi && i >= 0 && i < n) return true;
+  atomicAdd(&g_tf4_bounds, 1ull);
+  return false;
+#else
+  (void)i; (void)lo; (void)hi; (void)n;
+  return true;
+#endif
+}
+
 // ---------------------------------------------------------- small helpers
 __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
   uint32_t d;
@@ -490,7 +510,8 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, 
     for (; c + 7 * kThreads < c1; c += 8 * kThreads) {
       uint4 v[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = __ldg(xs + c + u * kThreads);
+      for (int u = 0; u < 8; ++u)
+        v[u] = unit_ok(c + u * kThreads, c0, c1, 2 * nblocks) ? __ldg(xs + c + u * kThreads) : make_uint4(0u, 0u, 0u, 0u);
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         m = vmax_u16x2(m, v[u].x & 0x7FFF7FFFu);
@@ -500,7 +521,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, 
       }
     }
     for (; c < c1; c += kThreads) {
-      const uint4 v = __ldg(xs + c);
+      const uint4 v = unit_ok(c, c0, c1, 2 * nblocks) ? __ldg(xs + c) : make_uint4(0u, 0u, 0u, 0u);
       m = vmax_u16x2(m, v.x & 0x7FFF7FFFu);
       m = vmax_u16x2(m, v.y & 0x7FFF7FFFu);
       m = vmax_u16x2(m, v.z & 0x7FFF7FFFu);
@@ -514,7 +535,7 @@ __global__ void __launch_bounds__(kThreads) k_amax(const uint4* __restrict__ x, 
       uint32_t t = red[0];
 #pragma unroll
       for (int w = 1; w < kThreads / 32; ++w) t = max(t, red[w]);
-      atomicMax(ws + s, t << 16);
+      if (unit_ok(s, 0, seg.count(), seg.count())) atomicMax(ws + s, t << 16);
     }
     __syncthreads();
     lo = hi;
@@ -892,7 +913,7 @@ __global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant
         for (int u = 0; u < U; ++u) {
           const int64_t k = j + u * kThreads + tid;
           blk[u] = hi - 1 - k;
-          if (k < n) {
+          if (k < n && unit_ok(blk[u], lo, hi, a.nblocks)) {
             const uint4 p = __ldg(xs + 2 * blk[u]), q = __ldg(xs + 2 * blk[u] + 1);
             w[u][0] = p.x; w[u][1] = p.y; w[u][2] = p.z; w[u][3] = p.w;
             w[u][4] = q.x; w[u][5] = q.y; w[u][6] = q.z; w[u][7] = q.w;
@@ -902,7 +923,7 @@ __global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant
         for (int u = 0; u < U; ++u) {
           const bool valid = j + u * kThreads + tid < n;
           bool bad = false;
-          if (valid) {
+          if (valid && unit_ok(blk[u], lo, hi, a.nblocks)) {
             uint32_t c0, c1, sc;
             if (tb.rz)
               nvfp4_block<UG, MODE, true>(w[u], st, tb, blk[u], pk.ks, c0, c1, sc, bad);
@@ -923,7 +944,7 @@ __global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant
         for (int u = 0; u < U; ++u) {
           const int64_t k = j + u * kThreads + tid;
           blk[u] = hi - 1 - k;
-          if (k < n) {
+          if (k < n && unit_ok(blk[u], lo, hi, a.nblocks)) {
 #pragma unroll
             for (int q = 0; q < 4; ++q) {
               const uint4 p = __ldg(xs + 4 * blk[u] + q);
@@ -935,7 +956,7 @@ __global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant
         for (int u = 0; u < U; ++u) {
           const bool valid = j + u * kThreads + tid < n;
           bool bad = false;
-          if (valid) {
+          if (valid && unit_ok(blk[u], lo, hi, a.nblocks)) {
             uint32_t c[4], sc;
             mxfp4_block<MODE>(w[u], blk[u], pk.ks, c, sc, bad);
             reinterpret_cast<uint4*>(a.codes)[blk[u]] = make_uint4(c[0], c[1], c[2], c[3]);
@@ -1031,7 +1052,7 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t k = j + u * kThreads + tid;
-        if (k < n) {
+        if (k < n && unit_ok(lo + k, lo, hi, a.nblocks)) {
           const int64_t blk = lo + k;
 #pragma unroll
           for (int q = 0; q < NW / 4; ++q) {
@@ -1047,7 +1068,7 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
       for (int u = 0; u < U; ++u) {
         const int64_t k = j + u * kThreads + tid;
         bool bad = false;
-        if (k < n) {
+        if (k < n && unit_ok(lo + k, lo, hi, a.nblocks)) {
           const int64_t blk = lo + k;
           const uint32_t mb = block_absmax_bits(w[u]);
           bad = mb >= 0x7F80u;
@@ -1150,7 +1171,7 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t o = ob + u * kThreads + tid;
-        if (o < o1) {
+        if (o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB)) {
           xv[u] = __ldg(a.x + o);
           sc[u] = __ldg(a.rec_scales + o / OPB);
           g[u] = __ldg(a.rec_bits + o);
@@ -1160,7 +1181,7 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
       for (int u = 0; u < U; ++u) {
         const int64_t o = ob + u * kThreads + tid;
         bool bad = false;
-        if (o < o1) {
+        if (o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB)) {
           const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
           const uint32_t mb = block_absmax_bits(w);
           bad = mb >= 0x7F80u;
@@ -1285,6 +1306,7 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
       build_tables<UG, false>(st, tcw);
     }
     for (int64_t blk = lo + threadIdx.x; blk < hi; blk += kThreads) {
+      if (!unit_ok(blk, lo, hi, a.nblocks)) continue;
       uint32_t w[NW], cw[NQ];
 #pragma unroll
       for (int q = 0; q < NW / 4; ++q) {
@@ -1404,7 +1426,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t q = qb + u * kThreads + tid;
-        if (q < q1) {
+        if (q < q1 && unit_ok(q, q0, q1, a.nblocks * QPB)) {
           cw[u] = __ldg(codes2 + q);
           sc[u] = __ldg(a.scales + q / QPB);
         }
@@ -1412,7 +1434,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant(DequantArgs a, SEG seg) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t q = qb + u * kThreads + tid;
-        if (q < q1) {
+        if (q < q1 && unit_ok(q, q0, q1, a.nblocks * QPB)) {
           float S;
           if constexpr (kE4M3<FMT>) S = __fmul_rn(st, e4m3_decode(sc[u]));
           else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
@@ -1449,7 +1471,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant8(DequantArgs a, SEG seg) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t o = ob + u * kThreads + tid;
-        if (o < o1) {
+        if (o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB)) {
           cw[u] = __ldg(codes4 + o);
           sc[u] = __ldg(a.scales + o / OPB);
         }
@@ -1457,7 +1479,7 @@ __global__ void __launch_bounds__(kThreads) k_dequant8(DequantArgs a, SEG seg) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int64_t o = ob + u * kThreads + tid;
-        if (o < o1) {
+        if (o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB)) {
           float S;
           if constexpr (kE4M3<FMT>) S = __fmul_rn(st, e4m3_decode(sc[u]));
           else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
@@ -1484,12 +1506,12 @@ __global__ void __launch_bounds__(kThreads) k_pack(const uint8_t* __restrict__ c
 #pragma unroll
     for (int k = 0; k < U; ++k) {
       const int64_t u = ub + k * kThreads + threadIdx.x;
-      if (u < u1) c[k] = __ldg(c4 + u);
+      if (u < u1 && unit_ok(u, u0, u1, nunits)) c[k] = __ldg(c4 + u);
     }
 #pragma unroll
     for (int k = 0; k < U; ++k) {
       const int64_t u = ub + k * kThreads + threadIdx.x;
-      if (u < u1)
+      if (u < u1 && unit_ok(u, u0, u1, nunits))
         reinterpret_cast<uint32_t*>(bits)[u] = nibble_lsbs(c[k].x) | (nibble_lsbs(c[k].y) << 8) |
                                                (nibble_lsbs(c[k].z) << 16) | (nibble_lsbs(c[k].w) << 24);
     }
@@ -1526,12 +1548,12 @@ __global__ void __launch_bounds__(kThreads) k_unpack(const uint8_t* __restrict__
 #pragma unroll
     for (int k = 0; k < U; ++k) {
       const int64_t u = ub + k * kThreads + threadIdx.x;
-      if (u < u1) b[k] = __ldg(b2 + u);
+      if (u < u1 && unit_ok(u, u0, u1, nunits)) b[k] = __ldg(b2 + u);
     }
 #pragma unroll
     for (int k = 0; k < U; ++k) {
       const int64_t u = ub + k * kThreads + threadIdx.x;
-      if (u < u1) {
+      if (u < u1 && unit_ok(u, u0, u1, nunits)) {
         const uint2 lo = spread8(b[k] & 0xFFu), hi = spread8(b[k] >> 8);
         out[u] = make_uint4(lo.x, lo.y, hi.x, hi.y);
       }
@@ -1560,10 +1582,11 @@ __global__ void __launch_bounds__(kThreads) k_swizzle(const uint8_t* __restrict_
       uint32_t v = 0u;
 #pragma unroll
       for (int c = 0; c < 4; ++c)
-        if (r < rows && c0 + c < nb) v |= (uint32_t)__ldg(scales + r * nb + c0 + c) << (8 * c);
+        if (r < rows && c0 + c < nb && unit_ok(r * nb + c0 + c, 0, rows * nb, rows * nb))
+          v |= (uint32_t)__ldg(scales + r * nb + c0 + c) << (8 * c);
       word[j] = v;
     }
-    out[l] = make_uint4(word[0], word[1], word[2], word[3]);
+    if (unit_ok(l, 0, nlines, nlines)) out[l] = make_uint4(word[0], word[1], word[2], word[3]);
   }
 }
 

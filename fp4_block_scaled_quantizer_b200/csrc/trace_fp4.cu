@@ -701,4 +701,24 @@ const char* tf4_status_string(tf4_status s) {
 
 int tf4_version(void) { return 1; }
 
+int tf4_debug_bounds_enabled(void) {
+#ifdef TF4_DEBUG_BOUNDS
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+tf4_status tf4_debug_bounds_violations(uint64_t* count, tf4_stream_t stream) {
+  if (!count) return TF4_ERR_INVALID_ARG;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) return TF4_ERR_CUDA;
+  unsigned long long v = 0ull;
+  if (cudaMemcpyFromSymbol(&v, tf4::g_tf4_bounds, sizeof v) != cudaSuccess) return TF4_ERR_CUDA;
+  const unsigned long long zero = 0ull;
+  if (cudaMemcpyToSymbol(tf4::g_tf4_bounds, &zero, sizeof zero) != cudaSuccess) return TF4_ERR_CUDA;
+  *count = (uint64_t)v;
+  return TF4_OK;
+}
+
 }  // extern "C"

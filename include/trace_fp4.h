@@ -284,6 +284,21 @@ tf4_status tf4_read_status(int32_t* dev_status, tf4_stream_t stream);
 const char* tf4_status_string(tf4_status status);
 int tf4_version(void);
 
+/* Debug bounds checking (a build option, not part of the method).  A library
+ * built with TF4_DEBUG_BOUNDS (python -m fp4_block_scaled_quantizer_b200.build
+ * --debug-bounds, which writes libtrace_fp4_debug.so) checks in every kernel
+ * that each work unit it reads or writes lies inside the range its CTA owns
+ * and inside the buffers' extent; a unit outside is skipped and counted in a
+ * library-wide device counter instead of being accessed (no trap).
+ *   tf4_debug_bounds_enabled: 1 for such a build, 0 otherwise.
+ *   tf4_debug_bounds_violations: synchronizes `stream`, writes the number of
+ *     skipped units counted since the last call (on the current device) to
+ *     *count (host pointer) and resets the counter; always 0 in a build
+ *     without the checks.  Returns TF4_OK, TF4_ERR_INVALID_ARG (count NULL)
+ *     or TF4_ERR_CUDA. */
+int tf4_debug_bounds_enabled(void);
+tf4_status tf4_debug_bounds_violations(uint64_t* count, tf4_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

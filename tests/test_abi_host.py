@@ -184,3 +184,13 @@ def test_binding_rejects_bad_tensors_before_the_library():
         B.tf4_quantize_capture_batched([])
     with pytest.raises(ValueError):
         B.tf4_pack_guidance(torch.zeros(8, dtype=torch.uint8), 1, 16)
+
+
+def test_debug_bounds_entry_points(L):
+    """The release library reports no bounds checking; the checked build
+    (if present) reports it; a NULL count is refused before any CUDA call."""
+    assert L.tf4_debug_bounds_enabled() == 0
+    assert L.tf4_debug_bounds_violations(None, None) == 1
+    if os.path.exists(B.DEBUG_LIB_PATH):
+        D = ctypes.CDLL(B.DEBUG_LIB_PATH)
+        assert D.tf4_debug_bounds_enabled() == 1
