@@ -499,6 +499,39 @@ def test_nonfinite_reported():
     assert B.read_status(xb.device) == 5
 
 
+@pytest.mark.parametrize("fmt", FMTS)
+@pytest.mark.parametrize("bad", [0x7F80, 0xFF80, 0x7FC1])  # +Inf, -Inf, NaN
+def test_nonfinite_reported_by_every_call(fmt, bad):
+    """Every call that reads bf16 values reports a non-finite input in the
+    status word (and the word clears on reading); the same calls on the
+    clean tensor report nothing."""
+    rows, cols = 48, 256
+    clean = W.random_bf16((rows, cols), seed=41, device=DEV)
+    xb = W.bf16_bits(clean)
+    xb[31, 77] = bad
+    dirty = W.from_bits(xb, DEV)
+    q = B.tf4_quantize_capture(clean, fmt=fmt)
+    assert B.read_status(clean.device) == 0
+    calls = {
+        "capture": lambda x: B.tf4_quantize_capture(x, fmt=fmt),
+        "rtn": lambda x: B.tf4_quantize_rtn(x, fmt=fmt),
+        "sr": lambda x: B.tf4_quantize_sr(x, 3, fmt=fmt),
+        "guided": lambda x: B.tf4_quantize_guided(x, q),
+        "fake_quant": lambda x: B.tf4_guided_fake_quant(x, q),
+        "fake_quant_bf16": lambda x: B.tf4_guided_fake_quant(x, q, out_dtype=torch.bfloat16),
+        "mismatch": lambda x: B.tf4_mismatch_stats(x, q),
+        "batched": lambda x: B.tf4_quantize_capture_batched([clean, x], fmt=fmt, keep=1),
+    }
+    if O.HAS_TENSOR_SCALE[fmt]:
+        calls["amax"] = lambda x: B.tf4_segment_amax(x)
+    for name, call in calls.items():
+        call(clean)
+        assert B.read_status(clean.device) == 0, name
+        call(dirty)
+        assert B.read_status(clean.device) == 5, name
+        assert B.read_status(clean.device) == 0, name
+
+
 def test_empty_tensor():
     xb = torch.zeros((0, 64), dtype=torch.bfloat16, device=DEV)
     q = B.tf4_quantize_capture(xb, seg_off=[0, 0, 0])
