@@ -29,12 +29,12 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _noalloc_capture(L, x, seg, with_bits=True):
+def _noalloc_capture(L, x, seg, with_bits=True, fmt=B.NVFP4):
     rows, cols = x.shape
-    d = B.Desc(B.NVFP4, rows, cols, seg)
+    d = B.Desc(fmt, rows, cols, seg)
     codes = torch.empty(rows * cols // 2, dtype=torch.uint8, device=x.device)
-    scales = torch.empty((rows, cols // 16), dtype=torch.uint8, device=x.device)
-    s_t = torch.empty(d.num_segments, dtype=torch.float32, device=x.device)
+    scales = torch.empty((rows, cols // B.BLOCK[fmt]), dtype=torch.uint8, device=x.device)
+    s_t = torch.empty(d.num_segments, dtype=torch.float32, device=x.device) if B.HAS_TENSOR_SCALE[fmt] else None
     bits = torch.empty(rows * cols // 8, dtype=torch.uint8, device=x.device) if with_bits else None
     stream = ctypes.c_void_p(torch.cuda.current_stream(x.device).cuda_stream)
     st = L.tf4_quantize_capture_noalloc(d.ptr, _p(x), _p(codes), _p(scales), _p(s_t), _p(bits),
@@ -42,7 +42,8 @@ def _noalloc_capture(L, x, seg, with_bits=True):
     return st, codes, scales, s_t, bits
 
 
-def test_noalloc_capture_matches_workspace_capture():
+@pytest.mark.parametrize("fmt", [B.NVFP4, B.UFP4, B.MXFP4])
+def test_noalloc_capture_matches_workspace_capture(fmt):
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     libbuild.build()
@@ -52,14 +53,17 @@ def test_noalloc_capture_matches_workspace_capture():
         ((257, 2048), None),                 # one segment, several CTAs
     ]
     for call, ((rows, cols), seg) in enumerate(cases):
+        if seg is not None and not B.HAS_TENSOR_SCALE[fmt]:
+            continue  # MXFP4 has no tensor scale, hence no segments
         x = W.random_bf16((rows, cols), seed=100 + call, device="cuda", outlier_frac=0.01)
-        ref = B.tf4_quantize_capture(x, seg_off=seg)
-        st, codes, scales, s_t, bits = _noalloc_capture(L, x, seg)
+        ref = B.tf4_quantize_capture(x, fmt=fmt, seg_off=seg)
+        st, codes, scales, s_t, bits = _noalloc_capture(L, x, seg, fmt=fmt)
         assert st == 0, B.STATUS.get(st, st)
         assert B.read_status(x.device) == 0
         assert torch.equal(codes, ref.codes)
-        assert torch.equal(scales, ref.scales)
-        assert torch.equal(s_t.view(torch.int32), ref.s_t.view(torch.int32))
+        assert torch.equal(scales.view(-1), ref.scales.view(-1))
+        if B.HAS_TENSOR_SCALE[fmt]:
+            assert torch.equal(s_t.view(torch.int32), ref.s_t.view(torch.int32))
         assert torch.equal(bits, ref.bits)
 
 
