@@ -41,12 +41,12 @@ STATUS = {
 
 # symbols declared in include/trace_fp4.h
 EXPORTS = (
-    "tf4_workspace_bytes", "tf4_codes_bytes", "tf4_scales_bytes", "tf4_guidance_bytes",
-    "tf4_record_bytes", "tf4_segment_amax", "tf4_quantize_rtn", "tf4_quantize_sr",
-    "tf4_quantize_capture", "tf4_quantize_guided", "tf4_dequantize", "tf4_pack_guidance",
-    "tf4_unpack_guidance", "tf4_guided_fake_quant", "tf4_mismatch_stats", "tf4_workspace_bytes_batched",
-    "tf4_quantize_capture_batched", "tf4_blocked_scales_bytes", "tf4_swizzle_scales", "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string",
-    "tf4_version", "tf4_debug_bounds_enabled", "tf4_debug_bounds_violations",
+    "tf4_workspace_bytes", "tf4_codes_bytes", "tf4_scales_bytes", "tf4_guidance_bytes", "tf4_record_bytes",
+    "tf4_segment_amax", "tf4_quantize_rtn", "tf4_quantize_sr", "tf4_quantize_capture", "tf4_quantize_guided",
+    "tf4_dequantize", "tf4_pack_guidance", "tf4_unpack_guidance", "tf4_guided_fake_quant", "tf4_mismatch_stats",
+    "tf4_workspace_bytes_batched", "tf4_quantize_capture_batched", "tf4_blocked_scales_bytes", "tf4_swizzle_scales",
+    "tf4_quantize_capture_noalloc", "tf4_read_status", "tf4_status_string", "tf4_version",
+    "tf4_debug_bounds_enabled", "tf4_debug_bounds_violations",
 )
 
 
