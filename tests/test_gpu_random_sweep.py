@@ -50,7 +50,7 @@ def random_values(rng, rows, cols):
     return torch.from_numpy(v.astype(np.float32)).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("case", range(48))
+@pytest.mark.parametrize("case", range(160))
 def test_random_case(case):
     rng = np.random.default_rng(1000 + case)
     fmt = int(rng.choice([O.NVFP4, O.MXFP4, O.UFP4]))
