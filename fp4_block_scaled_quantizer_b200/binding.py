@@ -215,6 +215,19 @@ _ws_cache: dict = {}
 _status_cache: dict = {}
 
 
+def _on(stream):
+    """Context in which torch allocates and fills on `stream` (the stream
+    the library call will launch on), so that a new output, workspace or
+    status word is ordered before the call's kernels; no-op for None (the
+    current stream)."""
+    return torch.cuda.stream(stream) if stream is not None else contextlib.nullcontext()
+
+
+def _stream_key(device, stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return (torch.device(device).index, s.cuda_stream), s
+
+
 def workspace(desc: Desc, device, stream=None) -> torch.Tensor:
     """A zero-filled workspace for this device/stream (reused: every call
     returns it to zero when it completes)."""
@@ -222,20 +235,25 @@ def workspace(desc: Desc, device, stream=None) -> torch.Tensor:
 
 
 def _workspace_bytes(need: int, device, stream=None) -> torch.Tensor:
-    s = stream if stream is not None else torch.cuda.current_stream(device)
-    key = (torch.device(device).index, s.cuda_stream)
+    key, s = _stream_key(device, stream)
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < need:
-        ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=device)
+        with torch.cuda.stream(s):  # zero-filled on the stream that will use it
+            ws = torch.zeros(max(need, 256), dtype=torch.uint8, device=device)
         _ws_cache[key] = ws
     return ws
 
 
-def status_word(device) -> torch.Tensor:
-    key = torch.device(device).index
+def status_word(device, stream=None) -> torch.Tensor:
+    """The device status word the library's calls on (device, stream) OR
+    their data-dependent errors into: one per stream, so that reading it
+    (read_status synchronizes that stream only) never races with kernels
+    still running on another stream."""
+    key, s = _stream_key(device, stream)
     t = _status_cache.get(key)
     if t is None:
-        t = torch.zeros(1, dtype=torch.int32, device=device)
+        with torch.cuda.stream(s):
+            t = torch.zeros(1, dtype=torch.int32, device=device)
         _status_cache[key] = t
     return t
 
@@ -266,8 +284,9 @@ def debug_bounds_violations(device=None, stream=None) -> int:
 
 
 def read_status(device, stream=None) -> int:
-    """Synchronize and return (and clear) the device status code."""
-    t = status_word(device)
+    """Synchronize `stream` (default: the current stream) and return (and
+    clear) the status code of the calls issued on it."""
+    t = status_word(device, stream)
     return int(lib().tf4_read_status(_ptr(t), _stream(stream, t.device)))
 
 
@@ -317,54 +336,60 @@ def _amax_in(amax_in, desc: Desc, device):
 
 
 def tf4_segment_amax(x: torch.Tensor, seg_off=None, stream=None, out=None) -> torch.Tensor:
-    x2 = _as_2d(x)
-    d = Desc(NVFP4, x2.shape[0], x2.shape[1], seg_off)
-    amax = (_buf(out, "out", d.num_segments, torch.float32, x.device) if out is not None
-            else torch.empty(d.num_segments, dtype=torch.float32, device=x.device))
-    ws = workspace(d, x.device, stream)
-    _check(lib().tf4_segment_amax(d.ptr, _ptr(x2), _ptr(amax), _ptr(ws), ws.numel(),
-                                  _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_segment_amax")
-    return amax
+    with _on(stream):
+        x2 = _as_2d(x)
+        d = Desc(NVFP4, x2.shape[0], x2.shape[1], seg_off)
+        amax = (_buf(out, "out", d.num_segments, torch.float32, x.device) if out is not None
+                else torch.empty(d.num_segments, dtype=torch.float32, device=x.device))
+        ws = workspace(d, x.device, stream)
+        _check(lib().tf4_segment_amax(d.ptr, _ptr(x2), _ptr(amax), _ptr(ws), ws.numel(),
+                                      _ptr(status_word(x.device, stream)), _stream(stream, x.device)),
+               "tf4_segment_amax")
+        return amax
 
 
 def tf4_quantize_rtn(x, fmt=NVFP4, seg_off=None, amax_in=None, stream=None, out=None) -> Quantized:
-    x2 = _as_2d(x)
-    d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
-    q = _outputs(d, x.device, False, out)
-    _amax_in(amax_in, d, x.device)
-    ws = workspace(d, x.device, stream)
-    _check(lib().tf4_quantize_rtn(d.ptr, _ptr(x2), _ptr(amax_in), _ptr(q.codes), _ptr(q.scales), _ptr(q.s_t),
-                                  _ptr(ws), ws.numel(), _ptr(status_word(x.device)), _stream(stream, x.device)),
-           "tf4_quantize_rtn")
-    return q
+    with _on(stream):
+        x2 = _as_2d(x)
+        d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
+        q = _outputs(d, x.device, False, out)
+        _amax_in(amax_in, d, x.device)
+        ws = workspace(d, x.device, stream)
+        _check(lib().tf4_quantize_rtn(d.ptr, _ptr(x2), _ptr(amax_in), _ptr(q.codes), _ptr(q.scales), _ptr(q.s_t),
+                                      _ptr(ws), ws.numel(), _ptr(status_word(x.device, stream)),
+                                      _stream(stream, x.device)),
+               "tf4_quantize_rtn")
+        return q
 
 
 def tf4_quantize_sr(x, seed: int, fmt=NVFP4, seg_off=None, amax_in=None, stream=None, out=None) -> Quantized:
-    x2 = _as_2d(x)
-    d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
-    q = _outputs(d, x.device, False, out)
-    _amax_in(amax_in, d, x.device)
-    ws = workspace(d, x.device, stream)
-    _check(lib().tf4_quantize_sr(d.ptr, _ptr(x2), ctypes.c_uint64(seed & (2**64 - 1)), _ptr(amax_in),
-                                 _ptr(q.codes), _ptr(q.scales), _ptr(q.s_t), _ptr(ws), ws.numel(),
-                                 _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_quantize_sr")
-    return q
+    with _on(stream):
+        x2 = _as_2d(x)
+        d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
+        q = _outputs(d, x.device, False, out)
+        _amax_in(amax_in, d, x.device)
+        ws = workspace(d, x.device, stream)
+        _check(lib().tf4_quantize_sr(d.ptr, _ptr(x2), ctypes.c_uint64(seed & (2**64 - 1)), _ptr(amax_in),
+                                     _ptr(q.codes), _ptr(q.scales), _ptr(q.s_t), _ptr(ws), ws.numel(),
+                                     _ptr(status_word(x.device, stream)), _stream(stream, x.device)), "tf4_quantize_sr")
+        return q
 
 
 def tf4_quantize_capture(x, fmt=NVFP4, seg_off=None, guidance=True, amax_in=None, stream=None,
                          out=None) -> Quantized:
     """Rollout-side capture; ``guidance=False`` for layers whose guidance is
     not kept (codes/scales/s_t are then those of round-to-nearest)."""
-    x2 = _as_2d(x)
-    d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
-    q = _outputs(d, x.device, guidance, out)
-    _amax_in(amax_in, d, x.device)
-    ws = workspace(d, x.device, stream)
-    _check(lib().tf4_quantize_capture(d.ptr, _ptr(x2), _ptr(amax_in), _ptr(q.codes), _ptr(q.scales),
-                                      _ptr(q.s_t), _ptr(q.bits if guidance else None), _ptr(ws), ws.numel(),
-                                      _ptr(status_word(x.device)), _stream(stream, x.device)),
-           "tf4_quantize_capture")
-    return q
+    with _on(stream):
+        x2 = _as_2d(x)
+        d = Desc(fmt, x2.shape[0], x2.shape[1], seg_off)
+        q = _outputs(d, x.device, guidance, out)
+        _amax_in(amax_in, d, x.device)
+        ws = workspace(d, x.device, stream)
+        _check(lib().tf4_quantize_capture(d.ptr, _ptr(x2), _ptr(amax_in), _ptr(q.codes), _ptr(q.scales),
+                                          _ptr(q.s_t), _ptr(q.bits if guidance else None), _ptr(ws), ws.numel(),
+                                          _ptr(status_word(x.device, stream)), _stream(stream, x.device)),
+               "tf4_quantize_capture")
+        return q
 
 
 @dataclass
@@ -389,54 +414,57 @@ class BatchedCapture:
 def tf4_quantize_capture_batched(xs, fmt=NVFP4, keep=0, stream=None, out: Optional[BatchedCapture] = None):
     """Capture a list of same-shaped bf16 tensors (layers) in two launches;
     guidance is kept for the last `keep` layers, in one contiguous buffer."""
-    L = len(xs)
-    if L == 0:
-        raise ValueError("tf4_quantize_capture_batched: no layers")
-    x2 = [_as_2d(x) for x in xs]
-    rows, cols = x2[0].shape
-    dev = x2[0].device
-    if any(t.shape != (rows, cols) or t.device != dev for t in x2):
-        raise ValueError("tf4_quantize_capture_batched: layers must share one shape and one device")
-    if not 0 <= keep <= L:
-        raise ValueError(f"tf4_quantize_capture_batched: keep={keep} outside [0, {L}]")
-    d = Desc(fmt, rows, cols)
-    if out is not None:
-        n = rows * cols
-        _buf(out.codes, "out.codes", L * (n // 2), torch.uint8, dev)
-        _buf(out.scales, "out.scales", L * (n // BLOCK[fmt]), torch.uint8, dev)
-        if HAS_TENSOR_SCALE[fmt]:
-            _buf(out.s_t, "out.s_t", L, torch.float32, dev)
-        if keep:
-            _buf(out.info_bits, "out.info_bits", keep * (n // 8), torch.uint8, dev)
-    else:
-        n = rows * cols
-        out = BatchedCapture(torch.empty((L, n // 2), dtype=torch.uint8, device=dev),
-                             torch.empty((L, rows, cols // BLOCK[fmt]), dtype=torch.uint8, device=dev),
-                             torch.empty(L, dtype=torch.float32, device=dev) if HAS_TENSOR_SCALE[fmt] else None,
-                             torch.empty((keep, n // 8), dtype=torch.uint8, device=dev) if keep else None,
-                             fmt, rows, cols, keep)
-    ptrs = (ctypes.c_void_p * L)(*[t.data_ptr() for t in x2])
-    ws = _workspace_bytes(lib().tf4_workspace_bytes_batched(L), dev, stream)
-    _check(lib().tf4_quantize_capture_batched(d.ptr, L, ptrs, _ptr(out.codes), _ptr(out.scales), _ptr(out.s_t),
-                                              keep, _ptr(out.info_bits), _ptr(ws), ws.numel(),
-                                              _ptr(status_word(dev)), _stream(stream, dev)),
-           "tf4_quantize_capture_batched")
-    return out
+    with _on(stream):
+        L = len(xs)
+        if L == 0:
+            raise ValueError("tf4_quantize_capture_batched: no layers")
+        x2 = [_as_2d(x) for x in xs]
+        rows, cols = x2[0].shape
+        dev = x2[0].device
+        if any(t.shape != (rows, cols) or t.device != dev for t in x2):
+            raise ValueError("tf4_quantize_capture_batched: layers must share one shape and one device")
+        if not 0 <= keep <= L:
+            raise ValueError(f"tf4_quantize_capture_batched: keep={keep} outside [0, {L}]")
+        d = Desc(fmt, rows, cols)
+        if out is not None:
+            n = rows * cols
+            _buf(out.codes, "out.codes", L * (n // 2), torch.uint8, dev)
+            _buf(out.scales, "out.scales", L * (n // BLOCK[fmt]), torch.uint8, dev)
+            if HAS_TENSOR_SCALE[fmt]:
+                _buf(out.s_t, "out.s_t", L, torch.float32, dev)
+            if keep:
+                _buf(out.info_bits, "out.info_bits", keep * (n // 8), torch.uint8, dev)
+        else:
+            n = rows * cols
+            out = BatchedCapture(torch.empty((L, n // 2), dtype=torch.uint8, device=dev),
+                                 torch.empty((L, rows, cols // BLOCK[fmt]), dtype=torch.uint8, device=dev),
+                                 torch.empty(L, dtype=torch.float32, device=dev) if HAS_TENSOR_SCALE[fmt] else None,
+                                 torch.empty((keep, n // 8), dtype=torch.uint8, device=dev) if keep else None,
+                                 fmt, rows, cols, keep)
+        ptrs = (ctypes.c_void_p * L)(*[t.data_ptr() for t in x2])
+        ws = _workspace_bytes(lib().tf4_workspace_bytes_batched(L), dev, stream)
+        _check(lib().tf4_quantize_capture_batched(d.ptr, L, ptrs, _ptr(out.codes), _ptr(out.scales), _ptr(out.s_t),
+                                                  keep, _ptr(out.info_bits), _ptr(ws), ws.numel(),
+                                                  _ptr(status_word(dev, stream)), _stream(stream, dev)),
+               "tf4_quantize_capture_batched")
+        return out
 
 
 def tf4_quantize_guided(x, rec: Quantized, stream=None, out=None, rec_bits=None) -> torch.Tensor:
     """Train-side guided quantization of x against a rollout record."""
-    x2 = _as_2d(x)
-    d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
-    bits = rec_bits if rec_bits is not None else rec.bits
-    if bits is None:
-        raise ValueError("tf4_quantize_guided: the record holds no guidance bits")
-    _check_record(rec, d, x.device, "tf4_quantize_guided", bits=bits)
-    codes = (_buf(out, "out", d.n // 2, torch.uint8, x.device) if out is not None
-             else torch.empty(d.n // 2, dtype=torch.uint8, device=x.device))
-    _check(lib().tf4_quantize_guided(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(bits), _ptr(codes),
-                                     _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_quantize_guided")
-    return codes
+    with _on(stream):
+        x2 = _as_2d(x)
+        d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
+        bits = rec_bits if rec_bits is not None else rec.bits
+        if bits is None:
+            raise ValueError("tf4_quantize_guided: the record holds no guidance bits")
+        _check_record(rec, d, x.device, "tf4_quantize_guided", bits=bits)
+        codes = (_buf(out, "out", d.n // 2, torch.uint8, x.device) if out is not None
+                 else torch.empty(d.n // 2, dtype=torch.uint8, device=x.device))
+        _check(lib().tf4_quantize_guided(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(bits), _ptr(codes),
+                                         _ptr(status_word(x.device, stream)), _stream(stream, x.device)),
+               "tf4_quantize_guided")
+        return codes
 
 
 def tf4_guided_fake_quant(x, rec: Quantized, out_dtype=torch.float32, want_codes=False, stream=None,
@@ -444,98 +472,105 @@ def tf4_guided_fake_quant(x, rec: Quantized, out_dtype=torch.float32, want_codes
     """Guided quantization + dequantization in one pass.  Returns (values,
     codes): values [rows, cols] in out_dtype (float32, or bfloat16 = RNE of
     the fp32 value); codes only if want_codes (else None)."""
-    if out_dtype not in (torch.float32, torch.bfloat16):
-        raise TypeError(f"tf4_guided_fake_quant: out_dtype must be float32 or bfloat16, got {out_dtype}")
-    x2 = _as_2d(x)
-    d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
-    bits = rec_bits if rec_bits is not None else rec.bits
-    if bits is None:
-        raise ValueError("tf4_guided_fake_quant: the record holds no guidance bits")
-    _check_record(rec, d, x.device, "tf4_guided_fake_quant", bits=bits)
-    if out is not None:
-        if not isinstance(out, torch.Tensor) or out.dtype not in (torch.float32, torch.bfloat16):
-            raise TypeError("tf4_guided_fake_quant: out must be a float32 or bfloat16 tensor")
-        o = _buf(out, "out", d.n, out.dtype, x.device)
-    else:
-        o = torch.empty(x2.shape, dtype=out_dtype, device=x.device)
-    if codes is not None:
-        c = _buf(codes, "codes", d.n // 2, torch.uint8, x.device)
-    else:
-        c = torch.empty(d.n // 2, dtype=torch.uint8, device=x.device) if want_codes else None
-    _check(lib().tf4_guided_fake_quant(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(bits), _ptr(c),
-                                       _ptr(o), 1 if o.dtype == torch.bfloat16 else 0,
-                                       _ptr(status_word(x.device)), _stream(stream, x.device)),
-           "tf4_guided_fake_quant")
-    return o, c
+    with _on(stream):
+        if out_dtype not in (torch.float32, torch.bfloat16):
+            raise TypeError(f"tf4_guided_fake_quant: out_dtype must be float32 or bfloat16, got {out_dtype}")
+        x2 = _as_2d(x)
+        d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
+        bits = rec_bits if rec_bits is not None else rec.bits
+        if bits is None:
+            raise ValueError("tf4_guided_fake_quant: the record holds no guidance bits")
+        _check_record(rec, d, x.device, "tf4_guided_fake_quant", bits=bits)
+        if out is not None:
+            if not isinstance(out, torch.Tensor) or out.dtype not in (torch.float32, torch.bfloat16):
+                raise TypeError("tf4_guided_fake_quant: out must be a float32 or bfloat16 tensor")
+            o = _buf(out, "out", d.n, out.dtype, x.device)
+        else:
+            o = torch.empty(x2.shape, dtype=out_dtype, device=x.device)
+        if codes is not None:
+            c = _buf(codes, "codes", d.n // 2, torch.uint8, x.device)
+        else:
+            c = torch.empty(d.n // 2, dtype=torch.uint8, device=x.device) if want_codes else None
+        _check(lib().tf4_guided_fake_quant(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(bits), _ptr(c),
+                                           _ptr(o), 1 if o.dtype == torch.bfloat16 else 0,
+                                           _ptr(status_word(x.device, stream)), _stream(stream, x.device)),
+               "tf4_guided_fake_quant")
+        return o, c
 
 
 def tf4_mismatch_stats(x, rec: Quantized, counts=None, stream=None) -> torch.Tensor:
     """Mismatch diagnostics of train values x against a rollout record
     (codes + scales): adds [#mismatch, #adjacent, #far, #after-guidance] to
     `counts` (int64 [4], zero-initialised if not given) and returns it."""
-    x2 = _as_2d(x)
-    d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
-    _check_record(rec, d, x.device, "tf4_mismatch_stats", codes=True)
-    c = (_buf(counts, "counts", 4, torch.int64, x.device) if counts is not None
-         else torch.zeros(4, dtype=torch.int64, device=x.device))
-    _check(lib().tf4_mismatch_stats(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(rec.codes), _ptr(c),
-                                    _ptr(status_word(x.device)), _stream(stream, x.device)), "tf4_mismatch_stats")
-    return c
+    with _on(stream):
+        x2 = _as_2d(x)
+        d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
+        _check_record(rec, d, x.device, "tf4_mismatch_stats", codes=True)
+        c = (_buf(counts, "counts", 4, torch.int64, x.device) if counts is not None
+             else torch.zeros(4, dtype=torch.int64, device=x.device))
+        _check(lib().tf4_mismatch_stats(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(rec.codes), _ptr(c),
+                                        _ptr(status_word(x.device, stream)), _stream(stream, x.device)),
+               "tf4_mismatch_stats")
+        return c
 
 
 def tf4_dequantize(q: Quantized, codes=None, stream=None, out=None) -> torch.Tensor:
-    d = Desc(q.fmt, q.rows, q.cols, q.seg_off)
-    c = codes if codes is not None else q.codes
-    if not isinstance(c, torch.Tensor) or not c.is_cuda:
-        raise ValueError("tf4_dequantize: codes must be a CUDA tensor")
-    _buf(c, "codes", d.n // 2, torch.uint8, c.device)
-    _check_record(q, d, c.device, "tf4_dequantize")
-    o = (_buf(out, "out", d.n, torch.float32, c.device) if out is not None
-         else torch.empty((q.rows, q.cols), dtype=torch.float32, device=c.device))
-    _check(lib().tf4_dequantize(d.ptr, _ptr(c), _ptr(q.scales), _ptr(q.s_t), _ptr(o), _stream(stream, c.device)),
-           "tf4_dequantize")
-    return o
+    with _on(stream):
+        d = Desc(q.fmt, q.rows, q.cols, q.seg_off)
+        c = codes if codes is not None else q.codes
+        if not isinstance(c, torch.Tensor) or not c.is_cuda:
+            raise ValueError("tf4_dequantize: codes must be a CUDA tensor")
+        _buf(c, "codes", d.n // 2, torch.uint8, c.device)
+        _check_record(q, d, c.device, "tf4_dequantize")
+        o = (_buf(out, "out", d.n, torch.float32, c.device) if out is not None
+             else torch.empty((q.rows, q.cols), dtype=torch.float32, device=c.device))
+        _check(lib().tf4_dequantize(d.ptr, _ptr(c), _ptr(q.scales), _ptr(q.s_t), _ptr(o), _stream(stream, c.device)),
+               "tf4_dequantize")
+        return o
 
 
 def tf4_swizzle_scales(q: Quantized, stream=None, out=None) -> torch.Tensor:
     """The record's block scales in the tiled layout block-scaled FP4 GEMMs
     read (uint8 [ceil(rows/128)*128, ceil(nb/4)*4] as laid out in memory)."""
-    d = Desc(q.fmt, q.rows, q.cols, q.seg_off)
-    nb = q.cols // BLOCK[q.fmt]
-    shape = ((q.rows + 127) // 128 * 128, (nb + 3) // 4 * 4)
-    if not isinstance(q.scales, torch.Tensor) or not q.scales.is_cuda:
-        raise ValueError("tf4_swizzle_scales: the record's scales must be a CUDA tensor")
-    dev = q.scales.device
-    _buf(q.scales, "record scales", q.rows * nb, torch.uint8, dev)
-    o = (_buf(out, "out", shape[0] * shape[1], torch.uint8, dev) if out is not None
-         else torch.empty(shape, dtype=torch.uint8, device=dev))
-    _check(lib().tf4_swizzle_scales(d.ptr, _ptr(q.scales), _ptr(o), _stream(stream, q.scales.device)),
-           "tf4_swizzle_scales")
-    return o
+    with _on(stream):
+        d = Desc(q.fmt, q.rows, q.cols, q.seg_off)
+        nb = q.cols // BLOCK[q.fmt]
+        shape = ((q.rows + 127) // 128 * 128, (nb + 3) // 4 * 4)
+        if not isinstance(q.scales, torch.Tensor) or not q.scales.is_cuda:
+            raise ValueError("tf4_swizzle_scales: the record's scales must be a CUDA tensor")
+        dev = q.scales.device
+        _buf(q.scales, "record scales", q.rows * nb, torch.uint8, dev)
+        o = (_buf(out, "out", shape[0] * shape[1], torch.uint8, dev) if out is not None
+             else torch.empty(shape, dtype=torch.uint8, device=dev))
+        _check(lib().tf4_swizzle_scales(d.ptr, _ptr(q.scales), _ptr(o), _stream(stream, q.scales.device)),
+               "tf4_swizzle_scales")
+        return o
 
 
 def tf4_pack_guidance(codes: torch.Tensor, rows: int, cols: int, fmt=NVFP4, stream=None, out=None):
-    d = Desc(fmt, rows, cols)
-    if not isinstance(codes, torch.Tensor) or not codes.is_cuda:
-        raise ValueError("tf4_pack_guidance: codes must be a CUDA tensor")
-    _buf(codes, "codes", d.n // 2, torch.uint8, codes.device)
-    o = (_buf(out, "out", d.n // 8, torch.uint8, codes.device) if out is not None
-         else torch.empty(d.n // 8, dtype=torch.uint8, device=codes.device))
-    _check(lib().tf4_pack_guidance(d.ptr, _ptr(codes), _ptr(o), _stream(stream, codes.device)),
-           "tf4_pack_guidance")
-    return o
+    with _on(stream):
+        d = Desc(fmt, rows, cols)
+        if not isinstance(codes, torch.Tensor) or not codes.is_cuda:
+            raise ValueError("tf4_pack_guidance: codes must be a CUDA tensor")
+        _buf(codes, "codes", d.n // 2, torch.uint8, codes.device)
+        o = (_buf(out, "out", d.n // 8, torch.uint8, codes.device) if out is not None
+             else torch.empty(d.n // 8, dtype=torch.uint8, device=codes.device))
+        _check(lib().tf4_pack_guidance(d.ptr, _ptr(codes), _ptr(o), _stream(stream, codes.device)),
+               "tf4_pack_guidance")
+        return o
 
 
 def tf4_unpack_guidance(bits: torch.Tensor, rows: int, cols: int, fmt=NVFP4, stream=None, out=None):
-    d = Desc(fmt, rows, cols)
-    if not isinstance(bits, torch.Tensor) or not bits.is_cuda:
-        raise ValueError("tf4_unpack_guidance: bits must be a CUDA tensor")
-    _buf(bits, "bits", d.n // 8, torch.uint8, bits.device)
-    o = (_buf(out, "out", d.n, torch.uint8, bits.device) if out is not None
-         else torch.empty(d.n, dtype=torch.uint8, device=bits.device))
-    _check(lib().tf4_unpack_guidance(d.ptr, _ptr(bits), _ptr(o), _stream(stream, bits.device)),
-           "tf4_unpack_guidance")
-    return o
+    with _on(stream):
+        d = Desc(fmt, rows, cols)
+        if not isinstance(bits, torch.Tensor) or not bits.is_cuda:
+            raise ValueError("tf4_unpack_guidance: bits must be a CUDA tensor")
+        _buf(bits, "bits", d.n // 8, torch.uint8, bits.device)
+        o = (_buf(out, "out", d.n, torch.uint8, bits.device) if out is not None
+             else torch.empty(d.n, dtype=torch.uint8, device=bits.device))
+        _check(lib().tf4_unpack_guidance(d.ptr, _ptr(bits), _ptr(o), _stream(stream, bits.device)),
+               "tf4_unpack_guidance")
+        return o
 
 
 def capture_layers(num_layers: int, keep: int) -> list:

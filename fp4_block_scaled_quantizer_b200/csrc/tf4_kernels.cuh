@@ -1005,7 +1005,8 @@ __device__ __forceinline__ uint32_t spread_bits(uint32_t b) {
 // Fix the nibbles of code word c (values in the four bf16-pair words
 // w0..w3) whose m3 & 1 differs from the recorded bit (mm: mismatch bits at
 // nibble bit 0): keep exact codewords and the saturated top, otherwise step
-// to the other neighbour.
+// to the other neighbour.  Zero is decided on x itself: a nonzero x whose
+// product with r underflows to 0 is still above the codeword 0.
 template <bool RZ, bool U = false>
 __device__ __forceinline__ uint32_t fix_mismatches(uint32_t c, uint32_t mm, uint32_t w0, uint32_t w1,
                                                    uint32_t w2, uint32_t w3, float r) {
@@ -1017,8 +1018,9 @@ __device__ __forceinline__ uint32_t fix_mismatches(uint32_t c, uint32_t mm, uint
     const float y = mul<RZ>(__uint_as_float((h & 0x7FFFu) << 16), r);
     const uint32_t n = (c >> (4 * e)) & 7u;
     const float v = grid_value<U>(n);
-    if (!(y == v || (n == 7u && y >= kGridMax<U>))) {
-      const uint32_t n2 = y > v ? n + 1u : n - 1u;
+    const bool exact = n ? (y == v) : ((h & 0x7FFFu) == 0u);
+    if (!(exact || (n == 7u && y >= kGridMax<U>))) {
+      const uint32_t n2 = (n == 0u || y > v) ? n + 1u : n - 1u;
       c = (c & ~(7u << (4 * e))) | (n2 << (4 * e));
     }
   }

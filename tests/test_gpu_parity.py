@@ -312,6 +312,41 @@ def test_guided_near_ties(fmt):
     assert_same("guided", host(g), want)
 
 
+def _large_scale_with_tiny_train_values(fmt, rows=64, cols=1024):
+    """Rollout values of order 2^20 (NVFP4, UFP4) or 2^115 (MXFP4), so that
+    every block scale is large; the train copy replaces a quarter of the
+    elements with zeros and bf16 subnormals of both signs.  A subnormal train
+    value times the block's reciprocal scale underflows fp32 to zero, yet
+    its exact quotient is positive and not a codeword: where the recorded bit
+    is 1 the guided code is the smallest nonzero codeword, never zero."""
+    big = 2.0 ** (115 if fmt == O.MXFP4 else 20)
+    xb = W.random_bf16((rows, cols), seed=91, device=DEV, scale=big)
+    bits = W.bf16_bits(xb).copy().reshape(-1)
+    rng = np.random.default_rng(92)
+    pos = rng.choice(bits.size, bits.size // 4, replace=False)
+    tiny = rng.choice(np.array([0x0000, 0x8000, 0x0001, 0x8001, 0x0003, 0x007F, 0x8040], dtype=np.uint16), pos.size)
+    bits[pos] = tiny
+    return xb, W.from_bits(bits.reshape(rows, cols), DEV)
+
+
+@pytest.mark.parametrize("fmt", FMTS)
+def test_guided_tiny_train_values_under_large_scales(fmt):
+    xb, xt = _large_scale_with_tiny_train_values(fmt)
+    q, r = check_quant(xb, fmt)
+    want, _ = O.quantize_guided(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"])
+    # the case is live: nonzero train subnormals recorded with bit 1 must move off zero
+    assert (O.unpack_codes(want, want.size * 2) & 7).astype(bool).any()
+    assert_same("guided", host(B.tf4_quantize_guided(xt, q)), want)
+    codes, vals, _ = O.guided_fake_quant(W.bf16_bits(xt), r["scales"], r["bits"], fmt, rec_s_t=r["s_t"])
+    y, c = B.tf4_guided_fake_quant(xt, q, want_codes=True)
+    assert_same("fake-quant codes", host(c), codes)
+    assert_same("fake-quant values", f32_bits(host(y)), f32_bits(vals))
+    counts = B.tf4_mismatch_stats(xt, q)
+    assert host(counts).tolist() == O.mismatch_stats(W.bf16_bits(xt), r["scales"], r["codes"], fmt,
+                                                     rec_s_t=r["s_t"]).tolist()
+    assert B.read_status(xb.device) == 0
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_dequant_parity(fmt):
     xb = W.random_bf16((77, 2048), seed=31, device=DEV, outlier_frac=0.01)
@@ -600,8 +635,49 @@ def test_cuda_graph_capture_and_replay():
         for name in ("codes", "scales", "s_t", "bits"):
             assert torch.equal(getattr(q, name), getattr(q2, name)), name
         assert torch.equal(y.view(torch.int16), y2.view(torch.int16))
-    assert B.read_status(x.device) == 0
+    assert B.read_status(x.device) == 0 and B.read_status(x.device, s) == 0
     del g
+
+
+def test_wrappers_on_a_stream_that_is_not_current():
+    """Every wrapper called with stream= a stream other than the current
+    one, while the current stream is still busy: the outputs, the fresh
+    workspace and the status word the call creates are ordered on that
+    stream, so the results equal the oracle's."""
+    rows, cols, seg = 96, 2048, [0, 40, 40, 96]
+    x = W.random_bf16((rows, cols), seed=85, device=DEV, outlier_frac=0.01)
+    xt = W.perturb(x, 86, rel=0.05)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()  # a new stream: new workspace and status-word keys
+    busy = torch.empty(1 << 28, dtype=torch.float32, device=DEV)
+    for _ in range(4):
+        busy.mul_(1.0001)  # ~4 GB of traffic left running on the current stream
+    q = B.tf4_quantize_capture(x, seg_off=seg, stream=s)
+    g = B.tf4_quantize_guided(xt, q, stream=s)
+    d = B.tf4_dequantize(q, stream=s)
+    y, c = B.tf4_guided_fake_quant(xt, q, want_codes=True, stream=s)
+    sr = B.tf4_quantize_sr(x, 2**33 + 5, seg_off=seg, stream=s)
+    am = B.tf4_segment_amax(x, seg_off=seg, stream=s)
+    bits = B.tf4_pack_guidance(q.codes, rows, cols, stream=s)
+    assert B.read_status(x.device, s) == 0
+    torch.cuda.synchronize()
+    xs, xts = W.bf16_bits(x), W.bf16_bits(xt)
+    r = O.quantize(xs, O.NVFP4, O.RTN, seg_off=seg, bits=True)
+    assert_same("codes", host(q.codes), r["codes"])
+    assert_same("s_t", f32_bits(host(q.s_t)), f32_bits(r["s_t"]))
+    assert_same("bits", host(q.bits), r["bits"])
+    assert_same("packed bits", host(bits), r["bits"])
+    rg, _ = O.quantize_guided(xts, r["scales"], r["bits"], O.NVFP4, rec_s_t=r["s_t"], seg_off=seg)
+    assert_same("guided", host(g), rg)
+    assert_same("fake-quant codes", host(c), rg)
+    rd = O.dequantize(r["codes"], r["scales"], rows, cols, O.NVFP4, s_t=r["s_t"], seg_off=seg)
+    assert_same("dequant", f32_bits(host(d)), f32_bits(rd))
+    _, rfq, _ = O.guided_fake_quant(xts, r["scales"], r["bits"], O.NVFP4, rec_s_t=r["s_t"], seg_off=seg)
+    assert_same("fake-quant", f32_bits(host(y)), f32_bits(rfq))
+    rs = O.quantize(xs, O.NVFP4, O.SR, seg_off=seg, seed=2**33 + 5)
+    assert_same("sr codes", host(sr.codes), rs["codes"])
+    assert_same("amax", f32_bits(host(am)), f32_bits(O.segment_amax(xs, seg)[0]))
+    del busy
 
 
 def test_ste_identity_backward():
