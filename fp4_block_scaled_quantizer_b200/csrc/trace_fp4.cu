@@ -250,13 +250,13 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
 constexpr int kNoAllocWords = ((TF4_NOALLOC_MAX_SEGMENTS + 1) * 4 + 255) / 256 * 64;
 static __device__ __align__(256) uint32_t tf4_noalloc_scratch[kNoAllocWords];
 
-// Device address of tf4_noalloc_scratch on the current device, looked up
-// once per device (with that device current) and cached.
-uint32_t* noalloc_scratch() {
+// Device address of tf4_noalloc_scratch on device `dev`, which must be the
+// current device: looked up once per device (with that device current) and
+// cached.
+uint32_t* noalloc_scratch(int dev) {
   static uint32_t* addr[128] = {nullptr};
   static std::mutex mu;
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return nullptr;
+  if (dev < 0 || dev >= 128) return nullptr;
   std::lock_guard<std::mutex> lock(mu);
   if (!addr[dev]) {
     void* p = nullptr;
@@ -665,7 +665,20 @@ tf4_status tf4_quantize_capture_noalloc(const tf4_desc* desc, const void* x, uin
   tf4_status e = check_desc(desc, &sh);
   if (e != TF4_OK) return e;
   if (sh.nseg > TF4_NOALLOC_MAX_SEGMENTS) return TF4_ERR_WORKSPACE;
-  uint32_t* scratch = noalloc_scratch();
+  // The scratch array has one copy per device; the one used must be that of
+  // the device the kernels run on, which is the current device, so a stream
+  // of another device is refused.
+  int cur = 0, sdev = 0;
+  if (cudaGetDevice(&cur) != cudaSuccess) return TF4_ERR_CUDA;
+  const cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cs == nullptr || cs == cudaStreamLegacy || cs == cudaStreamPerThread) {
+    sdev = cur;  // the default streams belong to the current device
+  } else if (cudaStreamGetDevice(cs, &sdev) != cudaSuccess) {
+    cudaGetLastError();
+    return TF4_ERR_INVALID_ARG;
+  }
+  if (sdev != cur) return TF4_ERR_INVALID_ARG;
+  uint32_t* scratch = noalloc_scratch(cur);
   if (!scratch) return TF4_ERR_CUDA;
   const size_t need = sizeof(uint32_t) * (size_t)(sh.nseg + 1);
   if (has_tensor_scale(sh.fmt) && sh.n > 0 &&

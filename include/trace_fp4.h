@@ -139,20 +139,33 @@ size_t tf4_record_bytes(const tf4_desc* desc, int with_codes);
 /* NVFP4 segment amax (the grid-wide |x| max pass) on its own: writes
  * amax[num_segments] (device, float).  With several shards of one tensor
  * on several GPUs, an all-reduce MAX of these values followed by
- * quantize calls with amax_in gives every shard the tensor-wide scale. */
+ * quantize calls with amax_in gives every shard the tensor-wide scale.
+ * Defined by: the per-tensor fp32 scale of the two-level NVFP4 scaling
+ * (aibr.jp/archives/130278, section 3: blocks of 16 share an E4M3 scale;
+ * the tensor-level factor amax / (6*448) under it is the format's own). */
 tf4_status tf4_segment_amax(const tf4_desc* desc, const void* x, float* amax, void* workspace,
                             size_t workspace_bytes, int32_t* dev_status, tf4_stream_t stream);
 
 /* Round-to-nearest quantization.  NVFP4: s_t (device, [num_segments]) is
  * written; amax_in (device, [num_segments], may be NULL) supplies the
  * segment amax and skips the amax pass (no workspace needed).  MXFP4:
- * amax_in, s_t and the workspace are ignored (pass NULL / 0). */
+ * amax_in, s_t and the workspace are ignored (pass NULL / 0).
+ * Defined by: aibr.jp/archives/130278, section 3 (NVFP4 blocks of 16 E2M1
+ * values with an E4M3 scale; round-to-nearest in the forward pass);
+ * aibr.jp/archives/132665, section 3 (MXFP4's per-group power-of-two
+ * scale); the TRACE summary (ai-papers.net), section
+ * "学習とロールアウトの不一致": the rollout rounds each value to its nearest
+ * codeword. */
 tf4_status tf4_quantize_rtn(const tf4_desc* desc, const void* x, const float* amax_in,
                             uint8_t* codes, uint8_t* scales, float* s_t, void* workspace,
                             size_t workspace_bytes, int32_t* dev_status, tf4_stream_t stream);
 
 /* Stochastic rounding with the Philox4x32-10 stream keyed by `seed`;
- * otherwise as tf4_quantize_rtn. */
+ * otherwise as tf4_quantize_rtn.
+ * Defined by: aibr.jp/archives/130278, section 3 (stochastic rounding for
+ * the backward pass and weight updates); the random stream is
+ * Philox4x32-10 of Salmon et al., "Parallel random numbers: as easy as
+ * 1, 2, 3" (SC'11), with the counter and key given under "Rounding" above. */
 tf4_status tf4_quantize_sr(const tf4_desc* desc, const void* x, uint64_t seed,
                            const float* amax_in, uint8_t* codes, uint8_t* scales, float* s_t,
                            void* workspace, size_t workspace_bytes, int32_t* dev_status,
@@ -162,7 +175,13 @@ tf4_status tf4_quantize_sr(const tf4_desc* desc, const void* x, uint64_t seed,
  * (m3 & 1 of every element) written to guidance_bits.  Pass
  * guidance_bits = NULL for layers whose guidance is not kept (the caller
  * picks the deepest L of N layers); the codes, scales and s_t are then
- * exactly those of tf4_quantize_rtn. */
+ * exactly those of tf4_quantize_rtn.
+ * Defined by: the TRACE summary (ai-papers.net), section "TRACEの仕組み"
+ * (the rollout records, at every quantization point, the codeword it
+ * chose) and section "量子化情報キャッシュ" (only the mantissa bit and the
+ * scale are kept, and only for the deeper layers); the Korean explainer
+ * (sns.style), section "작동 원리" (the rollout engine exports its
+ * quantization results). */
 tf4_status tf4_quantize_capture(const tf4_desc* desc, const void* x, const float* amax_in,
                                 uint8_t* codes, uint8_t* scales, float* s_t,
                                 uint8_t* guidance_bits, void* workspace, size_t workspace_bytes,
@@ -209,7 +228,12 @@ tf4_status tf4_swizzle_scales(const tf4_desc* desc, const uint8_t* scales, uint8
 
 /* Train-side guided quantization of x (the trainer's value) with the
  * rollout's recorded scale bytes, recorded s_t (NVFP4; NULL for MXFP4) and
- * recorded guidance bits.  One pass over x, no workspace. */
+ * recorded guidance bits.  One pass over x, no workspace.
+ * Defined by: the TRACE summary (ai-papers.net), section "TRACEの仕組み":
+ * instead of rounding to nearest, the train side takes whichever of the
+ * two adjacent codewords matches the rollout's record; section
+ * "量子化情報キャッシュ": the mantissa bit and the scale identify it,
+ * because mismatches fall between adjacent codewords. */
 tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_t* rec_scales,
                                const float* rec_s_t, const uint8_t* rec_bits, uint8_t* codes,
                                int32_t* dev_status, tf4_stream_t stream);
@@ -240,15 +264,25 @@ tf4_status tf4_mismatch_stats(const tf4_desc* desc, const void* x, const uint8_t
                               const float* rec_s_t, const uint8_t* rec_codes,
                               unsigned long long* counts, int32_t* dev_status, tf4_stream_t stream);
 
-/* out[i] = (-1)^sign * fl32(V[m3] * S) as fp32 [rows, cols]. */
+/* out[i] = (-1)^sign * fl32(V[m3] * S) as fp32 [rows, cols].
+ * Defined by: the TRACE summary (ai-papers.net), section "TRACEの仕組み":
+ * the forward pass carries the chosen quantized value (codeword times its
+ * block scale), through which the straight-through gradient flows;
+ * aibr.jp/archives/130278, section 3, for the value of an NVFP4 element
+ * (E2M1 magnitude times the E4M3 block scale). */
 tf4_status tf4_dequantize(const tf4_desc* desc, const uint8_t* codes, const uint8_t* scales,
                           const float* s_t, float* out, tf4_stream_t stream);
 
-/* Guidance extraction from codes produced elsewhere: bits = m3 & 1. */
+/* Guidance extraction from codes produced elsewhere: bits = m3 & 1.
+ * Defined by: the TRACE summary (ai-papers.net), section
+ * "量子化情報キャッシュ": of the full record only the mantissa bit (with the
+ * scale) is sent to the trainer; this packs it from full codes. */
 tf4_status tf4_pack_guidance(const tf4_desc* desc, const uint8_t* codes, uint8_t* bits,
                              tf4_stream_t stream);
 
-/* mant[i] = (bits[i >> 3] >> (i & 7)) & 1, one uint8 per element. */
+/* mant[i] = (bits[i >> 3] >> (i & 7)) & 1, one uint8 per element.
+ * Defined by: the same section ("量子化情報キャッシュ"): the per-element
+ * mantissa bit of the compact record, spread to one byte per element. */
 tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_t* mant,
                                tf4_stream_t stream);
 
@@ -263,6 +297,9 @@ tf4_status tf4_unpack_guidance(const tf4_desc* desc, const uint8_t* bits, uint8_
  * process exits (1280 bytes per GPU).
  *  - Limit: desc->num_segments <= TF4_NOALLOC_MAX_SEGMENTS, else
  *    TF4_ERR_WORKSPACE is returned and nothing is launched.
+ *  - `stream` must belong to the current device (the kernels run there and
+ *    use that device's copy of the array); a stream of another device
+ *    returns TF4_ERR_INVALID_ARG with nothing launched.
  *  - The first call on a device looks up that device's address of the
  *    array; make that first call before any stream capture.
  *  - Each call clears the scratch it needs (an asynchronous memset on

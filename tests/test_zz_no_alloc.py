@@ -29,16 +29,16 @@ def _p(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
-def _noalloc_capture(L, x, seg, with_bits=True, fmt=B.NVFP4):
+def _noalloc_capture(L, x, seg, with_bits=True, fmt=B.NVFP4, stream=None):
     rows, cols = x.shape
     d = B.Desc(fmt, rows, cols, seg)
     codes = torch.empty(rows * cols // 2, dtype=torch.uint8, device=x.device)
     scales = torch.empty((rows, cols // B.BLOCK[fmt]), dtype=torch.uint8, device=x.device)
     s_t = torch.empty(d.num_segments, dtype=torch.float32, device=x.device) if B.HAS_TENSOR_SCALE[fmt] else None
     bits = torch.empty(rows * cols // 8, dtype=torch.uint8, device=x.device) if with_bits else None
-    stream = ctypes.c_void_p(torch.cuda.current_stream(x.device).cuda_stream)
+    s = stream if stream is not None else torch.cuda.current_stream(x.device)
     st = L.tf4_quantize_capture_noalloc(d.ptr, _p(x), _p(codes), _p(scales), _p(s_t), _p(bits),
-                                        _p(B.status_word(x.device)), stream)
+                                        _p(B.status_word(x.device, stream)), ctypes.c_void_p(s.cuda_stream))
     return st, codes, scales, s_t, bits
 
 
@@ -81,3 +81,23 @@ def test_noalloc_capture_rejects_too_many_segments():
     assert st == 0
     ref = B.tf4_quantize_capture(x[:MAX_SEGMENTS].contiguous(), seg_off=list(range(MAX_SEGMENTS + 1)))
     assert torch.equal(codes, ref.codes)
+
+
+def test_noalloc_capture_on_a_created_stream():
+    """A stream the caller created on the current device is accepted (the
+    call checks that the stream belongs to the current device, whose copy
+    of the scratch array it uses)."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    libbuild.build()
+    L = B.lib()
+    x = W.random_bf16((130, 512), seed=9, device="cuda", outlier_frac=0.01)
+    ref = B.tf4_quantize_capture(x, seg_off=[0, 64, 130])
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    for _ in range(2):
+        st, codes, scales, s_t, bits = _noalloc_capture(L, x, [0, 64, 130], stream=s)
+        assert st == 0, B.STATUS.get(st, st)
+        s.synchronize()
+        assert torch.equal(codes, ref.codes) and torch.equal(bits, ref.bits)
+        assert torch.equal(s_t.view(torch.int32), ref.s_t.view(torch.int32))
