@@ -1,26 +1,20 @@
-"""The README's usage example runs as written (extracted from README.md and
-executed), and its straight-through backward returns the incoming gradient."""
-import os
-import re
-
+"""The usage example (tests/usage_example.py) runs as written, and its
+straight-through backward returns the incoming gradient."""
 import pytest
 import torch
 
 pytestmark = pytest.mark.gpu
 
-ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
-
-def test_readme_example_runs():
+def test_usage_example_runs():
     if not torch.cuda.is_available():
         pytest.skip("no CUDA device")
     from fp4_block_scaled_quantizer_b200 import build as libbuild
 
     libbuild.build()
-    text = open(os.path.join(ROOT, "README.md")).read()
-    (code,) = re.findall(r"```python\n(.*?)```", text, flags=re.S)
-    env = {}
-    exec(compile(code, "README.md", "exec"), env)
+    import usage_example
+
+    env = usage_example.main()
     y, x_train = env["y"], env["x_train"]
     y.sum().backward()
     assert torch.equal(x_train.grad, torch.ones_like(x_train))
