@@ -306,9 +306,12 @@ def grid_index(codes, n):
 
 
 def mismatch_stats(x, rec_scales, rec_codes, fmt=NVFP4, rec_s_t=None, seg_off=None):
-    """[#(n_r != n_o), #(|n_r - n_o| == 1), #(|n_r - n_o| >= 2), #(n_g != n_o)]
-    with n_r the train value's nearest rounding on the recorded grid, n_o the
-    rollout code, n_g the guided code."""
+    """[#(n_r != n_o), #(|n_r - n_o| == 1), #(|n_r - n_o| >= 2), #(n_g != n_o),
+    #(n_r != n_o, |n_o| < |n_r|), #(n_r != n_o, |n_o| > |n_r|)] with n_r the
+    train value's nearest rounding on the recorded grid, n_o the rollout
+    code, n_g the guided code, |.| the codeword magnitude: the last two split
+    the corrections guidance makes by direction, toward the smaller or the
+    larger codeword (TRACE summary, section 量子化情報キャッシュ)."""
     rows, cols = np.shape(x)
     n = rows * cols
     nr = rtn_with_scales(x, rec_scales, fmt, rec_s_t, seg_off)
@@ -316,4 +319,7 @@ def mismatch_stats(x, rec_scales, rec_codes, fmt=NVFP4, rec_s_t=None, seg_off=No
     ng, _ = quantize_guided(x, rec_scales, bits, fmt, rec_s_t=rec_s_t, seg_off=seg_off)
     io, ir, ig = grid_index(rec_codes, n), grid_index(nr, n), grid_index(ng, n)
     d = np.abs(ir - io)
-    return np.array([(d != 0).sum(), (d == 1).sum(), (d >= 2).sum(), (ig != io).sum()], dtype=np.int64)
+    smaller = (d != 0) & (np.abs(io) < np.abs(ir))
+    larger = (d != 0) & (np.abs(io) > np.abs(ir))
+    return np.array([(d != 0).sum(), (d == 1).sum(), (d >= 2).sum(), (ig != io).sum(), smaller.sum(),
+                     larger.sum()], dtype=np.int64)

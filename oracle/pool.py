@@ -2,16 +2,18 @@
 (spawned processes: safe after the parent has used a GPU).
 
 TEST INFRASTRUCTURE ONLY: the multi-core CPU baseline and reference leg of
-bench.py.  Each task is the oracle's own capture of one layer and, for a
-deep layer, its guided quantization of the perturbed copy -- the same calls
-the single-threaded baseline makes, unchanged, just spread over cores.
+bench.py, and the full-size parity tests.  Each task is the oracle's own
+capture of one layer and, for a deep layer, its guided quantization of the
+perturbed copy -- the same calls the single-threaded baseline makes,
+unchanged, just spread over cores -- or one of the oracle's tensor
+functions on a row range of a larger tensor (map_rows).
 """
 import concurrent.futures as cf
 import multiprocessing as mp
 import os
 import time
 
-from . import NVFP4, RTN, lib, quantize, quantize_guided
+from . import NVFP4, RTN, dequantize, lib, mismatch_stats, quantize, quantize_guided
 
 
 def _layer_task(task):
@@ -34,6 +36,27 @@ def _ready(_):
     return os.getpid()
 
 
+def _rows_task(task):
+    """One row range of a larger tensor, for the full-size parity tests:
+    `kind` is one of the oracle's own tensor functions, called unchanged on
+    the range (segment offsets already made relative to it, tensor scales
+    given)."""
+    kind, kw = task
+    lib()
+    fmt, seg, s_t = kw["fmt"], kw.get("seg"), kw.get("s_t")
+    if kind == "capture":
+        r = quantize(kw["x"], fmt, RTN, seg_off=seg, bits=True, s_t=s_t)
+        return r["codes"], r["scales"], r["bits"], r["status"]
+    if kind == "guided":
+        return quantize_guided(kw["x"], kw["scales"], kw["bits"], fmt, rec_s_t=s_t, seg_off=seg)
+    if kind == "dequant":
+        rows, cols = kw["shape"]
+        return dequantize(kw["codes"], kw["scales"], rows, cols, fmt, s_t=s_t, seg_off=seg)
+    if kind == "mismatch":
+        return mismatch_stats(kw["x"], kw["scales"], kw["codes"], fmt, rec_s_t=s_t, seg_off=seg)
+    raise ValueError(kind)
+
+
 class OraclePool:
     """A pool of `workers` spawned processes; run() does one step (every
     layer's capture, and the guided pass of the deep layers) across them."""
@@ -46,6 +69,10 @@ class OraclePool:
     def run(self, xs, xts, first_deep):
         tasks = [(x, xts[i - first_deep] if i >= first_deep else None) for i, x in enumerate(xs)]
         return list(self.ex.map(_layer_task, tasks))
+
+    def map_rows(self, kind, tasks):
+        """The oracle's `kind` on each row-range task (see _rows_task), in order."""
+        return list(self.ex.map(_rows_task, [(kind, kw) for kw in tasks]))
 
     def close(self):
         self.ex.shutdown()

@@ -367,6 +367,52 @@ def test_mismatch_example_golden(orc):
     assert float(V[orc.guided_m3(ax[1], S, g)]) == ex["codewords"][0]
 
 
+def _rows_scaled(rows, cols, seed):
+    """N(0,1) rows times 10^(0, -1, ..., -5) in turn, with 2% outliers x50:
+    block scales from the E4M3 top down to its subnormals and zero."""
+    x = W.random_bf16((rows, cols), seed=seed, outlier_frac=0.02).float()
+    x *= torch.tensor([10.0 ** -(r % 6) for r in range(rows)])[:, None]
+    x[rows // 2, :32] = 0.0
+    return W.bf16_bits(x.to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("seg", [None, [0, 20, 20, 64]])
+def test_nvfp4_dequant_vs_library_decodes(orc, seg):
+    """NVFP4 dequantization (TRACE summary, section TRACEの仕組み: the forward
+    carries the chosen quantized value): every element equals the numpy fp32
+    product of the code's E2M1 value (ml_dtypes' float4_e2m1fn decode, signed)
+    and fp32(s_t * E4M3 value) (torch's float8_e4m3fn decode of the scale
+    byte, s_t of the row's segment)."""
+    rows, cols = 64, 512
+    x = _rows_scaled(rows, cols, seed=21)
+    r = orc.quantize(x, orc.NVFP4, seg_off=seg)
+    assert r["status"] == 0
+    d = orc.dequantize(r["codes"], r["scales"], rows, cols, orc.NVFP4, s_t=r["s_t"], seg_off=seg)
+    nib = orc.unpack_codes(r["codes"], rows * cols).astype(np.uint8)
+    v = nib.view(ml_dtypes.float4_e2m1fn).astype(np.float32).reshape(rows, cols)
+    dec = torch.from_numpy(r["scales"].copy()).view(torch.float8_e4m3fn).float().numpy().reshape(rows, -1)
+    off = seg if seg is not None else [0, rows]
+    row_seg = np.searchsorted(np.asarray(off), np.arange(rows), side="right") - 1
+    st = np.asarray(r["s_t"], np.float32)[row_seg]
+    S = (st[:, None] * dec).astype(np.float32)                 # one fp32 rounding
+    want = (v * np.repeat(S, 16, axis=1)).astype(np.float32)   # one more
+    assert (r["scales"] < 8).any() and (r["scales"] == 0).any() and (r["scales"] == 0x7E).any()
+    assert np.array_equal(d.view(np.uint32), want.view(np.uint32))
+
+
+def test_mxfp4_dequant_vs_library_decodes(orc):
+    """MXFP4 dequantization: the code's E2M1 value (ml_dtypes) times 2^(byte - 127)."""
+    rows, cols = 64, 512
+    x = _rows_scaled(rows, cols, seed=22)
+    r = orc.quantize(x, orc.MXFP4)
+    d = orc.dequantize(r["codes"], r["scales"], rows, cols, orc.MXFP4)
+    nib = orc.unpack_codes(r["codes"], rows * cols).astype(np.uint8)
+    v = nib.view(ml_dtypes.float4_e2m1fn).astype(np.float64).reshape(rows, cols)
+    e = np.repeat(r["scales"].astype(np.int64).reshape(rows, -1) - 127, 32, axis=1)
+    want = np.ldexp(v, e).astype(np.float32)                    # exact: a power of two times an E2M1 value
+    assert np.array_equal(d.view(np.uint32), want.view(np.uint32))
+
+
 def test_mxfp4_dequant_quant_idempotent(orc):
     """MXFP4 dequantized values are bf16-representable; re-quantizing them
     gives the same codes and scale bytes, and the same values."""
@@ -504,14 +550,15 @@ def test_mismatch_stats_closed_form(orc):
     vals = np.array([4.0, 2.4, 1.0, 0.3] + [0.0] * 28, np.float32)
     x[0] = W.bf16_bits(torch.from_numpy(vals).to(torch.bfloat16).reshape(1, 32))[0]
     r = orc.quantize(x, orc.MXFP4, bits=True)  # block max 4 -> S = 1
-    assert orc.mismatch_stats(x, r["scales"], r["codes"], orc.MXFP4).tolist() == [0, 0, 0, 0]
+    assert orc.mismatch_stats(x, r["scales"], r["codes"], orc.MXFP4).tolist() == [0] * 6
     xt = x.copy()
     vt = vals.copy()
-    vt[1] = 2.6   # 2.4 -> 2 (rollout), 2.6 -> 3: adjacent
-    vt[2] = 1.9   # 1.0 -> 1, 1.9 -> 2: two codewords apart (1 -> 1.5 -> 2)
+    vt[1] = 2.6   # 2.4 -> 2 (rollout), 2.6 -> 3: adjacent; the rollout's codeword is the smaller
+    vt[2] = 1.9   # 1.0 -> 1, 1.9 -> 2: two codewords apart (1 -> 1.5 -> 2); smaller
+    vt[3] = 0.2   # 0.3 -> 0.5, 0.2 -> 0: adjacent; the rollout's codeword is the larger
     xt[0] = W.bf16_bits(torch.from_numpy(vt).to(torch.bfloat16).reshape(1, 32))[0]
     st = orc.mismatch_stats(xt, r["scales"], r["codes"], orc.MXFP4)
-    assert st.tolist() == [2, 1, 1, 1]
+    assert st.tolist() == [3, 2, 1, 1, 2, 1]
 
 
 def _torch_to_blocked():
