@@ -285,9 +285,18 @@ def debug_bounds_violations(device=None, stream=None) -> int:
 
 def read_status(device, stream=None) -> int:
     """Synchronize `stream` (default: the current stream) and return (and
-    clear) the status code of the calls issued on it."""
+    clear) the status code of the calls issued on it.  After a timed-out
+    wait (status 6) the stream's cached workspace is zero-filled again, as
+    the library requires before its reuse."""
     t = status_word(device, stream)
-    return int(lib().tf4_read_status(_ptr(t), _stream(stream, t.device)))
+    st = int(lib().tf4_read_status(_ptr(t), _stream(stream, t.device)))
+    if st == 6:
+        key, s = _stream_key(t.device, stream)
+        ws = _ws_cache.get(key)
+        if ws is not None:
+            with torch.cuda.stream(s):
+                ws.zero_()
+    return st
 
 
 def sizes(fmt: int, rows: int, cols: int, seg_off=None) -> dict:
@@ -498,16 +507,20 @@ def tf4_guided_fake_quant(x, rec: Quantized, out_dtype=torch.float32, want_codes
         return o, c
 
 
+MISMATCH_COUNTS = 6
+
+
 def tf4_mismatch_stats(x, rec: Quantized, counts=None, stream=None) -> torch.Tensor:
     """Mismatch diagnostics of train values x against a rollout record
-    (codes + scales): adds [#mismatch, #adjacent, #far, #after-guidance] to
-    `counts` (int64 [4], zero-initialised if not given) and returns it."""
+    (codes + scales): adds [#mismatch, #adjacent, #far, #after-guidance,
+    #toward-smaller, #toward-larger] to `counts` (int64 [6], zero-initialised
+    if not given) and returns it."""
     with _on(stream):
         x2 = _as_2d(x)
         d = Desc(rec.fmt, x2.shape[0], x2.shape[1], rec.seg_off)
         _check_record(rec, d, x.device, "tf4_mismatch_stats", codes=True)
-        c = (_buf(counts, "counts", 4, torch.int64, x.device) if counts is not None
-             else torch.zeros(4, dtype=torch.int64, device=x.device))
+        c = (_buf(counts, "counts", MISMATCH_COUNTS, torch.int64, x.device) if counts is not None
+             else torch.zeros(MISMATCH_COUNTS, dtype=torch.int64, device=x.device))
         _check(lib().tf4_mismatch_stats(d.ptr, _ptr(x2), _ptr(rec.scales), _ptr(rec.s_t), _ptr(rec.codes), _ptr(c),
                                         _ptr(status_word(x.device, stream)), _stream(stream, x.device)),
                "tf4_mismatch_stats")

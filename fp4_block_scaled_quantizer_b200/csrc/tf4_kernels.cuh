@@ -22,6 +22,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <type_traits>
+
 #include "../../include/trace_fp4.h"
 
 namespace tf4 {
@@ -147,13 +149,23 @@ __device__ __forceinline__ uint32_t vmax_u16x2(uint32_t a, uint32_t b) {
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Per half of two bf16 pairs: the larger magnitude (the sign bits are the
+// XOR of the inputs' and get masked off by the caller), NaN if either is
+// NaN.  Comparing bf16 values is exact.
+__device__ __forceinline__ uint32_t hmax_abs(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // Max |x| over words of bf16 pairs, as a bf16 bit pattern (0x7F80 or more
 // means a non-finite input: the magnitude bit order is the value order).
 template <int N>
 __device__ __forceinline__ uint32_t block_absmax_bits(const uint32_t (&w)[N]) {
-  uint32_t m = w[0] & 0x7FFF7FFFu;
+  uint32_t m = w[0];
 #pragma unroll
-  for (int i = 1; i < N; ++i) m = vmax_u16x2(m, w[i] & 0x7FFF7FFFu);
+  for (int i = 1; i < N; ++i) m = hmax_abs(m, w[i]);
+  m &= 0x7FFF7FFFu;
   return max(m & 0xFFFFu, m >> 16);
 }
 
@@ -448,37 +460,55 @@ __device__ __forceinline__ uint32_t sr_m3_exact(float axf, float Sf, uint32_t r2
   return lhs < rhs ? f + 1u : f;
 }
 
-// Stochastic rounding from y = |x| / S given either exactly (MXFP4) or as a
-// product that is on the correct side of every codeword and equals one iff
-// y does (NVFP4 fast path).  lo / gap come from the fp32 bits of y (for
-// y >= 1 the grid is the 1-mantissa-bit truncation, gap 2^(E-1); below 1 it
-// is {0, 0.5} with gap 0.5), and the threshold t = 2^24 (y - V_lo) / gap is
-// exact arithmetic on y (Sterbenz subtraction, power-of-two scaling).  With
-// an approximate y, |t - T_exact| < 64, so a uniform within 128 of t is
-// flagged `amb` for the exact test.  Returns the chosen codeword value.
-template <bool U = false>
-__device__ __forceinline__ float sr_pick(float y, uint32_t r24, bool margin, bool& amb) {
-  if constexpr (U) {
-    // uniform grid: lo = floor(y), gap 1; y - lo is exact (Sterbenz), so
-    // t = 2^24 (y - lo) is exact arithmetic on y; |y - y_exact| < 2^-17.5
-    // for y < 7.5, so |t - T_exact| < 96
-    const float vlo = floorf(y);
-    const float t = __fmul_rn(__fsub_rn(y, vlo), 0x1p24f);
-    const float rf = __uint2float_rn(r24);
-    amb = margin && fabsf(rf - t) <= 128.0f;
-    const float v = rf < t ? __fadd_rn(vlo, 1.0f) : vlo;
-    return fminf(v, 7.0f);
-  }
+// Stochastic rounding on the E2M1 grid from the exact quotient y = |x| / S
+// (MXFP4: a power-of-two scale): lo and gap come from the fp32 bits of y
+// (for y >= 1 the grid is the 1-mantissa-bit truncation, gap 2^(E-1); below
+// 1 it is {0, 0.5} with gap 0.5), and t = 2^24 (y - lo) / gap is exact
+// arithmetic on y (Sterbenz subtraction, power-of-two scaling), so r24 < t
+// decides exactly.  Returns the chosen codeword value.
+__device__ __forceinline__ float sr_pick_e2m1_exact(float y, uint32_t r24) {
   const uint32_t yb = __float_as_uint(y);
   const bool ge1 = y >= 1.0f;
   const float vlo = ge1 ? __uint_as_float(yb & 0xFFC00000u) : (y >= 0.5f ? 0.5f : 0.0f);
   const float gap = ge1 ? __uint_as_float((yb & 0x7F800000u) - 0x00800000u) : 0.5f;
   const float inv = ge1 ? __uint_as_float((279u - (yb >> 23)) << 23) : 0x1p25f;  // 2^24 / gap
   const float t = __fmul_rn(__fsub_rn(y, vlo), inv);
-  const float rf = __uint2float_rn(r24);  // exact: r24 < 2^24
-  amb = margin && fabsf(rf - t) <= 128.0f;
-  const float v = rf < t ? __fadd_rn(vlo, gap) : vlo;
+  const float v = __uint2float_rn(r24) < t ? __fadd_rn(vlo, gap) : vlo;  // r24 < 2^24: exact
   return fminf(v, 6.0f);
+}
+
+// Stochastic rounding on the uniform grid from y = |x| / S given as a
+// product that is on the correct side of every codeword and equals one iff
+// y does: lo = floor(y), gap 1, and t = 2^24 (y - lo) is exact arithmetic on
+// y (Sterbenz subtraction).  |y - y_exact| < 2^-17.5 for y < 7.5, so
+// |t - T_exact| < 96 and a uniform within 128 of t is flagged `amb` for the
+// exact test.  Returns the chosen codeword value (saturated at 7).
+__device__ __forceinline__ float sr_pick_uni(float y, uint32_t r24, bool& amb) {
+  const float vlo = floorf(y);
+  const float t = __fmul_rn(__fsub_rn(y, vlo), 0x1p24f);
+  const float rf = __uint2float_rn(r24);  // exact: r24 < 2^24
+  amb = fabsf(rf - t) <= 128.0f;
+  const float v = rf < t ? __fadd_rn(vlo, 1.0f) : vlo;
+  return fminf(v, 7.0f);
+}
+
+// Stochastic rounding on the E2M1 grid from y2 = 2y (y = |x| / S given
+// exactly, or as a product on the correct side of every codeword) and the
+// Philox word pw.  W = max(2y, RZ(y + 1)) maps the grid {0, .5, 1, 1.5, 2,
+// 3, 4, 6} onto the numbers with one mantissa bit {1, 1.5, 2, 3, 4, 6, 8,
+// 12} (W = 2y for y >= 1, y + 1 below), so the code of lo is
+// (bits(W) >> 22) - 254 and the threshold 2^24 (y - lo) / (hi - lo) is
+// 4 (bits(W) & 0x3FFFFF), four times the mantissa bits below the top one:
+// round up iff r24 = pw >> 8 is below it, i.e. iff pw >> 10 is below
+// bits(W) & 0x3FFFFF.  RZ(y + 1) (error < 2^-23) and an approximate y move
+// the threshold by less than 64, so a uniform within 128 of it is flagged
+// `amb` for the exact test.  Returns m3, saturated at 7 (y >= 6, and any
+// huge y, map to code 7 or above before the cap).
+__device__ __forceinline__ uint32_t sr_e2m1(float y2, uint32_t pw, bool& amb) {
+  const uint32_t wb = __float_as_uint(fmaxf(y2, __fmaf_rz(y2, 0.5f, 1.0f)));
+  const uint32_t m = wb & 0x3FFFFFu;
+  amb = (pw >> 8) - (m << 2) + 128u <= 256u;
+  return min((wb >> 22) - 254u + ((pw >> 10) < m ? 1u : 0u), 7u);
 }
 
 // -------------------------------------------------------------- amax pass
@@ -767,25 +797,42 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
           const float S = __fmul_rn(st, e4m3_decode(sc));
           const PhiloxBlk pb = philox_block((uint64_t)blk * 16u, ks);
           const uint32_t lo32 = (uint32_t)((uint64_t)blk * 16u);
-          uint32_t c[2];
+          if constexpr (!U) {
+            const float r2 = __uint_as_float(__float_as_uint(r) + 0x00800000u);  // 2 rho, exact
+            uint32_t c[2] = {0u, 0u};
 #pragma unroll
-          for (int q = 0; q < 2; ++q) {  // 8 elements at a time
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const int k = 8 * q + e;
+            for (int k = 0; k < 16; ++k) {
               const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
               const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-              const uint32_t r24 = philox_w0_blk(lo32 + (uint32_t)k, pb, ks) >> 8;
+              const uint32_t pw = philox_w0_blk(lo32 + (uint32_t)k, pb, ks);
               bool amb;
-              float val = sr_pick<U>(mul<RZ>(ax, r), r24, true, amb);
-              if (amb) val = grid_value<U>(sr_m3_exact<U>(ax, S, r24));
-              v[e] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
+              uint32_t m3 = sr_e2m1(mul<RZ>(ax, r2), pw, amb);
+              if (amb) m3 = sr_m3_exact<false>(ax, S, pw >> 8);
+              c[k >> 3] |= (m3 | ((h >> 12) & 8u)) << (4 * (k & 7));
             }
-            c[q] = cvt_grid_x8<U>(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+            c0 = c[0];
+            c1 = c[1];
+          } else {
+            uint32_t c[2];
+#pragma unroll
+            for (int q = 0; q < 2; ++q) {  // 8 elements at a time
+              float v[8];
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const int k = 8 * q + e;
+                const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
+                const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+                const uint32_t r24 = philox_w0_blk(lo32 + (uint32_t)k, pb, ks) >> 8;
+                bool amb;
+                float val = sr_pick_uni(mul<RZ>(ax, r), r24, amb);
+                if (amb) val = grid_value<U>(sr_m3_exact<U>(ax, S, r24));
+                v[e] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
+              }
+              c[q] = cvt_grid_x8<U>(v[0], v[1], v[2], v[3], v[4], v[5], v[6], v[7]);
+            }
+            c0 = c[0];
+            c1 = c[1];
           }
-          c0 = c[0];
-          c1 = c[1];
           return;
         }
       }
@@ -820,6 +867,21 @@ __device__ __forceinline__ void nvfp4_block(const uint32_t (&w)[8], float st, co
   c1 = out[1];
 }
 
+// MXFP4 stochastic rounding where y = |x| 2^-e underflowed to 0 for a
+// nonzero x (possible only for e > 16): the exact threshold is then in
+// (0, 1), so the element rounds up to 0.5 iff r24 == 0 (rare; kept out of
+// the main loop's registers).
+__device__ __noinline__ void mxfp4_sr_underflow(const uint32_t (&w)[16], float inv, uint32_t lo32,
+                                               const PhiloxBlk& pb, const uint32_t* ks, uint32_t (&c)[4]) {
+#pragma unroll 1
+  for (int k = 0; k < 32; ++k) {
+    const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
+    const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+    if (ax != 0.0f && __fmul_rn(ax, inv) == 0.0f && (philox_w0_blk(lo32 + (uint32_t)k, pb, ks) >> 8) == 0u)
+      c[k >> 3] |= 1u << (4 * (k & 7));  // m3 0 -> 1, the sign nibble bit kept
+  }
+}
+
 // One MXFP4 block (32 bf16 in w[0..15]) -> code words, scale byte, flags.
 template <int MODE>
 __device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk, const uint32_t* ks,
@@ -838,7 +900,10 @@ __device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk
     for (int q = 0; q < 4; ++q) c[q] = cvt_words(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3], inv);
     return;
   }
-  // stochastic rounding on the exact quotient y = |x| * 2^-e
+  // stochastic rounding on the quotient y = |x| * 2^-e, exact unless it
+  // underflows (possible only for e > 16: |x| >= 2^-133); a nonzero x whose
+  // y underflows to 0 has 0 < 2^24 (y - lo) / gap < 1, so it rounds up
+  // exactly when r24 == 0
   const float inv = __uint_as_float((uint32_t)(127 - e) << 23);
   const PhiloxBlk pb = philox_block((uint64_t)blk * 32u, ks);
   const uint32_t lo32 = (uint32_t)((uint64_t)blk * 32u);
@@ -847,14 +912,14 @@ __device__ __forceinline__ void mxfp4_block(const uint32_t (&w)[16], int64_t blk
   for (int k = 0; k < 32; ++k) {
     const uint32_t h = (k & 1) ? (w[k >> 1] >> 16) : (w[k >> 1] & 0xFFFFu);
     const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-    bool amb;
-    const float val = sr_pick(__fmul_rn(ax, inv), philox_w0_blk(lo32 + (uint32_t)k, pb, ks) >> 8, false, amb);
+    const float val = sr_pick_e2m1_exact(__fmul_rn(ax, inv), philox_w0_blk(lo32 + (uint32_t)k, pb, ks) >> 8);
     v[k] = __uint_as_float(__float_as_uint(val) | ((h & 0x8000u) << 16));
   }
 #pragma unroll
   for (int q = 0; q < 4; ++q)
     c[q] = cvt_e2m1x8(v[8 * q], v[8 * q + 1], v[8 * q + 2], v[8 * q + 3], v[8 * q + 4], v[8 * q + 5],
                       v[8 * q + 6], v[8 * q + 7]);
+  if (e > 16) mxfp4_sr_underflow(w, inv, lo32, pb, ks, c);
 }
 
 __device__ __forceinline__ void report_bad(bool bad, int32_t* status) {
@@ -877,21 +942,22 @@ constexpr int quant_min_ctas() {
   return (MODE != kSR && std::is_same<SEG, SegN>::value) ? 5 : 0;
 }
 
+// The quantize pass over the CTA's block range [b0, b1), walked backwards
+// (shared by the two-launch and the single-launch capture).
+// `stage` (may be NULL): the CTA's blocks [b0, b1) already in shared memory
+// (16-element formats only), read from there instead of from x.
 template <int FMT, int MODE, class SEG>
-__global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant(QuantArgs a, SEG seg, PhiloxKeys pk) {
-  pdl_enter();
+__device__ __forceinline__ void quant_range(const QuantArgs& a, const SEG& seg, const PhiloxKeys& pk, SegTables& tb,
+                                            int64_t b0, int64_t b1, const uint4* stage = nullptr) {
   // blocks per lane per iteration: 2 keeps 64 B per lane in flight for the
   // memory-bound modes; stochastic rounding is bound by the integer pipe
   // and gains more from the registers (resident warps) one block saves
   constexpr int U = MODE == kSR ? 1 : 2;
-  __shared__ SegTables tb;
-  const int64_t ci = (int64_t)gridDim.x - 1 - blockIdx.x;
-  const int64_t b0 = cta_begin(ci, gridDim.x, a.nblocks);
-  const int64_t b1 = cta_begin(ci + 1, gridDim.x, a.nblocks);
   const int tid = threadIdx.x;
   constexpr bool UG = kUni<FMT>;
   if (kE4M3<FMT> && a.st_from_amax && blockIdx.x == 0 && a.s_t_out)
     for (int k = tid; k < seg.count(); k += kThreads) a.s_t_out[k] = tensor_scale<UG>(a.st_src[k], a.status);
+  bool any_bad = false;  // non-finite inputs, reported once at the end
   int64_t hi = b1;
   while (hi > b0) {
     const int s = seg.find(hi - 1);
@@ -914,7 +980,14 @@ __global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant
           const int64_t k = j + u * kThreads + tid;
           blk[u] = hi - 1 - k;
           if (k < n && unit_ok(blk[u], lo, hi, a.nblocks)) {
-            const uint4 p = __ldg(xs + 2 * blk[u]), q = __ldg(xs + 2 * blk[u] + 1);
+            uint4 p, q;
+            if (stage) {
+              p = stage[2 * (blk[u] - b0)];
+              q = stage[2 * (blk[u] - b0) + 1];
+            } else {
+              p = __ldg(xs + 2 * blk[u]);
+              q = __ldg(xs + 2 * blk[u] + 1);
+            }
             w[u][0] = p.x; w[u][1] = p.y; w[u][2] = p.z; w[u][3] = p.w;
             w[u][4] = q.x; w[u][5] = q.y; w[u][6] = q.z; w[u][7] = q.w;
           }
@@ -935,7 +1008,7 @@ __global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant
               reinterpret_cast<uint16_t*>(bits)[blk[u]] =
                   (uint16_t)(nibble_lsbs(c0) | (nibble_lsbs(c1) << 8));
           }
-          report_bad(bad, a.status);
+          any_bad |= bad;
         }
       } else {
         uint32_t w[U][16];
@@ -966,22 +1039,159 @@ __global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant
                   nibble_lsbs(c[0]) | (nibble_lsbs(c[1]) << 8) | (nibble_lsbs(c[2]) << 16) |
                   (nibble_lsbs(c[3]) << 24);
           }
-          report_bad(bad, a.status);
+          any_bad |= bad;
         }
       }
     }
     hi = lo;
   }
+  report_bad(any_bad, a.status);
+}
+
+template <int FMT, int MODE, class SEG>
+__global__ void __launch_bounds__(kThreads, quant_min_ctas<MODE, SEG>()) k_quant(QuantArgs a, SEG seg, PhiloxKeys pk) {
+  pdl_enter();
+  __shared__ SegTables tb;
+  const int64_t ci = (int64_t)gridDim.x - 1 - blockIdx.x;
+  quant_range<FMT, MODE, SEG>(a, seg, pk, tb, cta_begin(ci, gridDim.x, a.nblocks),
+                              cta_begin(ci + 1, gridDim.x, a.nblocks));
+}
+
+// ------------------------------------------- single-launch capture (small)
+// The amax pass and the quantize pass of an NVFP4 / UFP4 tensor with one
+// segment in one cooperative launch (all CTAs resident at once): each CTA
+// reduces max |x| over its block range and atomicMax-es it into ws[0], then
+// counts itself in ws[1]; thread 0 waits until all gridDim.x CTAs have
+// arrived, and the CTA quantizes the same range, backwards, which it read
+// just before (for a tensor that fits in L2, from L2).  The wait is bounded
+// by wait_ns of %globaltimer: a CTA that gives up ORs TF4_DEV_TIMEOUT into
+// the status word and returns (its outputs are then unspecified, and ws is
+// left as it is).  The last CTA to finish (ws[2]) zeroes ws[0..2].
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ uint32_t ld_acquire(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// STAGED: the CTA's 16-byte chunks read by the amax phase are also kept in
+// dynamic shared memory (the host sizes it to the largest range), and the
+// quantize phase reads them from there.
+template <int FMT, int MODE, bool STAGED>
+__global__ void __launch_bounds__(kThreads) k_quant_fused(QuantArgs a, uint32_t* ws, PhiloxKeys pk,
+                                                          uint64_t wait_ns) {
+  extern __shared__ uint4 stage[];
+  __shared__ SegTables tb;
+  __shared__ uint32_t red[kThreads / 32];
+  __shared__ float amax_sh;
+  __shared__ int arrived;
+  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
+  const int tid = threadIdx.x;
+  // phase 1: max |x| over the range, 16-byte chunks, 8 in flight per thread
+  const int64_t c0 = 2 * b0, c1 = 2 * b1;
+  uint32_t m = 0;
+  int64_t c = c0 + tid;
+  for (; c + 7 * kThreads < c1; c += 8 * kThreads) {
+    uint4 v[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u)
+      v[u] = unit_ok(c + u * kThreads, c0, c1, 2 * a.nblocks) ? __ldg(a.x + c + u * kThreads) : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      if (STAGED) stage[c + u * kThreads - c0] = v[u];
+      m = vmax_u16x2(m, v[u].x & 0x7FFF7FFFu);
+      m = vmax_u16x2(m, v[u].y & 0x7FFF7FFFu);
+      m = vmax_u16x2(m, v[u].z & 0x7FFF7FFFu);
+      m = vmax_u16x2(m, v[u].w & 0x7FFF7FFFu);
+    }
+  }
+  for (; c < c1; c += kThreads) {
+    const uint4 v = unit_ok(c, c0, c1, 2 * a.nblocks) ? __ldg(a.x + c) : make_uint4(0u, 0u, 0u, 0u);
+    if (STAGED) stage[c - c0] = v;
+    m = vmax_u16x2(m, v.x & 0x7FFF7FFFu);
+    m = vmax_u16x2(m, v.y & 0x7FFF7FFFu);
+    m = vmax_u16x2(m, v.z & 0x7FFF7FFFu);
+    m = vmax_u16x2(m, v.w & 0x7FFF7FFFu);
+  }
+  uint32_t mb = __reduce_max_sync(0xFFFFFFFFu, max(m & 0xFFFFu, m >> 16));
+  if ((tid & 31) == 0) red[tid >> 5] = mb;
+  __syncthreads();
+  if (tid == 0) {
+    uint32_t t = red[0];
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) t = max(t, red[w]);
+    atomicMax(ws, t << 16);
+    __threadfence();
+    atomicAdd(ws + 1, 1u);
+    // grid-wide wait for every CTA's maximum, bounded
+    const uint64_t t0 = global_ns();
+    int ok = 1;
+    while (ld_acquire(ws + 1) != gridDim.x) {
+      if (global_ns() - t0 > wait_ns) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(64);
+    }
+    arrived = ok;
+    if (ok) amax_sh = __uint_as_float(__ldcg(ws));
+  }
+  __syncthreads();
+  if (!arrived) {
+    if (tid == 0 && a.status) atomicOr(a.status, TF4_DEV_TIMEOUT);
+    return;
+  }
+  // phase 2: the quantize pass with the tensor amax
+  QuantArgs q = a;
+  q.st_src = &amax_sh;
+  q.st_from_amax = 1;
+  quant_range<FMT, MODE, Seg1>(q, Seg1{}, pk, tb, b0, b1, STAGED ? stage : nullptr);
+  // the last CTA out returns the workspace to zero
+  __syncthreads();
+  if (tid == 0) {
+    __threadfence();
+    if (atomicAdd(ws + 2, 1u) == gridDim.x - 1) {
+      ws[0] = 0u;
+      ws[1] = 0u;
+      ws[2] = 0u;
+    }
+  }
 }
 
 // ----------------------------------------------------------- guided pass
-// Guided rounding = nearest rounding whenever the nearest neighbour already
-// carries the recorded mantissa bit: of the two neighbours lo < y < hi the
-// nearest is one of them, and exactly one has m3 & 1 == g.  So each block
-// is rounded to nearest on the fast path (a multiplier that decides every
-// codeword comparison exactly), the code words are compared with the
-// recorded bits nibble-wise, and only mismatching elements are moved to the
-// other neighbour (or kept: a value equal to a codeword, y >= 6).
+// Guided rounding picks, of the two codewords lo <= y < hi around y, the
+// one whose m3 & 1 equals the recorded bit (y a codeword keeps itself;
+// y >= grid max gives 7).  With the floor code f of y and y strictly
+// between codewords, that is f + ((f ^ g) & 1): only the floor and whether
+// y sits exactly on a codeword are needed, never the nearest code.
+//
+// Both come, for eight elements at once, from one rounding of y to a grid
+// four times finer whose points include every codeword: E2M3 (2 exponent
+// bits, 3 mantissa bits, subnormals 0..7/8) for the E2M1 grid -- an E2M1
+// value with code m3 is the E2M3 value with code m3 << 2 -- and the
+// half-integers for the uniform grid.  Let N be the fine code of y
+// (hardware RNE; for the uniform grid 2^22 + |y| is rounded once to a
+// multiple of 1/2), f = N >> 2 its codeword part and l = N & 3 the rest:
+//  * l != 0: N lies strictly between two codewords, and so does y (a tie
+//    between N and a codeword goes to the codeword, whose code is even):
+//    the answer is f + ((f ^ g) & 1), capped at 7;
+//  * l == 0: y lies within half a fine step of the codeword c = f, hence
+//    strictly between c's two neighbours.  If c's bit equals g the answer
+//    is c wherever y is; otherwise it is c - 1, c or c + 1 by the side of c
+//    that y is on, decided element by element (rare: it needs a train
+//    value next to a codeword the rollout did not choose).
+// With a codeword-safe product y (it is on the same side of every nonzero
+// codeword as the exact quotient, and equal to one iff the quotient is),
+// every step above holds for the exact quotient too; zero is decided on
+// the bf16 value itself, since a nonzero x times r may underflow to 0.
+// The fine codes are handled four to a 32-bit word, one per byte laid out
+// as s << 5 | f << 2 | l.
 struct GuidedArgs {
   const uint4* x;
   int64_t nblocks;
@@ -991,6 +1201,56 @@ struct GuidedArgs {
   uint8_t* codes;
   int32_t* status;
 };
+
+// Eight fp32 values -> eight E2M3 codes (hardware RNE, satfinite): element
+// k in byte k & 3 of b[k >> 2], each byte s << 5 | e << 3 | m.
+__device__ __forceinline__ void cvt_e2m3x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                                           float v7, uint32_t& b0, uint32_t& b1) {
+  asm("{\n\t.reg .b16 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 q0, %3, %2;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 q1, %5, %4;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 q2, %7, %6;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 q3, %9, %8;\n\t"
+      "mov.b32 %0, {q0, q1};\n\t"
+      "mov.b32 %1, {q2, q3};\n\t}"
+      : "=r"(b0), "=r"(b1)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+}
+
+// Fine codes of eight elements (bf16 pairs w0..w3) times r, four per word
+// as above.  Uniform grid: N = RN(2 min(|y|, 7.5)) read from the low byte
+// of 2^22 + min(|y|, 7.5), placed as f << 2 | (N & 1) << 1, sign from x.
+template <bool RZ, bool U, bool CLAMP>
+__device__ __forceinline__ void fine_codes(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
+                                           uint32_t& b0, uint32_t& b1) {
+  if constexpr (U) {
+    const uint32_t w[4] = {w0, w1, w2, w3};
+    uint32_t o[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t t[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint32_t wk = w[2 * h + (k >> 1)];
+        const float v = mul<RZ>((k & 1) ? bf_hi(wk) : bf_lo(wk), r);
+        t[k] = __float_as_uint(__fadd_rn(CLAMP ? fminf(fabsf(v), 7.5f) : fabsf(v), 0x1p22f));
+      }
+      const uint32_t n4 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
+      o[h] = (n4 << 1) | ((__byte_perm(w[2 * h], w[2 * h + 1], 0x7531) >> 2) & 0x20202020u);
+    }
+    b0 = o[0];
+    b1 = o[1];
+  } else {
+    cvt_e2m3x8(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r), mul<RZ>(bf_hi(w1), r),
+               mul<RZ>(bf_lo(w2), r), mul<RZ>(bf_hi(w2), r), mul<RZ>(bf_lo(w3), r), mul<RZ>(bf_hi(w3), r), b0, b1);
+  }
+}
+
+// Four bytes holding values < 16 in each of two words -> eight nibbles
+// (byte k of w0 -> nibble k, byte k of w1 -> nibble 4 + k).
+__device__ __forceinline__ uint32_t pack_nibbles(uint32_t w0, uint32_t w1) {
+  return __byte_perm(w0 | (w0 >> 4), w1 | (w1 >> 4), 0x6420);
+}
 
 // 8 guidance bits -> bit 0 of 8 nibbles (shift-or steps written as
 // multiplies: the shifted copies never overlap).
@@ -1002,42 +1262,197 @@ __device__ __forceinline__ uint32_t spread_bits(uint32_t b) {
   return x;
 }
 
-// Fix the nibbles of code word c (values in the four bf16-pair words
-// w0..w3) whose m3 & 1 differs from the recorded bit (mm: mismatch bits at
-// nibble bit 0): keep exact codewords and the saturated top, otherwise step
-// to the other neighbour.  Zero is decided on x itself: a nonzero x whose
-// product with r underflows to 0 is still above the codeword 0.
-template <bool RZ, bool U = false>
-__device__ __forceinline__ uint32_t fix_mismatches(uint32_t c, uint32_t mm, uint32_t w0, uint32_t w1,
-                                                   uint32_t w2, uint32_t w3, float r) {
-  while (mm) {
-    const int e = (__ffs(mm) - 1) >> 2;  // element within the word
-    mm &= mm - 1u;
-    const uint32_t wsel = (e & 4) ? ((e & 2) ? w3 : w2) : ((e & 2) ? w1 : w0);
-    const uint32_t h = (e & 1) ? (wsel >> 16) : (wsel & 0xFFFFu);
+// The side test for the flagged elements (fl: bit 0 of their nibbles):
+// c = f of the fine code (P's nibble, recorded bit different from c's), so
+// y == c (or y >= grid max at c = 7) keeps c, otherwise the answer is the
+// neighbour on y's side; zero is decided on x itself.
+template <bool RZ, bool U>
+__device__ __noinline__ uint32_t guided_sides(uint32_t c, uint32_t P, uint32_t fl, uint32_t w0, uint32_t w1,
+                                              uint32_t w2, uint32_t w3, float r) {
+  while (fl) {
+    const int e = (__ffs(fl) - 1) >> 2;
+    fl &= fl - 1u;
+    const uint32_t f = (P >> (4 * e)) & 7u;
+    const uint32_t wk = (e & 4) ? ((e & 2) ? w3 : w2) : ((e & 2) ? w1 : w0);
+    const uint32_t h = (e & 1) ? (wk >> 16) : (wk & 0xFFFFu);
     const float y = mul<RZ>(__uint_as_float((h & 0x7FFFu) << 16), r);
-    const uint32_t n = (c >> (4 * e)) & 7u;
-    const float v = grid_value<U>(n);
-    const bool exact = n ? (y == v) : ((h & 0x7FFFu) == 0u);
-    if (!(exact || (n == 7u && y >= kGridMax<U>))) {
-      const uint32_t n2 = (n == 0u || y > v) ? n + 1u : n - 1u;
-      c = (c & ~(7u << (4 * e))) | (n2 << (4 * e));
-    }
+    const float v = grid_value<U>(f);
+    uint32_t m3;
+    if (f == 0u) m3 = (h & 0x7FFFu) ? 1u : 0u;
+    else if (y == v || (f == 7u && y >= kGridMax<U>)) m3 = f;
+    else m3 = y > v ? f + 1u : f - 1u;
+    c = (c & ~(7u << (4 * e))) | (m3 << (4 * e));
   }
   return c;
+}
+
+// Guided rounding of eight elements (bf16 pairs w0..w3; recorded bits g8,
+// element k in bit k) on the codeword-safe multiplier r -> eight nibbles.
+// In nibble form (P: s << 3 | f per element) the answer is f + ((f ^ g) & 1)
+// with f = 7 left as it is; elements with l = 0 whose f's bit differs from
+// g take the side test.
+template <bool RZ, bool U, bool CLAMP>
+__device__ __forceinline__ uint32_t guided_x8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
+                                              uint32_t g8) {
+  uint32_t b0, b1;
+  fine_codes<RZ, U, CLAMP>(w0, w1, w2, w3, r, b0, b1);
+  const uint32_t P = pack_nibbles((b0 >> 2) & 0x0F0F0F0Fu, (b1 >> 2) & 0x0F0F0F0Fu);
+  const uint32_t A = (P ^ spread_bits(g8)) & 0x11111111u;       // f's bit != g
+  const uint32_t F7 = P & (P >> 1) & (P >> 2) & 0x11111111u;    // f == 7
+  const uint32_t c = P + (A & ~F7);
+  const uint32_t fl = A & ~pack_nibbles((b0 | (b0 >> 1)) & 0x01010101u, (b1 | (b1 >> 1)) & 0x01010101u);
+  return fl ? guided_sides<RZ, U>(c, P, fl, w0, w1, w2, w3, r) : c;
+}
+
+// Guided rounding of eight elements by nearest rounding first: where the
+// nearest code already carries the recorded bit it is the answer (it is one
+// of y's two neighbours); `mm` gets the nibbles (bit 0) where it does not.
+template <bool RZ, bool U, bool CLAMP>
+__device__ __forceinline__ uint32_t nearest_x8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
+                                               uint32_t g8, uint32_t& mm) {
+  const uint32_t c = cvt_words<RZ, U, CLAMP>(w0, w1, w2, w3, r);
+  mm = (c ^ spread_bits(g8)) & 0x11111111u;
+  return c;
+}
+
+// Per warp, guided rounding starts with nearest rounding plus the fine
+// rounding for the (warp-uniform) iterations where some lane's nearest code
+// has the wrong bit; once more than a quarter of the warp's iterations (at
+// least 3) needed it, the warp takes the fine rounding for everything.
+struct GuidedMode {
+  int fine = 0, hot = 0, seen = 0;
+  // One nearest-rounding iteration; `any`: some lane needs the fine rounding.
+  __device__ __forceinline__ bool note(bool any) {
+    ++seen;
+    if (!__any_sync(0xFFFFFFFFu, any)) return false;
+    ++hot;
+    fine = (hot >= 3 && 4 * hot > seen) ? 1 : 0;
+    return true;
+  }
+};
+
+#ifndef TF4_GUIDED_U
+#define TF4_GUIDED_U 1
+#endif
+#ifndef TF4_FQ_U
+#define TF4_FQ_U 1
+#endif
+
+// One piece [lo, hi) of a CTA's range (one segment, tensor scale st, rounding
+// mode of its multiplies RZ).  Per iteration every lane takes U blocks; the
+// warp either rounds them with the fine rounding, or (while mismatches are
+// rare) with nearest rounding, recomputing with the fine rounding only the
+// words where some lane's nearest code has the wrong bit.
+template <int FMT, bool RZ>
+__device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, int64_t hi, float st,
+                                             const SegTables& tb, GuidedMode& md, bool& any_bad) {
+  constexpr bool UG = kUni<FMT>;
+  constexpr int BE = kE4M3<FMT> ? 16 : 32;  // elements per block
+  constexpr int NW = BE / 2;                 // bf16 pair words per block
+  constexpr int NQ = BE / 8;                 // code words per block
+  constexpr int U = TF4_GUIDED_U;             // blocks per lane per iteration
+  const int tid = threadIdx.x;
+  const int64_t n = hi - lo;
+  for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
+    uint32_t w[U][NW], sc[U], g[U];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t k = j + u * kThreads + tid;
+      ok[u] = k < n && unit_ok(lo + k, lo, hi, a.nblocks);
+      if (ok[u]) {
+        const int64_t blk = lo + k;
+#pragma unroll
+        for (int q = 0; q < NW / 4; ++q) {
+          const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
+          w[u][4 * q] = p.x; w[u][4 * q + 1] = p.y; w[u][4 * q + 2] = p.z; w[u][4 * q + 3] = p.w;
+        }
+        sc[u] = a.rec_scales[blk];
+        if constexpr (kE4M3<FMT>) g[u] = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
+        else g[u] = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
+      }
+    }
+    uint32_t c[U][NQ];
+    float r[U];
+    bool bad[U], fast[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      bad[u] = false;
+      r[u] = 0.0f;
+      if (ok[u]) {
+        bad[u] = block_absmax_bits(w[u]) >= 0x7F80u;
+        if constexpr (kE4M3<FMT>) {
+          if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu) r[u] = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
+          if (tb.rho[sc[u] & 7u] == 0.0f) r[u] = 0.0f;
+        } else {
+          if (sc[u] >= 1u && sc[u] <= 252u) r[u] = __uint_as_float((254u - sc[u]) << 23);  // 2^-(sc-127), exact
+        }
+        if (r[u] == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
+          float S;
+          if constexpr (kE4M3<FMT>) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
+          else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) c[u][q] = 0u;
+#pragma unroll
+          for (int e = 0; e < BE; ++e) {
+            const uint32_t h = (e & 1) ? (w[u][e >> 1] >> 16) : (w[u][e >> 1] & 0xFFFFu);
+            const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+            const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
+            c[u][e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
+          }
+        }
+      }
+      fast[u] = ok[u] && r[u] != 0.0f;
+    }
+    // nearest rounding first (unless the warp has switched), then the fine
+    // rounding for every word (switched) or for the words that need it
+    const bool all = md.fine;
+    uint32_t mm[U][NQ];
+    bool redo = all;
+    if (!all) {
+      uint32_t any = 0u;
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const uint32_t* wq = &w[u][4 * q];
+          mm[u][q] = 0u;
+          if (fast[u]) c[u][q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r[u], g[u] >> (8 * q), mm[u][q]);
+          any |= mm[u][q];
+        }
+      redo = md.note(any != 0u);
+    }
+    if (redo) {
+#pragma unroll
+      for (int u = 0; u < U; ++u)
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const uint32_t* wq = &w[u][4 * q];
+          if (fast[u] && (all || mm[u][q] != 0u))
+            c[u][q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r[u], g[u] >> (8 * q));
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (ok[u]) {
+        const int64_t blk = lo + j + u * kThreads + tid;
+        if constexpr (kE4M3<FMT>) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[u][0], c[u][1]);
+        else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[u][0], c[u][1], c[u][2], c[u][3]);
+      }
+      any_bad |= bad[u];
+    }
+  }
 }
 
 template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
-  constexpr int BE = kE4M3<FMT> ? 16 : 32;  // elements per block
-  constexpr int NW = BE / 2;                       // bf16 pair words per block
-  constexpr int NQ = BE / 8;                       // code words per block
   __shared__ SegTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
-  const int tid = threadIdx.x;
+  GuidedMode md;
+  bool any_bad = false;  // non-finite inputs, reported once at the end
   int64_t lo = b0;
   while (lo < b1) {
     const int s = seg.find(lo);
@@ -1047,75 +1462,11 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
       st = a.rec_s_t[s];
       build_tables<UG, false>(st, tb);
     }
-    const int64_t n = hi - lo;
-    constexpr int U = 2;  // blocks per lane per iteration
-    for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
-      uint32_t w[U][NW], sc[U], g[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t k = j + u * kThreads + tid;
-        if (k < n && unit_ok(lo + k, lo, hi, a.nblocks)) {
-          const int64_t blk = lo + k;
-#pragma unroll
-          for (int q = 0; q < NW / 4; ++q) {
-            const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
-            w[u][4 * q] = p.x; w[u][4 * q + 1] = p.y; w[u][4 * q + 2] = p.z; w[u][4 * q + 3] = p.w;
-          }
-          sc[u] = a.rec_scales[blk];
-          if constexpr (kE4M3<FMT>) g[u] = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
-          else g[u] = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t k = j + u * kThreads + tid;
-        bool bad = false;
-        if (k < n && unit_ok(lo + k, lo, hi, a.nblocks)) {
-          const int64_t blk = lo + k;
-          const uint32_t mb = block_absmax_bits(w[u]);
-          bad = mb >= 0x7F80u;
-          uint32_t c[NQ];
-          float r = 0.0f;
-          if constexpr (kE4M3<FMT>) {
-            if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu) r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
-            if (tb.rho[sc[u] & 7u] == 0.0f) r = 0.0f;
-          } else {
-            if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);  // 2^-(sc-127), exact
-          }
-          if (r != 0.0f) {
-            const bool rz = kE4M3<FMT> && tb.rz;
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) {
-              const uint32_t* wq = &w[u][4 * q];
-              c[q] = rz ? cvt_words<true, UG>(wq[0], wq[1], wq[2], wq[3], r)
-                        : cvt_words<false, UG>(wq[0], wq[1], wq[2], wq[3], r);
-              const uint32_t mm = (c[q] ^ spread_bits(g[u] >> (8 * q))) & 0x11111111u;
-              if (mm)
-                c[q] = rz ? fix_mismatches<true, UG>(c[q], mm, wq[0], wq[1], wq[2], wq[3], r)
-                          : fix_mismatches<false, UG>(c[q], mm, wq[0], wq[1], wq[2], wq[3], r);
-            }
-          } else {
-            float S;
-            if constexpr (kE4M3<FMT>) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
-            else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
-#pragma unroll
-            for (int q = 0; q < NQ; ++q) c[q] = 0u;
-#pragma unroll
-            for (int e = 0; e < BE; ++e) {
-              const uint32_t h = (e & 1) ? (w[u][e >> 1] >> 16) : (w[u][e >> 1] & 0xFFFFu);
-              const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-              const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
-              c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
-            }
-          }
-          if constexpr (kE4M3<FMT>) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
-          else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);
-        }
-        report_bad(bad, a.status);
-      }
-    }
+    if (kE4M3<FMT> && tb.rz) guided_piece<FMT, true>(a, lo, hi, st, tb, md, any_bad);
+    else guided_piece<FMT, false>(a, lo, hi, st, tb, md, any_bad);
     lo = hi;
   }
+  report_bad(any_bad, a.status);
 }
 
 // --------------------------------------------- fused guided fake-quant
@@ -1144,19 +1495,116 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 // Output modes of the fused pass.
 enum { kOutBf16 = 0, kOutF32 = 1, kOutF32V8 = 2 };
 
+// One piece [lo, hi) of a CTA's range, as guided_piece but on octs of 8
+// elements (one guidance byte, one code word, 8 output values per unit).
+template <int FMT, int OUT, bool RZ>
+__device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t lo, int64_t hi, float st,
+                                                const SegTables& tb, GuidedMode& md, bool& any_bad) {
+  constexpr bool UG = kUni<FMT>;
+  constexpr int BE = kE4M3<FMT> ? 16 : 32;
+  constexpr int OPB = BE / 8;  // octs per block
+  constexpr int U = TF4_FQ_U;  // octs per lane per iteration
+  const int tid = threadIdx.x;
+  const int64_t o0 = lo * OPB, o1 = hi * OPB;
+  for (int64_t ob = o0; ob < o1; ob += (int64_t)U * kThreads) {
+    uint4 xv[U];
+    uint32_t sc[U], g[U];
+    bool ok[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t o = ob + u * kThreads + tid;
+      ok[u] = o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB);
+      if (ok[u]) {
+        xv[u] = __ldg(a.x + o);
+        sc[u] = __ldg(a.rec_scales + o / OPB);
+        g[u] = __ldg(a.rec_bits + o);
+      }
+    }
+    uint32_t c[U];
+    float r[U], S[U];
+    bool bad[U], fast[U];
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
+      bad[u] = false;
+      r[u] = 0.0f;
+      S[u] = 0.0f;
+      c[u] = 0u;
+      if (ok[u]) {
+        bad[u] = block_absmax_bits(w) >= 0x7F80u;
+        if constexpr (kE4M3<FMT>) {
+          S[u] = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
+          if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu && tb.rho[sc[u] & 7u] != 0.0f)
+            r[u] = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
+        } else {
+          S[u] = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
+          if (sc[u] >= 1u && sc[u] <= 252u) r[u] = __uint_as_float((254u - sc[u]) << 23);
+        }
+        if (r[u] == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+            const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+            const uint32_t m3 = S[u] > 0.0f ? guided_m3_exact<UG>(ax, S[u], (g[u] >> e) & 1u) : 0u;
+            c[u] |= (((h >> 15) << 3) | m3) << (4 * e);
+          }
+        }
+      }
+      fast[u] = ok[u] && r[u] != 0.0f;
+    }
+    const bool all = md.fine;
+    uint32_t mm[U];
+    bool redo = all;
+    if (!all) {
+      uint32_t any = 0u;
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint4 v = xv[u];
+        mm[u] = 0u;
+        if (fast[u]) c[u] = nearest_x8<RZ, UG, true>(v.x, v.y, v.z, v.w, r[u], g[u], mm[u]);
+        any |= mm[u];
+      }
+      redo = md.note(any != 0u);
+    }
+    if (redo) {
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const uint4 v = xv[u];
+        if (fast[u] && (all || mm[u] != 0u)) c[u] = guided_x8<RZ, UG, true>(v.x, v.y, v.z, v.w, r[u], g[u]);
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      if (ok[u]) {
+        const int64_t o = ob + u * kThreads + tid;
+        if (a.codes) reinterpret_cast<uint32_t*>(a.codes)[o] = c[u];
+        const float4 v0 = decode4_grid<UG>(c[u] & 0xFFFFu, S[u]), v1 = decode4_grid<UG>(c[u] >> 16, S[u]);
+        if constexpr (OUT == kOutBf16) {
+          reinterpret_cast<uint4*>(a.out)[o] = make_uint4(bf16x2_bits(v0.x, v0.y), bf16x2_bits(v0.z, v0.w),
+                                                          bf16x2_bits(v1.x, v1.y), bf16x2_bits(v1.z, v1.w));
+        } else if constexpr (OUT == kOutF32V8) {
+          st_v8(reinterpret_cast<float*>(a.out) + 8 * o, v0, v1);
+        } else {
+          reinterpret_cast<float4*>(a.out)[2 * o] = v0;
+          reinterpret_cast<float4*>(a.out)[2 * o + 1] = v1;
+        }
+      }
+      any_bad |= bad[u];
+    }
+  }
+}
+
 // OUT: kOutBf16 (one 16-B store per oct), kOutF32 (two 16-B stores),
 // kOutF32V8 (one 32-B store; the host picks it only for a 32-B aligned out).
 template <int FMT, class SEG, int OUT>
 __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
-  constexpr int BE = kE4M3<FMT> ? 16 : 32;
-  constexpr int OPB = BE / 8;  // octs per block
-  constexpr int U = 2;         // octs per lane per iteration
   __shared__ SegTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
-  const int tid = threadIdx.x;
+  GuidedMode md;
+  bool any_bad = false;  // non-finite inputs, reported once at the end
   int64_t lo = b0;
   while (lo < b1) {
     const int s = seg.find(lo);
@@ -1166,74 +1614,11 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
       st = a.rec_s_t[s];
       build_tables<UG, false>(st, tb);
     }
-    const int64_t o0 = lo * OPB, o1 = hi * OPB;
-    for (int64_t ob = o0; ob < o1; ob += (int64_t)U * kThreads) {
-      uint4 xv[U];
-      uint32_t sc[U], g[U];
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t o = ob + u * kThreads + tid;
-        if (o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB)) {
-          xv[u] = __ldg(a.x + o);
-          sc[u] = __ldg(a.rec_scales + o / OPB);
-          g[u] = __ldg(a.rec_bits + o);
-        }
-      }
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int64_t o = ob + u * kThreads + tid;
-        bool bad = false;
-        if (o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB)) {
-          const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
-          const uint32_t mb = block_absmax_bits(w);
-          bad = mb >= 0x7F80u;
-          float r = 0.0f, S;
-          bool rz = false;
-          if constexpr (kE4M3<FMT>) {
-            S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
-            if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu && tb.rho[sc[u] & 7u] != 0.0f) {
-              r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
-              rz = tb.rz;
-            }
-          } else {
-            S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
-            if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);
-          }
-          uint32_t c;
-          if (r != 0.0f) {
-            c = rz ? cvt_words<true, UG>(w[0], w[1], w[2], w[3], r)
-                   : cvt_words<false, UG>(w[0], w[1], w[2], w[3], r);
-            const uint32_t mm = (c ^ spread_bits(g[u])) & 0x11111111u;
-            if (mm)
-              c = rz ? fix_mismatches<true, UG>(c, mm, w[0], w[1], w[2], w[3], r)
-                     : fix_mismatches<false, UG>(c, mm, w[0], w[1], w[2], w[3], r);
-          } else {
-            c = 0u;
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-              const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-              const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
-              c |= (((h >> 15) << 3) | m3) << (4 * e);
-            }
-          }
-          if (a.codes) reinterpret_cast<uint32_t*>(a.codes)[o] = c;
-          const float4 v0 = decode4_grid<UG>(c & 0xFFFFu, S), v1 = decode4_grid<UG>(c >> 16, S);
-          if constexpr (OUT == kOutBf16) {
-            reinterpret_cast<uint4*>(a.out)[o] = make_uint4(bf16x2_bits(v0.x, v0.y), bf16x2_bits(v0.z, v0.w),
-                                                            bf16x2_bits(v1.x, v1.y), bf16x2_bits(v1.z, v1.w));
-          } else if constexpr (OUT == kOutF32V8) {
-            st_v8(reinterpret_cast<float*>(a.out) + 8 * o, v0, v1);
-          } else {
-            reinterpret_cast<float4*>(a.out)[2 * o] = v0;
-            reinterpret_cast<float4*>(a.out)[2 * o + 1] = v1;
-          }
-        }
-        report_bad(bad, a.status);
-      }
-    }
+    if (kE4M3<FMT> && tb.rz) guided_fq_piece<FMT, OUT, true>(a, lo, hi, st, tb, md, any_bad);
+    else guided_fq_piece<FMT, OUT, false>(a, lo, hi, st, tb, md, any_bad);
     lo = hi;
   }
+  report_bad(any_bad, a.status);
 }
 
 // ------------------------------------------------ mismatch diagnostics
@@ -1244,7 +1629,11 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
 // guided code (recorded bit = n_o's mantissa bit); codes compare by signed
 // grid index (sign ? -m3 : m3, so +0 and -0 are equal).  Accumulates
 // counts[0] += #(n_r != n_o), counts[1] += #(|n_r - n_o| == 1),
-// counts[2] += #(|n_r - n_o| >= 2), counts[3] += #(n_g != n_o).
+// counts[2] += #(|n_r - n_o| >= 2), counts[3] += #(n_g != n_o), and the
+// direction of the correction: counts[4] += #(n_r != n_o, m3(n_o) < m3(n_r))
+// (toward the smaller codeword), counts[5] += #(n_r != n_o, m3(n_o) > m3(n_r)).
+constexpr int kMismatchCounts = 6;
+
 struct MismatchArgs {
   const uint4* x;
   int64_t nblocks;
@@ -1262,18 +1651,22 @@ __device__ __forceinline__ int grid_index(uint32_t nib) {
 
 // Counts over the nibbles where code word cx differs from the rollout's co:
 // with d = |index(cx) - index(co)|, cnt[0..2] += (d != 0, d == 1, d >= 2)
-// (NEAREST) or cnt[3] += (d != 0) (guided).  Equal nibbles count nothing.
+// and cnt[4..5] += (d != 0 and m3(co) < m3(cx), d != 0 and m3(co) > m3(cx))
+// (NEAREST), or cnt[3] += (d != 0) (guided).  Equal nibbles count nothing.
 template <bool NEAREST>
-__device__ __forceinline__ void count_diffs(uint32_t cx, uint32_t co, uint32_t (&cnt)[4]) {
+__device__ __forceinline__ void count_diffs(uint32_t cx, uint32_t co, uint32_t (&cnt)[kMismatchCounts]) {
   uint32_t d = cx ^ co;
   while (d) {
     const int e = (__ffs(d) - 1) >> 2;
     d &= ~(0xFu << (4 * e));
-    const int dd = abs(grid_index((cx >> (4 * e)) & 0xFu) - grid_index((co >> (4 * e)) & 0xFu));
+    const uint32_t nx = (cx >> (4 * e)) & 0xFu, no = (co >> (4 * e)) & 0xFu;
+    const int dd = abs(grid_index(nx) - grid_index(no));
     if (NEAREST) {
       cnt[0] += dd != 0;
       cnt[1] += dd == 1;
       cnt[2] += dd >= 2;
+      cnt[4] += dd != 0 && (no & 7u) < (nx & 7u);
+      cnt[5] += dd != 0 && (no & 7u) > (nx & 7u);
     } else {
       cnt[3] += dd != 0;
     }
@@ -1296,7 +1689,7 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
   __shared__ SegTables tmid, tcw;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
-  uint32_t cnt[4] = {0u, 0u, 0u, 0u};
+  uint32_t cnt[kMismatchCounts] = {0u, 0u, 0u, 0u, 0u, 0u};
   int64_t lo = b0;
   bool bad = false;
   while (lo < b1) {
@@ -1362,16 +1755,12 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
         // Where the train value's nearest code equals the rollout's, the
         // rollout code is one of its neighbours and carries the recorded
         // bit, so guided rounding returns it too: only octs with a differing
-        // nibble can add to either count.  (MXFP4's guided conversion is
-        // cheap enough that the branch measured slower there.)
-        if (kE4M3<FMT> && cr == co) continue;
+        // nibble can add to any count.
+        if (cr == co) continue;
         if (rc != 0.0f) {
-          cg = rzc ? cvt_words<true, UG>(wq[0], wq[1], wq[2], wq[3], rc)
-                   : cvt_words<false, UG>(wq[0], wq[1], wq[2], wq[3], rc);
-          const uint32_t mm = (cg ^ co) & 0x11111111u;  // mantissa bit vs the rollout's
-          if (mm)
-            cg = rzc ? fix_mismatches<true, UG>(cg, mm, wq[0], wq[1], wq[2], wq[3], rc)
-                     : fix_mismatches<false, UG>(cg, mm, wq[0], wq[1], wq[2], wq[3], rc);
+          const uint32_t go = nibble_lsbs(co);  // the rollout codes' bits
+          cg = rzc ? guided_x8<true, UG, true>(wq[0], wq[1], wq[2], wq[3], rc, go)
+                   : guided_x8<false, UG, true>(wq[0], wq[1], wq[2], wq[3], rc, go);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
@@ -1389,7 +1778,7 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
   }
   report_bad(bad, a.status);
 #pragma unroll
-  for (int k = 0; k < 4; ++k) {
+  for (int k = 0; k < kMismatchCounts; ++k) {
     const uint32_t t = __reduce_add_sync(0xFFFFFFFFu, cnt[k]);
     if ((threadIdx.x & 31) == 0 && t) atomicAdd(a.counts + k, (unsigned long long)t);
   }

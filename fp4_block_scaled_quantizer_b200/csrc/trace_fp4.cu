@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <climits>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 #include <type_traits>
@@ -177,6 +178,72 @@ tf4_status launch_amax(const Shape& sh, int64_t grid, const void* x, uint32_t* w
   return launched();
 }
 
+// Tensors of at most this many elements (64 MiB of bf16, half the L2)
+// with one segment are captured by the single-launch kernel; larger ones
+// by the amax launch and the quantize launch.
+constexpr int64_t kFusedMaxElems = int64_t(1) << 25;
+// Bound of the single-launch kernel's grid-wide wait (ns of %globaltimer):
+// its amax phase over 64 MiB takes about 10 us.
+constexpr uint64_t kFusedWaitNs = 100000000ull;
+
+int64_t fused_max_elems() {
+  static const int64_t v = [] {
+    const char* e = getenv("TF4_FUSED_MAX_ELEMS");
+    return e ? (int64_t)atoll(e) : kFusedMaxElems;
+  }();
+  return v;
+}
+
+// Resident CTAs per SM of `kernel` with `smem` bytes of dynamic shared
+// memory on the current device (not cached).
+int occupancy_smem(const void* kernel, size_t smem) {
+  int occ = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, smem) != cudaSuccess || occ <= 0) {
+    cudaGetLastError();
+    occ = 0;
+  }
+  return occ;
+}
+
+// Dynamic shared memory the staged single-launch capture may use per CTA
+// (the default limit, no opt-in needed).
+constexpr size_t kStageMaxBytes = 48 * 1024;
+
+// The single-launch capture (k_quant_fused): a cooperative launch, so that
+// every CTA is resident while the CTAs wait for one another; at least 256
+// quantization blocks per CTA.  When every CTA's range of x fits in
+// kStageMaxBytes of shared memory at full residency, the staged variant
+// keeps it there between the two phases.
+template <int FMT, int MODE>
+tf4_status launch_fused(const Shape& sh, const tf4::QuantArgs& a, uint32_t* ws, const tf4::PhiloxKeys& pk,
+                        cudaStream_t st) {
+  auto plain = tf4::k_quant_fused<FMT, MODE, false>;
+  auto staged = tf4::k_quant_fused<FMT, MODE, true>;
+  const int64_t resident = (int64_t)sm_count() * occupancy(reinterpret_cast<const void*>(plain));
+  int64_t g = (sh.nblocks + 255) / 256;
+  g = g < resident ? g : resident;
+  g = g < 1 ? 1 : g;
+  const size_t stage_bytes = (size_t)((sh.nblocks + g - 1) / g) * 32;  // 16 bf16 per block
+  bool use_stage = stage_bytes <= kStageMaxBytes;
+  if (use_stage) {
+    const int64_t r2 = (int64_t)sm_count() * occupancy_smem(reinterpret_cast<const void*>(staged), stage_bytes);
+    use_stage = r2 >= g;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)g);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = use_stage ? stage_bytes : 0;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (use_stage) cudaLaunchKernelEx(&cfg, staged, a, ws, pk, kFusedWaitNs);
+  else cudaLaunchKernelEx(&cfg, plain, a, ws, pk, kFusedWaitNs);
+  return launched();
+}
+
 template <int MODE>
 tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const float* amax_in,
                          uint8_t* codes, uint8_t* scales, float* s_t, uint8_t* bits, void* ws,
@@ -216,6 +283,12 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
       constexpr int FMT = decltype(f)::value;
       if constexpr (tf4::kE4M3<FMT>) {
         const int64_t grid = nvfp4_grid<FMT, MODE>(sh);
+        if constexpr (MODE != tf4::kSR) {
+          if (!amax_in && !multi(sh) && sh.n <= fused_max_elems()) {
+            e = launch_fused<FMT, MODE>(sh, a, static_cast<uint32_t*>(ws), pk, st);
+            return;
+          }
+        }
         if (amax_in) {
           a.st_src = amax_in;
           a.st_from_amax = 1;
@@ -680,7 +753,8 @@ tf4_status tf4_quantize_capture_noalloc(const tf4_desc* desc, const void* x, uin
   if (sdev != cur) return TF4_ERR_INVALID_ARG;
   uint32_t* scratch = noalloc_scratch(cur);
   if (!scratch) return TF4_ERR_CUDA;
-  const size_t need = sizeof(uint32_t) * (size_t)(sh.nseg + 1);
+  // the amax pass uses num_segments + 1 words, the single-launch capture 3
+  const size_t need = sizeof(uint32_t) * (size_t)(sh.nseg + 1 > 3 ? sh.nseg + 1 : 3);
   if (has_tensor_scale(sh.fmt) && sh.n > 0 &&
       cudaMemsetAsync(scratch, 0, need, reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
     return TF4_ERR_CUDA;
@@ -715,7 +789,7 @@ const char* tf4_status_string(tf4_status s) {
   return "unknown status";
 }
 
-int tf4_version(void) { return 1; }
+int tf4_version(void) { return 2; }
 
 int tf4_debug_bounds_enabled(void) {
 #ifdef TF4_DEBUG_BOUNDS

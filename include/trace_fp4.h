@@ -87,6 +87,16 @@
  * zero-filled before its first use; each call leaves it zero-filled again
  * when it completes.  Calls that may run concurrently must not share a
  * workspace.
+ *
+ * Single-launch capture.  An NVFP4 / UFP4 rtn or capture call without
+ * amax_in on one segment of at most 2^25 elements (a tensor that fits in
+ * half of the L2 cache) runs its amax pass and its quantize pass in one
+ * cooperative launch, whose CTAs wait for one another between the two
+ * (same results as the two-launch path).  The wait is bounded (100 ms);
+ * if it gives up, TF4_DEV_TIMEOUT is OR-ed into *dev_status
+ * (tf4_read_status then returns TF4_ERR_TIMEOUT), the call's outputs are
+ * unspecified and the workspace is left non-zero: zero-fill it again
+ * before reusing it.
  */
 #ifndef TRACE_FP4_H
 #define TRACE_FP4_H
@@ -252,14 +262,20 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
 
 /* Train/rollout mismatch diagnostics (TRACE summary, section
  * "量子化情報キャッシュ": more than 99% of mismatches fall between adjacent
- * codewords, which is why one mantissa bit suffices).  For each element of
- * the train value x, with the rollout's recorded scale bytes / s_t: n_r =
- * nearest rounding of x, n_o = the rollout code (rec_codes), n_g = the
- * guided code (recorded bit = mantissa bit of n_o).  Codes compare by signed
- * grid index (sign ? -m3 : m3; +0 == -0).  ADDS to counts (device, 4 x
- * uint64, 8-byte aligned; the caller zeroes it):
+ * codewords, which is why one mantissa bit suffices, and the corrections
+ * toward the smaller codeword concentrate in the deeper layers).  For each
+ * element of the train value x, with the rollout's recorded scale bytes /
+ * s_t: n_r = nearest rounding of x, n_o = the rollout code (rec_codes), n_g
+ * = the guided code (recorded bit = mantissa bit of n_o).  Codes compare by
+ * signed grid index (sign ? -m3 : m3; +0 == -0).  ADDS to counts (device,
+ * TF4_MISMATCH_COUNTS = 6 x uint64, 8-byte aligned; the caller zeroes it):
  *   counts[0] elements with n_r != n_o, counts[1] with |n_r - n_o| == 1,
- *   counts[2] with |n_r - n_o| >= 2, counts[3] with n_g != n_o. */
+ *   counts[2] with |n_r - n_o| >= 2, counts[3] with n_g != n_o,
+ *   counts[4] with n_r != n_o and m3(n_o) < m3(n_r) (the rollout's codeword
+ *   is the smaller: guidance corrects toward the smaller codeword),
+ *   counts[5] with n_r != n_o and m3(n_o) > m3(n_r).
+ * (Library version 2; version 1 wrote counts[0..3] only.) */
+#define TF4_MISMATCH_COUNTS 6
 tf4_status tf4_mismatch_stats(const tf4_desc* desc, const void* x, const uint8_t* rec_scales,
                               const float* rec_s_t, const uint8_t* rec_codes,
                               unsigned long long* counts, int32_t* dev_status, tf4_stream_t stream);

@@ -81,7 +81,7 @@ def test_outputs_stay_inside_their_buffers(fmt, rows, cols, seg):
     B.tf4_guided_fake_quant(xt, q, out=g((rows, cols), torch.float32), codes=g((rows * cols // 2,), torch.uint8))
     B.tf4_guided_fake_quant(xt, q, out=g((rows, cols), torch.bfloat16))
     B.tf4_guided_fake_quant(xt, q, out=f32_16)
-    B.tf4_mismatch_stats(xt, q, counts=g((4,), torch.int64).zero_())
+    B.tf4_mismatch_stats(xt, q, counts=g((B.MISMATCH_COUNTS,), torch.int64).zero_())
     B.tf4_pack_guidance(q.codes, rows, cols, fmt, out=g((rows * cols // 8,), torch.uint8))
     B.tf4_unpack_guidance(q.bits, rows, cols, fmt, out=g((rows * cols,), torch.uint8))
     nb = cols // B.BLOCK[fmt]
@@ -129,7 +129,9 @@ def test_short_or_mistyped_buffers_are_refused_before_launch():
     with pytest.raises(TypeError):
         B.tf4_dequantize(q, out=torch.empty((rows, cols), dtype=torch.float16, device=DEV))
     with pytest.raises(TypeError):
-        B.tf4_mismatch_stats(x, q, counts=torch.zeros(4, dtype=torch.int32, device=DEV))
+        B.tf4_mismatch_stats(x, q, counts=torch.zeros(B.MISMATCH_COUNTS, dtype=torch.int32, device=DEV))
+    with pytest.raises(ValueError):  # the four counts of library version 1 are too few
+        B.tf4_mismatch_stats(x, q, counts=torch.zeros(4, dtype=torch.int64, device=DEV))
     with pytest.raises(TypeError):
         B.tf4_guided_fake_quant(x, q, out=torch.empty((rows, cols), dtype=torch.float16, device=DEV))
     torch.cuda.synchronize()

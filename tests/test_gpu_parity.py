@@ -94,6 +94,45 @@ def test_sr_parity(fmt, seed):
     check_quant(xb, fmt, O.SR, seed=seed)
 
 
+def _seed_with_zero_uniform(idx):
+    """A seed < 2^32 whose Philox4x32-10 word 0 at counter idx has its top 24
+    bits zero (about one seed in 2^24), found with a vectorised search and
+    confirmed by the oracle's own Philox."""
+    M0, M1, W0, W1 = 0xD2511F53, 0xCD9E8D57, 0x9E3779B9, 0xBB67AE85
+    mask = np.uint64(0xFFFFFFFF)
+    for base in range(0, 1 << 32, 1 << 24):
+        k0 = np.arange(base, base + (1 << 24), dtype=np.uint64)
+        k1 = np.zeros_like(k0)
+        c0 = np.full_like(k0, idx)
+        c1, c2, c3 = np.zeros_like(k0), np.zeros_like(k0), np.zeros_like(k0)
+        for _ in range(10):
+            p0, p1 = np.uint64(M0) * c0, np.uint64(M1) * c2
+            c0, c1, c2, c3 = ((p1 >> np.uint64(32)) ^ c1 ^ k0) & mask, p1 & mask, \
+                ((p0 >> np.uint64(32)) ^ c3 ^ k1) & mask, p0 & mask
+            k0, k1 = (k0 + np.uint64(W0)) & mask, (k1 + np.uint64(W1)) & mask
+        hit = np.nonzero((c0 >> np.uint64(8)) == 0)[0]
+        if hit.size:
+            seed = base + int(hit[0])
+            assert O.sr_uniform24(idx, seed) == 0
+            return seed
+    raise AssertionError("no seed found")
+
+
+def test_mxfp4_sr_quotient_underflow():
+    """MXFP4 with block scale 2^118 and a subnormal element: |x| 2^-118
+    underflows fp32 to 0, but the exact threshold is positive, so with the
+    uniform 0 the element rounds up to 0.5 (times the scale)."""
+    idx = 5
+    seed = _seed_with_zero_uniform(idx)
+    for tiny, want in ((0x0001, 0x1), (0x8003, 0x9)):  # +2^-133, -3 * 2^-133
+        x = np.zeros((1, 64), np.uint16)
+        x[0, 0] = 0x7B80        # 2^120: e = 118
+        x[0, idx] = tiny        # the uniform at this index is 0
+        x[0, 7] = 0x3F80        # 1.0: also far below the grid's first point
+        q, r = check_quant(W.from_bits(x, DEV), O.MXFP4, O.SR, seed=seed)
+        assert O.unpack_codes(r["codes"], x.size)[idx] == want  # rounded up, sign kept
+
+
 @pytest.mark.parametrize("fmt", FMTS)
 def test_sr_full_compare_16m(fmt):
     """Every element of a 16.8M-element SR call against the oracle: enough
@@ -680,6 +719,36 @@ def test_wrappers_on_a_stream_that_is_not_current():
     del busy
 
 
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
+@pytest.mark.parametrize("world", [2, 3])
+def test_row_sharded_capture_on_one_gpu(fmt, world):
+    """The row-sharded path with its real CUDA calls: each shard's amax pass
+    (tf4_segment_amax on its rows, every segment kept), the MAX over shards
+    (what the all-reduce computes), then each shard's capture with amax_in.
+    The shards' codes, scales, bits and s_t are exactly the unsharded
+    capture's, which equals the oracle's."""
+    from fp4_block_scaled_quantizer_b200 import sharded
+
+    rows, cols, seg = 203, 1024, [0, 50, 50, 130, 203]
+    x = W.random_bf16((rows, cols), seed=97, device=DEV, outlier_frac=0.01)
+    full, r = check_quant(x, fmt, seg=seg)
+    parts = []
+    for rank in range(world):
+        b, e = sharded.shard_rows(rows, world, rank)
+        parts.append((b, e, x[b:e].contiguous(), sharded.shard_segments(seg, b, e)))
+    amax = [B.tf4_segment_amax(xs, so) for _, _, xs, so in parts]
+    gmax = amax[0]
+    for a in amax[1:]:
+        gmax = torch.maximum(gmax, a)
+    for b, e, xs, so in parts:
+        q = B.tf4_quantize_capture(xs, fmt=fmt, seg_off=so, amax_in=gmax)
+        assert torch.equal(q.codes, full.codes[b * cols // 2:e * cols // 2])
+        assert torch.equal(q.scales.view(-1), full.scales.view(-1)[b * cols // 16:e * cols // 16])
+        assert torch.equal(q.bits, full.bits[b * cols // 8:e * cols // 8])
+        assert torch.equal(q.s_t.view(torch.int32), full.s_t.view(torch.int32))
+    assert B.read_status(x.device) == 0
+
+
 def test_ste_identity_backward():
     from fp4_block_scaled_quantizer_b200 import ste
     xb = W.random_bf16((16, 256), seed=41, device=DEV).requires_grad_(True)
@@ -839,7 +908,7 @@ def test_dequant_fake_quant_unpack_diagnostics_beyond_2_32_elements():
     x = torch.randn((rows, cols), generator=g, device=DEV, dtype=torch.bfloat16)
     q = B.tf4_quantize_capture(x)
     cnt = B.tf4_mismatch_stats(x, q)
-    assert cnt.tolist() == [0, 0, 0, 0]
+    assert cnt.tolist() == [0] * B.MISMATCH_COUNTS
     r0 = 2**32 // cols
     sample = (0, r0 - 1, r0, r0 + 1, rows - 1)
     st = host(q.s_t)
