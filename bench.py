@@ -66,6 +66,9 @@ def parse():
     p.add_argument("--cpu-mc-factor", type=int, default=8,
                    help="the all-core oracle sample is this many times the single-core one")
     p.add_argument("--ref-rows", type=int, default=256, help="rows per layer per reference step")
+    p.add_argument("--train-rel", type=float, default=1e-3,
+                   help="relative perturbation of the train-side copies (x' = bf16(x (1 + rel N(0,1)))); "
+                        "larger values make more train values round to another codeword than the rollout's")
     p.add_argument("--suite", action="store_true",
                    help="time every call of the path on every workload (a table, not the bench line)")
     p.add_argument("--only", action="append",
@@ -205,7 +208,7 @@ def make_stack(args, dev):
         x = W.layer_stack_layer(layer, dev, rows=args.rows, cols=args.cols)
         xs.append(x)
         if layer >= args.layers - args.deep:
-            xts.append(W.perturb(x, 1000 + layer))
+            xts.append(W.perturb(x, 1000 + layer, rel=args.train_rel))
     torch.cuda.synchronize()
     return xs, xts
 
@@ -263,6 +266,11 @@ def run_ours(args, world, rank, local):
         step(None)
     torch.cuda.synchronize()
     assert B.read_status(dev) == 0, "non-finite input in the workload"
+    # how often a train value's nearest code differs from the rollout's (outside the timed region)
+    cnt = torch.zeros(B.MISMATCH_COUNTS, dtype=torch.int64, device=dev)
+    for j in range(D):
+        B.tf4_mismatch_stats(xts[j], recs[first_deep + j], counts=cnt)
+    mismatch_fraction = float(cnt[0].item()) / (D * n) if D else 0.0
     # per-kernel events on every event_every-th timed step, read after the timed region
     every = max(1, args.event_every)
     evs = [dict(amax=new_events(L), quant=new_events(L), guided=new_events(D)) if k % every == 0 else None
@@ -323,7 +331,8 @@ def run_ours(args, world, rank, local):
                config=dict(workload=f"layer_stack: {L} layers x {args.rows}x{args.cols} bf16 "
                                     f"(0.5*t4 x LogNormal channel scales), NVFP4 capture with guidance for "
                                     f"layers {first_deep}-{L - 1}, guided quantization of perturbed copies "
-                                    f"of those layers",
+                                    f"of those layers (x (1 + {args.train_rel:g} N(0,1)))",
+                           train_rel=args.train_rel, train_mismatch_fraction=round(mismatch_fraction, 6),
                            layers=L, deep_layers=D, rows=args.rows, cols=args.cols, format="NVFP4",
                            parallelism=f"dp{world} (independent stacks)",
                            l2="inputs 512 MiB per layer > 126 MB L2; no flush",
@@ -478,7 +487,7 @@ def sample_host(args, rows):
         x = W.layer_stack_layer(layer, dev, rows=args.rows, cols=args.cols)
         xs.append(W.bf16_bits(x[:rows].contiguous()))
         if layer >= args.layers - args.deep:
-            xts.append(W.bf16_bits(W.perturb(x, 1000 + layer)[:rows].contiguous()))
+            xts.append(W.bf16_bits(W.perturb(x, 1000 + layer, rel=args.train_rel)[:rows].contiguous()))
         del x
     return xs, xts
 
@@ -638,12 +647,21 @@ def run_suite(args):
         del g
         return a.elapsed_time(b) / reps * 1e3
 
+    L2_BYTES = 126e6
+
     def run(workload, fmt, call, n, fn, cold=False, **extra):
-        if sel(workload, fmt, call):
-            record(workload, fmt, call, n, timed(fn), l2="warm" if cold else None, **extra)
-            if cold:
-                record(workload, fmt, call, n, timed_graph(fn), l2="warm, CUDA graph", **extra)
-                record(workload, fmt, call, n, timed_cold(fn), l2="cold", **extra)
+        if not sel(workload, fmt, call):
+            return
+        if cold:
+            record(workload, fmt, call, n, timed(fn), l2="warm", **extra)
+            record(workload, fmt, call, n, timed_graph(fn), l2="warm, CUDA graph", **extra)
+            record(workload, fmt, call, n, timed_cold(fn), l2="cold", **extra)
+        elif CALL_BYTES[(fmt, call)] * n < 2 * L2_BYTES:
+            # a working set that back-to-back calls would find in L2: flush before each call so that
+            # the figure is an HBM one
+            record(workload, fmt, call, n, timed_cold(fn), l2="cold (flushed: working set < 2 x L2)", **extra)
+        else:
+            record(workload, fmt, call, n, timed(fn), **extra)
 
     def record(workload, fmt, call, n, us, l2=None, **extra):
         gbs = CALL_BYTES[(fmt, call)] * n / (us * 1e-6) / 1e9
@@ -661,10 +679,11 @@ def run_suite(args):
         run(name, fmt, "guided_fq_bf16", n, lambda: B.tf4_guided_fake_quant(xt, q, out=yb))
         if not sel(name, fmt, "mismatch"):
             return
-        cnt = torch.zeros(4, dtype=torch.int64, device=dev)
+        cnt = torch.zeros(B.MISMATCH_COUNTS, dtype=torch.int64, device=dev)
         us = timed(lambda: B.tf4_mismatch_stats(xt, q, counts=cnt.zero_()))
         c = [int(v) for v in B.tf4_mismatch_stats(xt, q).tolist()]
-        record(name, fmt, "mismatch", n, us, counts=dict(mismatch=c[0], adjacent=c[1], far=c[2], after_guidance=c[3]),
+        record(name, fmt, "mismatch", n, us, counts=dict(mismatch=c[0], adjacent=c[1], far=c[2], after_guidance=c[3],
+                                                        toward_smaller=c[4], toward_larger=c[5]),
                adjacent_fraction=(round(c[1] / c[0], 6) if c[0] else None))
 
     def nv_calls(name, x, xt, seg=None, cold=False):
@@ -786,6 +805,29 @@ def run_suite(args):
         mx_calls(name, x, xt)
         uf_calls(name, x, xt)
         del x, xt
+    name = "layer_stack layer 65536x4096, train copy x (1 + rel N(0,1))"
+    if sel(name):
+        # guided rounding, fused fake-quant and diagnostics at growing train/rollout mismatch rates
+        x = W.layer_stack_layer(20, dev)
+        n = x.numel()
+        for fmt, fname in ((B.NVFP4, "nvfp4"), (B.MXFP4, "mxfp4"), (B.UFP4, "ufp4")):
+            q = B.tf4_quantize_capture(x, fmt=fmt)
+            g = torch.empty_like(q.codes)
+            yf = torch.empty(x.shape, dtype=torch.float32, device=dev)
+            yb = torch.empty(x.shape, dtype=torch.bfloat16, device=dev)
+            cnt = torch.zeros(B.MISMATCH_COUNTS, dtype=torch.int64, device=dev)
+            for rel in (0.0, 1e-3, 1e-2, 5e-2, None):
+                xt = (W.perturb(x, 1020, rel=rel) if rel else x) if rel is not None else \
+                    W.layer_stack_layer(21, dev)
+                frac = int(B.tf4_mismatch_stats(xt, q)[0]) / n
+                tag = dict(train_rel=("unrelated tensor" if rel is None else rel), mismatch_fraction=round(frac, 6))
+                run(name, fname, "guided", n, lambda: B.tf4_quantize_guided(xt, q, out=g), **tag)
+                run(name, fname, "guided_fq_f32", n, lambda: B.tf4_guided_fake_quant(xt, q, out=yf), **tag)
+                run(name, fname, "guided_fq_bf16", n, lambda: B.tf4_guided_fake_quant(xt, q, out=yb), **tag)
+                run(name, fname, "mismatch", n, lambda: B.tf4_mismatch_stats(xt, q, counts=cnt.zero_()), **tag)
+                del xt
+            del q, g, yf, yb
+        del x
     name = "moe_dispatch 262144x2048, 128 experts"
     if sel(name):
         w = W.moe_dispatch(dev)
