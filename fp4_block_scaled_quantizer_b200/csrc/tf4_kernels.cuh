@@ -957,7 +957,6 @@ __device__ __forceinline__ void quant_range(const QuantArgs& a, const SEG& seg, 
   constexpr bool UG = kUni<FMT>;
   if (kE4M3<FMT> && a.st_from_amax && blockIdx.x == 0 && a.s_t_out)
     for (int k = tid; k < seg.count(); k += kThreads) a.s_t_out[k] = tensor_scale<UG>(a.st_src[k], a.status);
-  bool any_bad = false;  // non-finite inputs, reported once at the end
   int64_t hi = b1;
   while (hi > b0) {
     const int s = seg.find(hi - 1);
@@ -1008,7 +1007,7 @@ __device__ __forceinline__ void quant_range(const QuantArgs& a, const SEG& seg, 
               reinterpret_cast<uint16_t*>(bits)[blk[u]] =
                   (uint16_t)(nibble_lsbs(c0) | (nibble_lsbs(c1) << 8));
           }
-          any_bad |= bad;
+          report_bad(bad, a.status);
         }
       } else {
         uint32_t w[U][16];
@@ -1039,13 +1038,12 @@ __device__ __forceinline__ void quant_range(const QuantArgs& a, const SEG& seg, 
                   nibble_lsbs(c[0]) | (nibble_lsbs(c[1]) << 8) | (nibble_lsbs(c[2]) << 16) |
                   (nibble_lsbs(c[3]) << 24);
           }
-          any_bad |= bad;
+          report_bad(bad, a.status);
         }
       }
     }
     hi = lo;
   }
-  report_bad(any_bad, a.status);
 }
 
 template <int FMT, int MODE, class SEG>
@@ -1317,16 +1315,20 @@ __device__ __forceinline__ uint32_t nearest_x8(uint32_t w0, uint32_t w1, uint32_
 
 // Per warp, guided rounding starts with nearest rounding plus the fine
 // rounding for the (warp-uniform) iterations where some lane's nearest code
-// has the wrong bit; once more than a quarter of the warp's iterations (at
-// least 3) needed it, the warp takes the fine rounding for everything.
+// has the wrong bit.  A score (one register) gains 4 on such an iteration
+// and loses 1 on a clean one, kept within [-16, 0]; once it passes 0 (at
+// least 3 such iterations in a row from the start, or about one in four
+// later on) the warp takes the fine rounding for the rest of its range.
 struct GuidedMode {
-  int fine = 0, hot = 0, seen = 0;
-  // One nearest-rounding iteration; `any`: some lane needs the fine rounding.
+  int score = -8;
+  __device__ __forceinline__ bool fine() const { return score > 0; }
+  // One nearest-rounding iteration; `any`: this lane needs the fine rounding.
   __device__ __forceinline__ bool note(bool any) {
-    ++seen;
-    if (!__any_sync(0xFFFFFFFFu, any)) return false;
-    ++hot;
-    fine = (hot >= 3 && 4 * hot > seen) ? 1 : 0;
+    if (!__any_sync(0xFFFFFFFFu, any)) {
+      score = max(score - 1, -16);
+      return false;
+    }
+    score += 4;
     return true;
   }
 };
@@ -1339,13 +1341,14 @@ struct GuidedMode {
 #endif
 
 // One piece [lo, hi) of a CTA's range (one segment, tensor scale st, rounding
-// mode of its multiplies RZ).  Per iteration every lane takes U blocks; the
-// warp either rounds them with the fine rounding, or (while mismatches are
-// rare) with nearest rounding, recomputing with the fine rounding only the
-// words where some lane's nearest code has the wrong bit.
+// mode of its multiplies RZ).  Per iteration every lane loads U blocks, then
+// takes them one at a time: the warp rounds the block either with the fine
+// rounding, or (while mismatches are rare) with nearest rounding,
+// recomputing with the fine rounding only the words where some lane's
+// nearest code has the wrong bit.
 template <int FMT, bool RZ>
 __device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, int64_t hi, float st,
-                                             const SegTables& tb, GuidedMode& md, bool& any_bad) {
+                                             const SegTables& tb, GuidedMode& md) {
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;  // elements per block
   constexpr int NW = BE / 2;                 // bf16 pair words per block
@@ -1372,87 +1375,88 @@ __device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, in
         else g[u] = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
       }
     }
-    uint32_t c[U][NQ];
-    float r[U];
-    bool bad[U], fast[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
-      bad[u] = false;
-      r[u] = 0.0f;
+      uint32_t c[NQ];
+      float r = 0.0f;
+      bool bad = false;
       if (ok[u]) {
-        bad[u] = block_absmax_bits(w[u]) >= 0x7F80u;
+        bad = block_absmax_bits(w[u]) >= 0x7F80u;
         if constexpr (kE4M3<FMT>) {
-          if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu) r[u] = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
-          if (tb.rho[sc[u] & 7u] == 0.0f) r[u] = 0.0f;
+          if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu) r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
+          if (tb.rho[sc[u] & 7u] == 0.0f) r = 0.0f;
         } else {
-          if (sc[u] >= 1u && sc[u] <= 252u) r[u] = __uint_as_float((254u - sc[u]) << 23);  // 2^-(sc-127), exact
+          if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);  // 2^-(sc-127), exact
         }
-        if (r[u] == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
+        if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
           float S;
           if constexpr (kE4M3<FMT>) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
           else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) c[u][q] = 0u;
+          for (int q = 0; q < NQ; ++q) c[q] = 0u;
 #pragma unroll
           for (int e = 0; e < BE; ++e) {
             const uint32_t h = (e & 1) ? (w[u][e >> 1] >> 16) : (w[u][e >> 1] & 0xFFFFu);
             const float ax = __uint_as_float((h & 0x7FFFu) << 16);
             const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
-            c[u][e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
+            c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
           }
         }
       }
-      fast[u] = ok[u] && r[u] != 0.0f;
-    }
-    // nearest rounding first (unless the warp has switched), then the fine
-    // rounding for every word (switched) or for the words that need it
-    const bool all = md.fine;
-    uint32_t mm[U][NQ];
-    bool redo = all;
-    if (!all) {
-      uint32_t any = 0u;
-#pragma unroll
-      for (int u = 0; u < U; ++u)
+      const bool fast = ok[u] && r != 0.0f;
+      // nearest rounding first (unless the warp has switched), then the fine
+      // rounding for every word (switched) or for the words that need it
+      const bool all = md.fine();
+      uint32_t mm[NQ];
+      bool redo = all;
+      if (!all) {
+        uint32_t any = 0u;
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           const uint32_t* wq = &w[u][4 * q];
-          mm[u][q] = 0u;
-          if (fast[u]) c[u][q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r[u], g[u] >> (8 * q), mm[u][q]);
-          any |= mm[u][q];
+          mm[q] = 0u;
+          if (fast) c[q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
+          any |= mm[q];
         }
-      redo = md.note(any != 0u);
-    }
-    if (redo) {
-#pragma unroll
-      for (int u = 0; u < U; ++u)
+        redo = md.note(any != 0u);
+      }
+      if (redo) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           const uint32_t* wq = &w[u][4 * q];
-          if (fast[u] && (all || mm[u][q] != 0u))
-            c[u][q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r[u], g[u] >> (8 * q));
+          if (fast && (all || mm[q] != 0u))
+            c[q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q));
         }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
+      }
       if (ok[u]) {
         const int64_t blk = lo + j + u * kThreads + tid;
-        if constexpr (kE4M3<FMT>) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[u][0], c[u][1]);
-        else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[u][0], c[u][1], c[u][2], c[u][3]);
+        if constexpr (kE4M3<FMT>) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
+        else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);
       }
-      any_bad |= bad[u];
+      report_bad(bad, a.status);
     }
   }
 }
 
+// Resident CTAs per SM the guided kernels are compiled for.  They are
+// latency-bound, so occupancy decides their speed more than spare
+// registers: k_guided at <= 40 registers keeps 6 CTAs (48 warps) per SM for
+// the 16-element formats (MXFP4 needs more without spilling), k_guided_fq
+// at <= 32 keeps 8 (64 warps).
+template <int FMT>
+constexpr int guided_min_ctas() {
+  return kE4M3<FMT> ? 6 : 1;
+}
+constexpr int kGuidedFqMinCtas = 8;
+
 template <int FMT, class SEG>
-__global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
+__global__ void __launch_bounds__(kThreads, guided_min_ctas<FMT>()) k_guided(GuidedArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
   __shared__ SegTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   GuidedMode md;
-  bool any_bad = false;  // non-finite inputs, reported once at the end
   int64_t lo = b0;
   while (lo < b1) {
     const int s = seg.find(lo);
@@ -1462,11 +1466,10 @@ __global__ void __launch_bounds__(kThreads) k_guided(GuidedArgs a, SEG seg) {
       st = a.rec_s_t[s];
       build_tables<UG, false>(st, tb);
     }
-    if (kE4M3<FMT> && tb.rz) guided_piece<FMT, true>(a, lo, hi, st, tb, md, any_bad);
-    else guided_piece<FMT, false>(a, lo, hi, st, tb, md, any_bad);
+    if (kE4M3<FMT> && tb.rz) guided_piece<FMT, true>(a, lo, hi, st, tb, md);
+    else guided_piece<FMT, false>(a, lo, hi, st, tb, md);
     lo = hi;
   }
-  report_bad(any_bad, a.status);
 }
 
 // --------------------------------------------- fused guided fake-quant
@@ -1499,7 +1502,7 @@ enum { kOutBf16 = 0, kOutF32 = 1, kOutF32V8 = 2 };
 // elements (one guidance byte, one code word, 8 output values per unit).
 template <int FMT, int OUT, bool RZ>
 __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t lo, int64_t hi, float st,
-                                                const SegTables& tb, GuidedMode& md, bool& any_bad) {
+                                                const SegTables& tb, GuidedMode& md) {
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int OPB = BE / 8;  // octs per block
@@ -1520,65 +1523,45 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
         g[u] = __ldg(a.rec_bits + o);
       }
     }
-    uint32_t c[U];
-    float r[U], S[U];
-    bool bad[U], fast[U];
 #pragma unroll
     for (int u = 0; u < U; ++u) {
       const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
-      bad[u] = false;
-      r[u] = 0.0f;
-      S[u] = 0.0f;
-      c[u] = 0u;
+      uint32_t c = 0u;
+      float r = 0.0f, S = 0.0f;
+      bool bad = false;
       if (ok[u]) {
-        bad[u] = block_absmax_bits(w) >= 0x7F80u;
+        bad = block_absmax_bits(w) >= 0x7F80u;
         if constexpr (kE4M3<FMT>) {
-          S[u] = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
+          S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
           if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu && tb.rho[sc[u] & 7u] != 0.0f)
-            r[u] = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
+            r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
         } else {
-          S[u] = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
-          if (sc[u] >= 1u && sc[u] <= 252u) r[u] = __uint_as_float((254u - sc[u]) << 23);
+          S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
+          if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);
         }
-        if (r[u] == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
+        if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
             const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
             const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-            const uint32_t m3 = S[u] > 0.0f ? guided_m3_exact<UG>(ax, S[u], (g[u] >> e) & 1u) : 0u;
-            c[u] |= (((h >> 15) << 3) | m3) << (4 * e);
+            const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
+            c |= (((h >> 15) << 3) | m3) << (4 * e);
           }
         }
       }
-      fast[u] = ok[u] && r[u] != 0.0f;
-    }
-    const bool all = md.fine;
-    uint32_t mm[U];
-    bool redo = all;
-    if (!all) {
-      uint32_t any = 0u;
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint4 v = xv[u];
-        mm[u] = 0u;
-        if (fast[u]) c[u] = nearest_x8<RZ, UG, true>(v.x, v.y, v.z, v.w, r[u], g[u], mm[u]);
-        any |= mm[u];
+      const bool fast = ok[u] && r != 0.0f;
+      const bool all = md.fine();
+      uint32_t mm = 0u;
+      bool redo = all;
+      if (!all) {
+        if (fast) c = nearest_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u], mm);
+        redo = md.note(mm != 0u);
       }
-      redo = md.note(any != 0u);
-    }
-    if (redo) {
-#pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const uint4 v = xv[u];
-        if (fast[u] && (all || mm[u] != 0u)) c[u] = guided_x8<RZ, UG, true>(v.x, v.y, v.z, v.w, r[u], g[u]);
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < U; ++u) {
+      if (redo && fast && (all || mm != 0u)) c = guided_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u]);
       if (ok[u]) {
         const int64_t o = ob + u * kThreads + tid;
-        if (a.codes) reinterpret_cast<uint32_t*>(a.codes)[o] = c[u];
-        const float4 v0 = decode4_grid<UG>(c[u] & 0xFFFFu, S[u]), v1 = decode4_grid<UG>(c[u] >> 16, S[u]);
+        if (a.codes) reinterpret_cast<uint32_t*>(a.codes)[o] = c;
+        const float4 v0 = decode4_grid<UG>(c & 0xFFFFu, S), v1 = decode4_grid<UG>(c >> 16, S);
         if constexpr (OUT == kOutBf16) {
           reinterpret_cast<uint4*>(a.out)[o] = make_uint4(bf16x2_bits(v0.x, v0.y), bf16x2_bits(v0.z, v0.w),
                                                           bf16x2_bits(v1.x, v1.y), bf16x2_bits(v1.z, v1.w));
@@ -1589,7 +1572,7 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
           reinterpret_cast<float4*>(a.out)[2 * o + 1] = v1;
         }
       }
-      any_bad |= bad[u];
+      report_bad(bad, a.status);
     }
   }
 }
@@ -1597,14 +1580,13 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
 // OUT: kOutBf16 (one 16-B store per oct), kOutF32 (two 16-B stores),
 // kOutF32V8 (one 32-B store; the host picks it only for a 32-B aligned out).
 template <int FMT, class SEG, int OUT>
-__global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg) {
+__global__ void __launch_bounds__(kThreads, kGuidedFqMinCtas) k_guided_fq(GuidedFqArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
   __shared__ SegTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   GuidedMode md;
-  bool any_bad = false;  // non-finite inputs, reported once at the end
   int64_t lo = b0;
   while (lo < b1) {
     const int s = seg.find(lo);
@@ -1614,11 +1596,10 @@ __global__ void __launch_bounds__(kThreads) k_guided_fq(GuidedFqArgs a, SEG seg)
       st = a.rec_s_t[s];
       build_tables<UG, false>(st, tb);
     }
-    if (kE4M3<FMT> && tb.rz) guided_fq_piece<FMT, OUT, true>(a, lo, hi, st, tb, md, any_bad);
-    else guided_fq_piece<FMT, OUT, false>(a, lo, hi, st, tb, md, any_bad);
+    if (kE4M3<FMT> && tb.rz) guided_fq_piece<FMT, OUT, true>(a, lo, hi, st, tb, md);
+    else guided_fq_piece<FMT, OUT, false>(a, lo, hi, st, tb, md);
     lo = hi;
   }
-  report_bad(any_bad, a.status);
 }
 
 // ------------------------------------------------ mismatch diagnostics
