@@ -1302,6 +1302,15 @@ __device__ __forceinline__ uint32_t guided_x8(uint32_t w0, uint32_t w1, uint32_t
   return fl ? guided_sides<RZ, U>(c, P, fl, w0, w1, w2, w3, r) : c;
 }
 
+// The same as a call: the nearest-rounding loops recompute a word with it
+// only where a lane's nearest code has the wrong bit, which keeps the fine
+// rounding's registers out of their (two-unit) iteration.
+template <bool RZ, bool U>
+__device__ __noinline__ uint32_t guided_x8_call(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
+                                                uint32_t g8) {
+  return guided_x8<RZ, U, true>(w0, w1, w2, w3, r, g8);
+}
+
 // Guided rounding of eight elements by nearest rounding first: where the
 // nearest code already carries the recorded bit it is the answer (it is one
 // of y's two neighbours); `mm` gets the nibbles (bit 0) where it does not.
@@ -1333,119 +1342,162 @@ struct GuidedMode {
   }
 };
 
-#ifndef TF4_GUIDED_U
-#define TF4_GUIDED_U 1
-#endif
-#ifndef TF4_FQ_U
-#define TF4_FQ_U 1
-#endif
+// Per-segment tables of the guided kernels (E4M3-scaled formats), indexed
+// by the recorded scale byte: the block's multiplier r (0: the block takes
+// the exact comparisons) and its scale S = s_t * decode(byte), so a block
+// reads both with one shared-memory load each.
+struct GuidedTables : SegTables {
+  float rblk[256];
+  float sblk[256];
+};
+
+// After build_tables (all threads of the CTA call this; it synchronizes).
+__device__ void build_block_tables(float st, GuidedTables& t) {
+  static_assert(kThreads == 256, "one table entry per thread");
+  const uint32_t sc = threadIdx.x;
+  float r = 0.0f;
+  if (t.fast && (sc >> 3) >= 1u && sc < 0x7Fu && t.rho[sc & 7u] != 0.0f) r = block_rho(t.rho[sc & 7u], sc >> 3);
+  t.rblk[sc] = r;
+  t.sblk[sc] = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
+  __syncthreads();
+}
+
+// Non-finite input seen by this lane (rare: each lane reports on its own,
+// with no warp vote on the common path).
+__device__ __forceinline__ void report_bad_lane(bool bad, int32_t* status) {
+  if (bad && status) atomicOr(status, TF4_DEV_NONFINITE);
+}
+
+// One block of a guided pass: its codeword-safe multiplier r (0 when the
+// block takes the exact comparisons, whose codes then go to c) and whether
+// it holds a non-finite input.
+template <int FMT>
+__device__ __forceinline__ float guided_block_r(const uint32_t (&w)[kE4M3<FMT> ? 8 : 16], uint32_t sc, uint32_t g,
+                                                const GuidedTables& tb, uint32_t (&c)[kE4M3<FMT> ? 2 : 4],
+                                                bool& bad) {
+  constexpr bool UG = kUni<FMT>;
+  constexpr int BE = kE4M3<FMT> ? 16 : 32;
+  constexpr int NQ = BE / 8;
+  bad = block_absmax_bits(w) >= 0x7F80u;
+  float r;
+  if constexpr (kE4M3<FMT>) r = tb.rblk[sc];
+  else r = (sc >= 1u && sc <= 252u) ? __uint_as_float((254u - sc) << 23) : 0.0f;  // 2^-(sc-127), exact
+  if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
+    float S;
+    if constexpr (kE4M3<FMT>) S = tb.sblk[sc];
+    else S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) c[q] = 0u;
+#pragma unroll
+    for (int e = 0; e < BE; ++e) {
+      const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+      const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+      const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g >> e) & 1u) : 0u;
+      c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
+    }
+  }
+  return r;
+}
+
+template <int FMT>
+__device__ __forceinline__ void guided_load(const GuidedArgs& a, int64_t blk, uint32_t (&w)[kE4M3<FMT> ? 8 : 16],
+                                            uint32_t& sc, uint32_t& g) {
+  constexpr int NC = kE4M3<FMT> ? 2 : 4;  // 16-B pieces of x per block
+#pragma unroll
+  for (int q = 0; q < NC; ++q) {
+    const uint4 p = __ldg(a.x + NC * blk + q);
+    w[4 * q] = p.x; w[4 * q + 1] = p.y; w[4 * q + 2] = p.z; w[4 * q + 3] = p.w;
+  }
+  sc = a.rec_scales[blk];
+  if constexpr (kE4M3<FMT>) g = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
+  else g = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
+}
+
+template <int FMT>
+__device__ __forceinline__ void guided_store(const GuidedArgs& a, int64_t blk, const uint32_t (&c)[kE4M3<FMT> ? 2 : 4]) {
+  if constexpr (kE4M3<FMT>) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
+  else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);
+}
 
 // One piece [lo, hi) of a CTA's range (one segment, tensor scale st, rounding
-// mode of its multiplies RZ).  Per iteration every lane loads U blocks, then
-// takes them one at a time: the warp rounds the block either with the fine
-// rounding, or (while mismatches are rare) with nearest rounding,
-// recomputing with the fine rounding only the words where some lane's
-// nearest code has the wrong bit.
+// mode of its multiplies RZ).  While the warp's mismatches are rare it runs
+// nearest rounding on two blocks per lane per iteration, recomputing with
+// the fine rounding (a call) only the words where some lane's nearest code
+// has the wrong bit; once GuidedMode switches, the rest of the range takes
+// the fine rounding, one block per lane per iteration.
 template <int FMT, bool RZ>
-__device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, int64_t hi, float st,
-                                             const SegTables& tb, GuidedMode& md) {
+__device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, int64_t hi,
+                                             const GuidedTables& tb, GuidedMode& md) {
   constexpr bool UG = kUni<FMT>;
-  constexpr int BE = kE4M3<FMT> ? 16 : 32;  // elements per block
-  constexpr int NW = BE / 2;                 // bf16 pair words per block
-  constexpr int NQ = BE / 8;                 // code words per block
-  constexpr int U = TF4_GUIDED_U;             // blocks per lane per iteration
+  constexpr int NW = kE4M3<FMT> ? 8 : 16;  // bf16 pair words per block
+  constexpr int NQ = NW / 4;               // code words per block
   const int tid = threadIdx.x;
   const int64_t n = hi - lo;
-  for (int64_t j = 0; j < n; j += (int64_t)U * kThreads) {
-    uint32_t w[U][NW], sc[U], g[U];
-    bool ok[U];
+  int64_t j = 0;
+  for (; j < n && !md.fine(); j += 2 * kThreads) {
+    uint32_t w[2][NW], sc[2], g[2];
+    bool ok[2];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int64_t k = j + u * kThreads + tid;
       ok[u] = k < n && unit_ok(lo + k, lo, hi, a.nblocks);
-      if (ok[u]) {
-        const int64_t blk = lo + k;
-#pragma unroll
-        for (int q = 0; q < NW / 4; ++q) {
-          const uint4 p = __ldg(a.x + (NW / 4) * blk + q);
-          w[u][4 * q] = p.x; w[u][4 * q + 1] = p.y; w[u][4 * q + 2] = p.z; w[u][4 * q + 3] = p.w;
-        }
-        sc[u] = a.rec_scales[blk];
-        if constexpr (kE4M3<FMT>) g[u] = __ldg(reinterpret_cast<const uint16_t*>(a.rec_bits) + blk);
-        else g[u] = __ldg(reinterpret_cast<const uint32_t*>(a.rec_bits) + blk);
-      }
+      if (ok[u]) guided_load<FMT>(a, lo + k, w[u], sc[u], g[u]);
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
-      uint32_t c[NQ];
-      float r = 0.0f;
+    for (int u = 0; u < 2; ++u) {
+      uint32_t c[NQ], mm[NQ];
       bool bad = false;
-      if (ok[u]) {
-        bad = block_absmax_bits(w[u]) >= 0x7F80u;
-        if constexpr (kE4M3<FMT>) {
-          if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu) r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
-          if (tb.rho[sc[u] & 7u] == 0.0f) r = 0.0f;
-        } else {
-          if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);  // 2^-(sc-127), exact
-        }
-        if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
-          float S;
-          if constexpr (kE4M3<FMT>) S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
-          else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
-#pragma unroll
-          for (int q = 0; q < NQ; ++q) c[q] = 0u;
-#pragma unroll
-          for (int e = 0; e < BE; ++e) {
-            const uint32_t h = (e & 1) ? (w[u][e >> 1] >> 16) : (w[u][e >> 1] & 0xFFFFu);
-            const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-            const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
-            c[e >> 3] |= (((h >> 15) << 3) | m3) << (4 * (e & 7));
-          }
-        }
-      }
+      float r = 0.0f;
+      if (ok[u]) r = guided_block_r<FMT>(w[u], sc[u], g[u], tb, c, bad);
       const bool fast = ok[u] && r != 0.0f;
-      // nearest rounding first (unless the warp has switched), then the fine
-      // rounding for every word (switched) or for the words that need it
-      const bool all = md.fine();
-      uint32_t mm[NQ];
-      bool redo = all;
-      if (!all) {
-        uint32_t any = 0u;
+      uint32_t any = 0u;
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) {
+        const uint32_t* wq = &w[u][4 * q];
+        mm[q] = 0u;
+        if (fast) c[q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
+        any |= mm[q];
+      }
+      if (md.note(any != 0u)) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
           const uint32_t* wq = &w[u][4 * q];
-          mm[q] = 0u;
-          if (fast) c[q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
-          any |= mm[q];
-        }
-        redo = md.note(any != 0u);
-      }
-      if (redo) {
-#pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const uint32_t* wq = &w[u][4 * q];
-          if (fast && (all || mm[q] != 0u))
-            c[q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q));
+          if (mm[q] != 0u) c[q] = guided_x8_call<RZ, UG>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q));
         }
       }
-      if (ok[u]) {
-        const int64_t blk = lo + j + u * kThreads + tid;
-        if constexpr (kE4M3<FMT>) reinterpret_cast<uint2*>(a.codes)[blk] = make_uint2(c[0], c[1]);
-        else reinterpret_cast<uint4*>(a.codes)[blk] = make_uint4(c[0], c[1], c[2], c[3]);
-      }
-      report_bad(bad, a.status);
+      if (ok[u]) guided_store<FMT>(a, lo + j + u * kThreads + tid, c);
+      report_bad_lane(bad, a.status);
     }
+  }
+  for (; j < n; j += kThreads) {
+    const int64_t k = j + tid;
+    const bool ok = k < n && unit_ok(lo + k, lo, hi, a.nblocks);
+    uint32_t w[NW], sc = 0u, g = 0u, c[NQ];
+    bool bad = false;
+    if (ok) {
+      guided_load<FMT>(a, lo + k, w, sc, g);
+      const float r = guided_block_r<FMT>(w, sc, g, tb, c, bad);
+      if (r != 0.0f) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          const uint32_t* wq = &w[4 * q];
+          c[q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g >> (8 * q));
+        }
+      }
+      guided_store<FMT>(a, lo + k, c);
+    }
+    report_bad_lane(bad, a.status);
   }
 }
 
 // Resident CTAs per SM the guided kernels are compiled for.  They are
 // latency-bound, so occupancy decides their speed more than spare
 // registers: k_guided at <= 40 registers keeps 6 CTAs (48 warps) per SM for
-// the 16-element formats (MXFP4 needs more without spilling), k_guided_fq
-// at <= 32 keeps 8 (64 warps).
+// the 16-element formats, at <= 64 4 CTAs for MXFP4 (twice the data per
+// block), k_guided_fq at <= 32 keeps 8 (64 warps).
 template <int FMT>
 constexpr int guided_min_ctas() {
-  return kE4M3<FMT> ? 6 : 1;
+  return kE4M3<FMT> ? 6 : 4;
 }
 constexpr int kGuidedFqMinCtas = 8;
 
@@ -1453,7 +1505,7 @@ template <int FMT, class SEG>
 __global__ void __launch_bounds__(kThreads, guided_min_ctas<FMT>()) k_guided(GuidedArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
-  __shared__ SegTables tb;
+  __shared__ GuidedTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   GuidedMode md;
@@ -1465,9 +1517,10 @@ __global__ void __launch_bounds__(kThreads, guided_min_ctas<FMT>()) k_guided(Gui
     if constexpr (kE4M3<FMT>) {
       st = a.rec_s_t[s];
       build_tables<UG, false>(st, tb);
+      build_block_tables(st, tb);
     }
-    if (kE4M3<FMT> && tb.rz) guided_piece<FMT, true>(a, lo, hi, st, tb, md);
-    else guided_piece<FMT, false>(a, lo, hi, st, tb, md);
+    if (kE4M3<FMT> && tb.rz) guided_piece<FMT, true>(a, lo, hi, tb, md);
+    else guided_piece<FMT, false>(a, lo, hi, tb, md);
     lo = hi;
   }
 }
@@ -1498,23 +1551,70 @@ __device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
 // Output modes of the fused pass.
 enum { kOutBf16 = 0, kOutF32 = 1, kOutF32V8 = 2 };
 
-// One piece [lo, hi) of a CTA's range, as guided_piece but on octs of 8
-// elements (one guidance byte, one code word, 8 output values per unit).
-template <int FMT, int OUT, bool RZ>
-__device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t lo, int64_t hi, float st,
-                                                const SegTables& tb, GuidedMode& md) {
+// One oct of the fused pass: scale S of its block, codeword-safe multiplier
+// r (0 when the oct takes the exact comparisons, whose codes then go to c)
+// and whether it holds a non-finite input.
+template <int FMT>
+__device__ __forceinline__ float fq_oct_r(const uint32_t (&w)[4], uint32_t sc, uint32_t g, const GuidedTables& tb,
+                                          float& S, uint32_t& c, bool& bad) {
   constexpr bool UG = kUni<FMT>;
-  constexpr int BE = kE4M3<FMT> ? 16 : 32;
-  constexpr int OPB = BE / 8;  // octs per block
-  constexpr int U = TF4_FQ_U;  // octs per lane per iteration
+  bad = block_absmax_bits(w) >= 0x7F80u;
+  float r;
+  if constexpr (kE4M3<FMT>) {
+    S = tb.sblk[sc];
+    r = tb.rblk[sc];
+  } else {
+    S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
+    r = (sc >= 1u && sc <= 252u) ? __uint_as_float((254u - sc) << 23) : 0.0f;
+  }
+  if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
+    c = 0u;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
+      const float ax = __uint_as_float((h & 0x7FFFu) << 16);
+      const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g >> e) & 1u) : 0u;
+      c |= (((h >> 15) << 3) | m3) << (4 * e);
+    }
+  }
+  return r;
+}
+
+// Codes (optional) and dequantized values of oct o.
+template <int FMT, int OUT>
+__device__ __forceinline__ void fq_store(const GuidedFqArgs& a, int64_t o, uint32_t c, float S) {
+  constexpr bool UG = kUni<FMT>;
+  if (a.codes) reinterpret_cast<uint32_t*>(a.codes)[o] = c;
+  const float4 v0 = decode4_grid<UG>(c & 0xFFFFu, S), v1 = decode4_grid<UG>(c >> 16, S);
+  if constexpr (OUT == kOutBf16) {
+    reinterpret_cast<uint4*>(a.out)[o] = make_uint4(bf16x2_bits(v0.x, v0.y), bf16x2_bits(v0.z, v0.w),
+                                                    bf16x2_bits(v1.x, v1.y), bf16x2_bits(v1.z, v1.w));
+  } else if constexpr (OUT == kOutF32V8) {
+    st_v8(reinterpret_cast<float*>(a.out) + 8 * o, v0, v1);
+  } else {
+    reinterpret_cast<float4*>(a.out)[2 * o] = v0;
+    reinterpret_cast<float4*>(a.out)[2 * o + 1] = v1;
+  }
+}
+
+// One piece [lo, hi) of a CTA's range, as guided_piece but on octs of 8
+// elements (one guidance byte, one code word, 8 output values per unit):
+// two octs per lane per iteration in the nearest-rounding phase, one in
+// the fine-rounding phase.
+template <int FMT, int OUT, bool RZ>
+__device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t lo, int64_t hi,
+                                                const GuidedTables& tb, GuidedMode& md) {
+  constexpr bool UG = kUni<FMT>;
+  constexpr int OPB = kE4M3<FMT> ? 2 : 4;  // octs per block
   const int tid = threadIdx.x;
   const int64_t o0 = lo * OPB, o1 = hi * OPB;
-  for (int64_t ob = o0; ob < o1; ob += (int64_t)U * kThreads) {
-    uint4 xv[U];
-    uint32_t sc[U], g[U];
-    bool ok[U];
+  int64_t ob = o0;
+  for (; ob < o1 && !md.fine(); ob += 2 * kThreads) {
+    uint4 xv[2];
+    uint32_t sc[2], g[2];
+    bool ok[2];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const int64_t o = ob + u * kThreads + tid;
       ok[u] = o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB);
       if (ok[u]) {
@@ -1524,56 +1624,33 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
       }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < 2; ++u) {
       const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
-      uint32_t c = 0u;
+      uint32_t c = 0u, mm = 0u;
       float r = 0.0f, S = 0.0f;
       bool bad = false;
-      if (ok[u]) {
-        bad = block_absmax_bits(w) >= 0x7F80u;
-        if constexpr (kE4M3<FMT>) {
-          S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc[u])) : 0.0f;
-          if (tb.fast && (sc[u] >> 3) >= 1u && sc[u] < 0x7Fu && tb.rho[sc[u] & 7u] != 0.0f)
-            r = block_rho(tb.rho[sc[u] & 7u], sc[u] >> 3);
-        } else {
-          S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
-          if (sc[u] >= 1u && sc[u] <= 252u) r = __uint_as_float((254u - sc[u]) << 23);
-        }
-        if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const uint32_t h = (e & 1) ? (w[e >> 1] >> 16) : (w[e >> 1] & 0xFFFFu);
-            const float ax = __uint_as_float((h & 0x7FFFu) << 16);
-            const uint32_t m3 = S > 0.0f ? guided_m3_exact<UG>(ax, S, (g[u] >> e) & 1u) : 0u;
-            c |= (((h >> 15) << 3) | m3) << (4 * e);
-          }
-        }
-      }
-      const bool fast = ok[u] && r != 0.0f;
-      const bool all = md.fine();
-      uint32_t mm = 0u;
-      bool redo = all;
-      if (!all) {
-        if (fast) c = nearest_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u], mm);
-        redo = md.note(mm != 0u);
-      }
-      if (redo && fast && (all || mm != 0u)) c = guided_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u]);
-      if (ok[u]) {
-        const int64_t o = ob + u * kThreads + tid;
-        if (a.codes) reinterpret_cast<uint32_t*>(a.codes)[o] = c;
-        const float4 v0 = decode4_grid<UG>(c & 0xFFFFu, S), v1 = decode4_grid<UG>(c >> 16, S);
-        if constexpr (OUT == kOutBf16) {
-          reinterpret_cast<uint4*>(a.out)[o] = make_uint4(bf16x2_bits(v0.x, v0.y), bf16x2_bits(v0.z, v0.w),
-                                                          bf16x2_bits(v1.x, v1.y), bf16x2_bits(v1.z, v1.w));
-        } else if constexpr (OUT == kOutF32V8) {
-          st_v8(reinterpret_cast<float*>(a.out) + 8 * o, v0, v1);
-        } else {
-          reinterpret_cast<float4*>(a.out)[2 * o] = v0;
-          reinterpret_cast<float4*>(a.out)[2 * o + 1] = v1;
-        }
-      }
-      report_bad(bad, a.status);
+      if (ok[u]) r = fq_oct_r<FMT>(w, sc[u], g[u], tb, S, c, bad);
+      if (ok[u] && r != 0.0f) c = nearest_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u], mm);
+      if (md.note(mm != 0u) && mm != 0u) c = guided_x8_call<RZ, UG>(w[0], w[1], w[2], w[3], r, g[u]);
+      if (ok[u]) fq_store<FMT, OUT>(a, ob + u * kThreads + tid, c, S);
+      report_bad_lane(bad, a.status);
     }
+  }
+  for (; ob < o1; ob += kThreads) {
+    const int64_t o = ob + tid;
+    const bool ok = o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB);
+    bool bad = false;
+    if (ok) {
+      const uint4 xv = __ldg(a.x + o);
+      const uint32_t sc = __ldg(a.rec_scales + o / OPB), g = __ldg(a.rec_bits + o);
+      const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+      uint32_t c = 0u;
+      float S = 0.0f;
+      const float r = fq_oct_r<FMT>(w, sc, g, tb, S, c, bad);
+      if (r != 0.0f) c = guided_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g);
+      fq_store<FMT, OUT>(a, o, c, S);
+    }
+    report_bad_lane(bad, a.status);
   }
 }
 
@@ -1583,7 +1660,7 @@ template <int FMT, class SEG, int OUT>
 __global__ void __launch_bounds__(kThreads, kGuidedFqMinCtas) k_guided_fq(GuidedFqArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
-  __shared__ SegTables tb;
+  __shared__ GuidedTables tb;
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   GuidedMode md;
@@ -1595,9 +1672,10 @@ __global__ void __launch_bounds__(kThreads, kGuidedFqMinCtas) k_guided_fq(Guided
     if constexpr (kE4M3<FMT>) {
       st = a.rec_s_t[s];
       build_tables<UG, false>(st, tb);
+      build_block_tables(st, tb);
     }
-    if (kE4M3<FMT> && tb.rz) guided_fq_piece<FMT, OUT, true>(a, lo, hi, st, tb, md);
-    else guided_fq_piece<FMT, OUT, false>(a, lo, hi, st, tb, md);
+    if (kE4M3<FMT> && tb.rz) guided_fq_piece<FMT, OUT, true>(a, lo, hi, tb, md);
+    else guided_fq_piece<FMT, OUT, false>(a, lo, hi, tb, md);
     lo = hi;
   }
 }
