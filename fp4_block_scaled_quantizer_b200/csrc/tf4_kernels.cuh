@@ -52,6 +52,13 @@ __device__ __forceinline__ void pdl_enter() {
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// First unit of part i when n units are split into `grid` parts whose
+// sizes differ by at most one (part i is [cta_begin(i), cta_begin(i + 1))).
+__device__ __forceinline__ int64_t cta_begin(int64_t i, int64_t grid, int64_t n) {
+  const int64_t q = n / grid, r = n % grid;
+  return i * q + (i < r ? i : r);
+}
+
 // ------------------------------------------------------------- segments
 // One per-tensor-scale segment covering everything (the common case).
 struct Seg1 {
@@ -86,6 +93,32 @@ struct SegN {
   __device__ __forceinline__ uint8_t* bitsptr(int /*s*/, uint8_t* b) const { return b; }
 };
 
+// Ragged segments with one piece per CTA (the guided kernels): the host
+// gives each non-empty segment its own CTAs (cta[s] .. cta[s+1] - 1, about
+// in proportion to its blocks), so no CTA walks from one segment into the
+// next; that walk, carried in registers around two instantiations of the
+// block loop, made the loop spill.
+struct SegPieces {
+  int32_t nseg;
+  int64_t bpr;                         // quantization blocks per row
+  int32_t off[TF4_MAX_SEGMENTS + 1];   // row offsets of the segments
+  int32_t cta[TF4_MAX_SEGMENTS + 1];   // first CTA of each segment (non-decreasing; cta[nseg] = grid)
+  // CTA i's segment s (the largest s with cta[s] <= i: non-empty) and its
+  // part [lo, hi), part i - cta[s] of cta[s+1] - cta[s] near-equal parts.
+  __device__ __forceinline__ void piece(int i, int& s, int64_t& lo, int64_t& hi) const {
+    int l = 0, h = nseg;  // answer in [l, h)
+    while (h - l > 1) {
+      const int mid = (l + h) >> 1;
+      if (cta[mid] <= i) l = mid; else h = mid;
+    }
+    s = l;
+    const int64_t b = (int64_t)off[l] * bpr, e = (int64_t)off[l + 1] * bpr;
+    const int k = i - cta[l], cnt = cta[l + 1] - cta[l];
+    lo = b + cta_begin(k, cnt, e - b);
+    hi = b + cta_begin(k + 1, cnt, e - b);
+  }
+};
+
 // A batch of same-shaped tensors (layers) quantized by one launch: segment s
 // is layer s with its own input pointer and its own tensor scale; codes and
 // scales are contiguous across layers (global block index), guidance bits
@@ -112,11 +145,6 @@ struct SegBatch {
                                       (uintptr_t)(start(first_kept) * bits_per_block));
   }
 };
-
-__device__ __forceinline__ int64_t cta_begin(int64_t i, int64_t grid, int64_t n) {
-  const int64_t q = n / grid, r = n % grid;
-  return i * q + (i < r ? i : r);
-}
 
 // ------------------------------------------------------- debug bounds
 // Builds with TF4_DEBUG_BOUNDS check every work unit a kernel is about to
@@ -1506,23 +1534,22 @@ __global__ void __launch_bounds__(kThreads, guided_min_ctas<FMT>()) k_guided(Gui
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
   __shared__ GuidedTables tb;
-  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
-  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
-  GuidedMode md;
-  int64_t lo = b0;
-  while (lo < b1) {
-    const int s = seg.find(lo);
-    const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
-    float st = 0.0f;
-    if constexpr (kE4M3<FMT>) {
-      st = a.rec_s_t[s];
-      build_tables<UG, false>(st, tb);
-      build_block_tables(st, tb);
-    }
-    if (kE4M3<FMT> && tb.rz) guided_piece<FMT, true>(a, lo, hi, tb, md);
-    else guided_piece<FMT, false>(a, lo, hi, tb, md);
-    lo = hi;
+  int s = 0;
+  int64_t lo, hi;
+  if constexpr (std::is_same<SEG, SegPieces>::value) {
+    seg.piece(blockIdx.x, s, lo, hi);
+  } else {
+    lo = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+    hi = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   }
+  GuidedMode md;
+  if constexpr (kE4M3<FMT>) {
+    const float st = a.rec_s_t[s];
+    build_tables<UG, false>(st, tb);
+    build_block_tables(st, tb);
+  }
+  if (kE4M3<FMT> && tb.rz) guided_piece<FMT, true>(a, lo, hi, tb, md);
+  else guided_piece<FMT, false>(a, lo, hi, tb, md);
 }
 
 // --------------------------------------------- fused guided fake-quant
@@ -1661,23 +1688,22 @@ __global__ void __launch_bounds__(kThreads, kGuidedFqMinCtas) k_guided_fq(Guided
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
   __shared__ GuidedTables tb;
-  const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
-  const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
-  GuidedMode md;
-  int64_t lo = b0;
-  while (lo < b1) {
-    const int s = seg.find(lo);
-    const int64_t hi = (s + 1 < seg.count()) ? min(b1, seg.start(s + 1)) : b1;
-    float st = 0.0f;
-    if constexpr (kE4M3<FMT>) {
-      st = a.rec_s_t[s];
-      build_tables<UG, false>(st, tb);
-      build_block_tables(st, tb);
-    }
-    if (kE4M3<FMT> && tb.rz) guided_fq_piece<FMT, OUT, true>(a, lo, hi, tb, md);
-    else guided_fq_piece<FMT, OUT, false>(a, lo, hi, tb, md);
-    lo = hi;
+  int s = 0;
+  int64_t lo, hi;
+  if constexpr (std::is_same<SEG, SegPieces>::value) {
+    seg.piece(blockIdx.x, s, lo, hi);
+  } else {
+    lo = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
+    hi = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   }
+  GuidedMode md;
+  if constexpr (kE4M3<FMT>) {
+    const float st = a.rec_s_t[s];
+    build_tables<UG, false>(st, tb);
+    build_block_tables(st, tb);
+  }
+  if (kE4M3<FMT> && tb.rz) guided_fq_piece<FMT, OUT, true>(a, lo, hi, tb, md);
+  else guided_fq_piece<FMT, OUT, false>(a, lo, hi, tb, md);
 }
 
 // ------------------------------------------------ mismatch diagnostics

@@ -73,6 +73,30 @@ tf4::SegN make_segn(const Shape& sh) {
   return s;
 }
 
+// Ragged segments for the guided kernels: each non-empty segment gets its
+// own CTAs, about grid_target x its share of the blocks (at least one, at
+// most one per block).
+tf4::SegPieces make_segpieces(const Shape& sh, int64_t grid_target) {
+  tf4::SegPieces p;
+  std::memset(&p, 0, sizeof p);
+  p.nseg = sh.nseg;
+  p.bpr = sh.cols / sh.be;
+  for (int k = 0; k <= sh.nseg; ++k) p.off[k] = (int32_t)sh.off[k];
+  const int64_t n = sh.nblocks > 0 ? sh.nblocks : 1;
+  int64_t c = 0;
+  for (int k = 0; k < sh.nseg; ++k) {
+    p.cta[k] = (int32_t)c;
+    const int64_t len = (int64_t)(sh.off[k + 1] - sh.off[k]) * p.bpr;
+    if (len > 0) {
+      int64_t cnt = (len * grid_target + n / 2) / n;
+      cnt = cnt < 1 ? 1 : (cnt > len ? len : cnt);
+      c += cnt;
+    }
+  }
+  p.cta[sh.nseg] = (int32_t)c;
+  return p;
+}
+
 bool multi(const Shape& sh) { return sh.nseg > 1; }
 
 int sm_count() {
@@ -543,8 +567,9 @@ tf4_status tf4_quantize_guided(const tf4_desc* desc, const void* x, const uint8_
     constexpr int FMT = decltype(f)::value;
     if constexpr (tf4::kE4M3<FMT>) {
       if (multi(sh)) {
-        const int64_t g = wave_grid(tf4::k_guided<FMT, tf4::SegN>, sh.nblocks, sh.be);
-        launch_k(tf4::k_guided<FMT, tf4::SegN>, g, st, a, make_segn(sh));
+        const tf4::SegPieces p =
+            make_segpieces(sh, wave_grid(tf4::k_guided<FMT, tf4::SegPieces>, sh.nblocks, sh.be));
+        launch_k(tf4::k_guided<FMT, tf4::SegPieces>, p.cta[p.nseg], st, a, p);
         return;
       }
     }
@@ -579,8 +604,14 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
   a.status = status;
 #define TF4_LAUNCH_FQ(FMT, SEG, OUT, segv)                                            \
   do {                                                                                \
-    const int64_t g = wave_grid(tf4::k_guided_fq<FMT, SEG, OUT>, sh.nblocks, sh.be);         \
+    const int64_t g = wave_grid(tf4::k_guided_fq<FMT, SEG, OUT>, sh.nblocks, sh.be);   \
     launch_k(tf4::k_guided_fq<FMT, SEG, OUT>, g, st, a, segv);                        \
+  } while (0)
+#define TF4_LAUNCH_FQ_PIECES(FMT, OUT)                                                \
+  do {                                                                                \
+    const tf4::SegPieces p = make_segpieces(                                          \
+        sh, wave_grid(tf4::k_guided_fq<FMT, tf4::SegPieces, OUT>, sh.nblocks, sh.be)); \
+    launch_k(tf4::k_guided_fq<FMT, tf4::SegPieces, OUT>, p.cta[p.nseg], st, a, p);     \
   } while (0)
   // fp32 output: one 32-byte store per 8 elements when out allows it
   const int mode = out_bf16 ? tf4::kOutBf16 : (aligned(out, 32) ? tf4::kOutF32V8 : tf4::kOutF32);
@@ -588,9 +619,9 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
     constexpr int FMT = decltype(f)::value;
     if constexpr (tf4::kE4M3<FMT>) {
       if (multi(sh)) {
-        if (mode == tf4::kOutBf16) TF4_LAUNCH_FQ(FMT, tf4::SegN, tf4::kOutBf16, make_segn(sh));
-        else if (mode == tf4::kOutF32V8) TF4_LAUNCH_FQ(FMT, tf4::SegN, tf4::kOutF32V8, make_segn(sh));
-        else TF4_LAUNCH_FQ(FMT, tf4::SegN, tf4::kOutF32, make_segn(sh));
+        if (mode == tf4::kOutBf16) TF4_LAUNCH_FQ_PIECES(FMT, tf4::kOutBf16);
+        else if (mode == tf4::kOutF32V8) TF4_LAUNCH_FQ_PIECES(FMT, tf4::kOutF32V8);
+        else TF4_LAUNCH_FQ_PIECES(FMT, tf4::kOutF32);
         return;
       }
     }
@@ -599,6 +630,7 @@ tf4_status tf4_guided_fake_quant(const tf4_desc* desc, const void* x, const uint
     else TF4_LAUNCH_FQ(FMT, tf4::Seg1, tf4::kOutF32, tf4::Seg1{});
   });
 #undef TF4_LAUNCH_FQ
+#undef TF4_LAUNCH_FQ_PIECES
   return launched();
 }
 
