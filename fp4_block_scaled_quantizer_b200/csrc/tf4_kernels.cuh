@@ -1398,18 +1398,22 @@ __device__ __forceinline__ void report_bad_lane(bool bad, int32_t* status) {
 
 // One block of a guided pass: its codeword-safe multiplier r (0 when the
 // block takes the exact comparisons, whose codes then go to c) and whether
-// it holds a non-finite input.
-template <int FMT>
+// it holds a non-finite input.  Uniform grid: `clamp` when a product may
+// reach 7.5 (the block max times r, rounded as the products are, bounds
+// them all), else the conversions may skip their clamp.
+template <int FMT, bool RZ>
 __device__ __forceinline__ float guided_block_r(const uint32_t (&w)[kE4M3<FMT> ? 8 : 16], uint32_t sc, uint32_t g,
                                                 const GuidedTables& tb, uint32_t (&c)[kE4M3<FMT> ? 2 : 4],
-                                                bool& bad) {
+                                                bool& bad, bool& clamp) {
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int NQ = BE / 8;
-  bad = block_absmax_bits(w) >= 0x7F80u;
+  const uint32_t mb = block_absmax_bits(w);
+  bad = mb >= 0x7F80u;
   float r;
   if constexpr (kE4M3<FMT>) r = tb.rblk[sc];
   else r = (sc >= 1u && sc <= 252u) ? __uint_as_float((254u - sc) << 23) : 0.0f;  // 2^-(sc-127), exact
+  clamp = UG && !(mul<RZ>(__uint_as_float(mb << 16), r) < 7.5f);
   if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
     float S;
     if constexpr (kE4M3<FMT>) S = tb.sblk[sc];
@@ -1474,18 +1478,31 @@ __device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, in
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       uint32_t c[NQ], mm[NQ];
-      bool bad = false;
+      bool bad = false, clamp = false;
       float r = 0.0f;
-      if (ok[u]) r = guided_block_r<FMT>(w[u], sc[u], g[u], tb, c, bad);
+      if (ok[u]) r = guided_block_r<FMT, RZ>(w[u], sc[u], g[u], tb, c, bad, clamp);
       const bool fast = ok[u] && r != 0.0f;
+      if (UG) clamp = __any_sync(0xFFFFFFFFu, clamp);  // one conversion per warp
+#pragma unroll
+      for (int q = 0; q < NQ; ++q) mm[q] = 0u;
+      if (fast) {
+        if (UG && clamp) {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const uint32_t* wq = &w[u][4 * q];
+            c[q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const uint32_t* wq = &w[u][4 * q];
+            c[q] = nearest_x8<RZ, UG, false>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
+          }
+        }
+      }
       uint32_t any = 0u;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) {
-        const uint32_t* wq = &w[u][4 * q];
-        mm[q] = 0u;
-        if (fast) c[q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
-        any |= mm[q];
-      }
+      for (int q = 0; q < NQ; ++q) any |= mm[q];
       if (md.note(any != 0u)) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
@@ -1501,15 +1518,27 @@ __device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, in
     const int64_t k = j + tid;
     const bool ok = k < n && unit_ok(lo + k, lo, hi, a.nblocks);
     uint32_t w[NW], sc = 0u, g = 0u, c[NQ];
-    bool bad = false;
+    bool bad = false, clamp = false;
+    float r = 0.0f;
     if (ok) {
       guided_load<FMT>(a, lo + k, w, sc, g);
-      const float r = guided_block_r<FMT>(w, sc, g, tb, c, bad);
+      r = guided_block_r<FMT, RZ>(w, sc, g, tb, c, bad, clamp);
+    }
+    if (UG) clamp = __any_sync(0xFFFFFFFFu, clamp);  // one conversion per warp
+    if (ok) {
       if (r != 0.0f) {
+        if (UG && clamp) {
 #pragma unroll
-        for (int q = 0; q < NQ; ++q) {
-          const uint32_t* wq = &w[4 * q];
-          c[q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g >> (8 * q));
+          for (int q = 0; q < NQ; ++q) {
+            const uint32_t* wq = &w[4 * q];
+            c[q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g >> (8 * q));
+          }
+        } else {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            const uint32_t* wq = &w[4 * q];
+            c[q] = guided_x8<RZ, UG, false>(wq[0], wq[1], wq[2], wq[3], r, g >> (8 * q));
+          }
         }
       }
       guided_store<FMT>(a, lo + k, c);
@@ -1581,11 +1610,12 @@ enum { kOutBf16 = 0, kOutF32 = 1, kOutF32V8 = 2 };
 // One oct of the fused pass: scale S of its block, codeword-safe multiplier
 // r (0 when the oct takes the exact comparisons, whose codes then go to c)
 // and whether it holds a non-finite input.
-template <int FMT>
+template <int FMT, bool RZ>
 __device__ __forceinline__ float fq_oct_r(const uint32_t (&w)[4], uint32_t sc, uint32_t g, const GuidedTables& tb,
-                                          float& S, uint32_t& c, bool& bad) {
+                                          float& S, uint32_t& c, bool& bad, bool& clamp) {
   constexpr bool UG = kUni<FMT>;
-  bad = block_absmax_bits(w) >= 0x7F80u;
+  const uint32_t mb = block_absmax_bits(w);
+  bad = mb >= 0x7F80u;
   float r;
   if constexpr (kE4M3<FMT>) {
     S = tb.sblk[sc];
@@ -1594,6 +1624,7 @@ __device__ __forceinline__ float fq_oct_r(const uint32_t (&w)[4], uint32_t sc, u
     S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
     r = (sc >= 1u && sc <= 252u) ? __uint_as_float((254u - sc) << 23) : 0.0f;
   }
+  clamp = UG && !(mul<RZ>(__uint_as_float(mb << 16), r) < 7.5f);
   if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
     c = 0u;
 #pragma unroll
@@ -1655,9 +1686,13 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
       const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
       uint32_t c = 0u, mm = 0u;
       float r = 0.0f, S = 0.0f;
-      bool bad = false;
-      if (ok[u]) r = fq_oct_r<FMT>(w, sc[u], g[u], tb, S, c, bad);
-      if (ok[u] && r != 0.0f) c = nearest_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u], mm);
+      bool bad = false, clamp = false;
+      if (ok[u]) r = fq_oct_r<FMT, RZ>(w, sc[u], g[u], tb, S, c, bad, clamp);
+      if (UG) clamp = __any_sync(0xFFFFFFFFu, clamp);  // one conversion per warp
+      if (ok[u] && r != 0.0f) {
+        if (UG && clamp) c = nearest_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u], mm);
+        else c = nearest_x8<RZ, UG, false>(w[0], w[1], w[2], w[3], r, g[u], mm);
+      }
       if (md.note(mm != 0u) && mm != 0u) c = guided_x8_call<RZ, UG>(w[0], w[1], w[2], w[3], r, g[u]);
       if (ok[u]) fq_store<FMT, OUT>(a, ob + u * kThreads + tid, c, S);
       report_bad_lane(bad, a.status);
@@ -1666,15 +1701,22 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
   for (; ob < o1; ob += kThreads) {
     const int64_t o = ob + tid;
     const bool ok = o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB);
-    bool bad = false;
+    bool bad = false, clamp = false;
+    uint32_t w[4] = {0u, 0u, 0u, 0u}, g = 0u, c = 0u;
+    float r = 0.0f, S = 0.0f;
     if (ok) {
       const uint4 xv = __ldg(a.x + o);
-      const uint32_t sc = __ldg(a.rec_scales + o / OPB), g = __ldg(a.rec_bits + o);
-      const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
-      uint32_t c = 0u;
-      float S = 0.0f;
-      const float r = fq_oct_r<FMT>(w, sc, g, tb, S, c, bad);
-      if (r != 0.0f) c = guided_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g);
+      const uint32_t sc = __ldg(a.rec_scales + o / OPB);
+      g = __ldg(a.rec_bits + o);
+      w[0] = xv.x; w[1] = xv.y; w[2] = xv.z; w[3] = xv.w;
+      r = fq_oct_r<FMT, RZ>(w, sc, g, tb, S, c, bad, clamp);
+    }
+    if (UG) clamp = __any_sync(0xFFFFFFFFu, clamp);  // one conversion per warp
+    if (ok) {
+      if (r != 0.0f) {
+        if (UG && clamp) c = guided_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g);
+        else c = guided_x8<RZ, UG, false>(w[0], w[1], w[2], w[3], r, g);
+      }
       fq_store<FMT, OUT>(a, o, c, S);
     }
     report_bad_lane(bad, a.status);
