@@ -213,6 +213,27 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float v0, float v1, float v2, flo
   return r;
 }
 
+// Eight fp32 values -> eight E2M3 codes (hardware RNE, satfinite): element
+// k in byte k & 3 of b[k >> 2], each byte s << 5 | e << 3 | m.
+__device__ __forceinline__ void cvt_e2m3x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
+                                           float v7, uint32_t& b0, uint32_t& b1) {
+  asm("{\n\t.reg .b16 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 q0, %3, %2;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 q1, %5, %4;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 q2, %7, %6;\n\t"
+      "cvt.rn.satfinite.e2m3x2.f32 q3, %9, %8;\n\t"
+      "mov.b32 %0, {q0, q1};\n\t"
+      "mov.b32 %1, {q2, q3};\n\t}"
+      : "=r"(b0), "=r"(b1)
+      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
+}
+
+// Four bytes holding values < 16 in each of two words -> eight nibbles
+// (byte k of w0 -> nibble k, byte k of w1 -> nibble 4 + k).
+__device__ __forceinline__ uint32_t pack_nibbles(uint32_t w0, uint32_t w1) {
+  return __byte_perm(w0 | (w0 >> 4), w1 | (w1 >> 4), 0x6420);
+}
+
 // Eight fp32 values -> eight uniform-grid nibbles: round |v| to the nearest
 // integer, ties to even (adding 2^23 does exactly that: the sum is rounded
 // once, to a neighbouring integer), saturating at 7; sign bit kept.  Element
@@ -736,32 +757,30 @@ __device__ __forceinline__ float block_rho(float rho_c, uint32_t e_b) {
   return __uint_as_float(__float_as_uint(rho_c) + (uint32_t)((7 - (int)e_b) << 23));
 }
 
-// Uniform grid, 4 bf16 (two words) times r -> the 4 nibble bytes
-// [n0, n1, n2, n3] (byte i = sign<<3 | k_i).  k = round-half-even of |v|:
-// 2^23 + |v| is rounded once, to an integer, whose value sits in the low
-// mantissa bits (byte 0 of the fp32 pattern while k < 256).  CLAMP
-// saturates |v| at 7 first; without it the caller guarantees |v| < 7.5.
-// The signs are the bf16 sign bits (byte_perm picks the high byte of each
-// bf16; bit 7 of each byte moves to bit 3).
-template <bool RZ, bool CLAMP>
-__device__ __forceinline__ uint32_t uni_bytes4(uint32_t w0, uint32_t w1, float r) {
-  const float v[4] = {mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r), mul<RZ>(bf_hi(w1), r)};
-  uint32_t t[4];
-#pragma unroll
-  for (int k = 0; k < 4; ++k)
-    t[k] = __float_as_uint(__fadd_rn(CLAMP ? fminf(fabsf(v[k]), 7.0f) : fabsf(v[k]), 0x1p23f));
-  const uint32_t k4 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-  return k4 | ((__byte_perm(w0, w1, 0x7531) >> 4) & 0x08080808u);
-}
-
-// Nibble bytes [n0, n1, n2, n3] -> n0 | n1 << 4 in byte 0 and n2 | n3 << 4
-// in byte 2 (bytes 1 and 3 are don't-care).
-__device__ __forceinline__ uint32_t nib_pairs(uint32_t b) { return b | (b >> 4); }
-
+// Uniform grid through the E2M3 conversion: the E2M3 values below 2 are
+// the multiples of 1/8 (subnormals m/8, then 1 + m/8), so for |v| < 7.5 RNE
+// of v/8 to E2M3 is RNE of v to an integer k <= 7, held in the code's
+// magnitude bits (ties to even m are ties to even k); v/8 = RN(x r)/8 =
+// RN(x (r/8)) exactly (a power-of-two factor; below the normal range both
+// round to code 0).  CLAMP: larger |v| (magnitude bits >= 8, up to the
+// satfinite maximum) saturate to k = 7.  Byte s << 5 | k -> nibble
+// s << 3 | k.  (Non-finite inputs give unspecified codes.)
 template <bool RZ, bool CLAMP>
 __device__ __forceinline__ uint32_t cvt_uni_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r) {
-  return __byte_perm(nib_pairs(uni_bytes4<RZ, CLAMP>(w0, w1, r)), nib_pairs(uni_bytes4<RZ, CLAMP>(w2, w3, r)),
-                     0x6420);
+  const float r8 = r * 0.125f;
+  uint32_t b[2];
+  cvt_e2m3x8(mul<RZ>(bf_lo(w0), r8), mul<RZ>(bf_hi(w0), r8), mul<RZ>(bf_lo(w1), r8), mul<RZ>(bf_hi(w1), r8),
+             mul<RZ>(bf_lo(w2), r8), mul<RZ>(bf_hi(w2), r8), mul<RZ>(bf_lo(w3), r8), mul<RZ>(bf_hi(w3), r8), b[0],
+             b[1]);
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    if (CLAMP) {
+      const uint32_t t = (b[h] | (b[h] >> 1)) & 0x08080808u;  // magnitude >= 8
+      b[h] |= t - (t >> 3);                                   // -> low three bits all ones
+    }
+    b[h] = ((b[h] >> 2) & 0x08080808u) | (b[h] & 0x07070707u);
+  }
+  return pack_nibbles(b[0], b[1]);
 }
 
 // Eight bf16 (four words) times rho -> eight grid nibbles (signed, RNE).
@@ -1228,54 +1247,26 @@ struct GuidedArgs {
   int32_t* status;
 };
 
-// Eight fp32 values -> eight E2M3 codes (hardware RNE, satfinite): element
-// k in byte k & 3 of b[k >> 2], each byte s << 5 | e << 3 | m.
-__device__ __forceinline__ void cvt_e2m3x8(float v0, float v1, float v2, float v3, float v4, float v5, float v6,
-                                           float v7, uint32_t& b0, uint32_t& b1) {
-  asm("{\n\t.reg .b16 q0, q1, q2, q3;\n\t"
-      "cvt.rn.satfinite.e2m3x2.f32 q0, %3, %2;\n\t"
-      "cvt.rn.satfinite.e2m3x2.f32 q1, %5, %4;\n\t"
-      "cvt.rn.satfinite.e2m3x2.f32 q2, %7, %6;\n\t"
-      "cvt.rn.satfinite.e2m3x2.f32 q3, %9, %8;\n\t"
-      "mov.b32 %0, {q0, q1};\n\t"
-      "mov.b32 %1, {q2, q3};\n\t}"
-      : "=r"(b0), "=r"(b1)
-      : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
-}
-
 // Fine codes of eight elements (bf16 pairs w0..w3) times r, four per word
-// as above.  Uniform grid: N = RN(2 min(|y|, 7.5)) read from the low byte
-// of 2^22 + min(|y|, 7.5), placed as f << 2 | (N & 1) << 1, sign from x.
+// as above.  Uniform grid: N = RN(2 min(|y|, 7.5)), from RNE of y/4 to
+// E2M3 (as in cvt_uni_words, at half the step: magnitude bits = N, clamped
+// to 15 when CLAMP), placed as s << 5 | N << 1 = s << 5 | f << 2 |
+// (N & 1) << 1.
 template <bool RZ, bool U, bool CLAMP>
 __device__ __forceinline__ void fine_codes(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
                                            uint32_t& b0, uint32_t& b1) {
+  const float rr = U ? r * 0.25f : r;
+  cvt_e2m3x8(mul<RZ>(bf_lo(w0), rr), mul<RZ>(bf_hi(w0), rr), mul<RZ>(bf_lo(w1), rr), mul<RZ>(bf_hi(w1), rr),
+             mul<RZ>(bf_lo(w2), rr), mul<RZ>(bf_hi(w2), rr), mul<RZ>(bf_lo(w3), rr), mul<RZ>(bf_hi(w3), rr), b0, b1);
   if constexpr (U) {
-    const uint32_t w[4] = {w0, w1, w2, w3};
-    uint32_t o[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t t[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t wk = w[2 * h + (k >> 1)];
-        const float v = mul<RZ>((k & 1) ? bf_hi(wk) : bf_lo(wk), r);
-        t[k] = __float_as_uint(__fadd_rn(CLAMP ? fminf(fabsf(v), 7.5f) : fabsf(v), 0x1p22f));
-      }
-      const uint32_t n4 = __byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410);
-      o[h] = (n4 << 1) | ((__byte_perm(w[2 * h], w[2 * h + 1], 0x7531) >> 2) & 0x20202020u);
+    if (CLAMP) {
+      const uint32_t t0 = b0 & 0x10101010u, t1 = b1 & 0x10101010u;  // N >= 16
+      b0 |= t0 - (t0 >> 4);                                        // -> low four bits all ones
+      b1 |= t1 - (t1 >> 4);
     }
-    b0 = o[0];
-    b1 = o[1];
-  } else {
-    cvt_e2m3x8(mul<RZ>(bf_lo(w0), r), mul<RZ>(bf_hi(w0), r), mul<RZ>(bf_lo(w1), r), mul<RZ>(bf_hi(w1), r),
-               mul<RZ>(bf_lo(w2), r), mul<RZ>(bf_hi(w2), r), mul<RZ>(bf_lo(w3), r), mul<RZ>(bf_hi(w3), r), b0, b1);
+    b0 = ((b0 << 1) & 0x1E1E1E1Eu) | (b0 & 0x20202020u);
+    b1 = ((b1 << 1) & 0x1E1E1E1Eu) | (b1 & 0x20202020u);
   }
-}
-
-// Four bytes holding values < 16 in each of two words -> eight nibbles
-// (byte k of w0 -> nibble k, byte k of w1 -> nibble 4 + k).
-__device__ __forceinline__ uint32_t pack_nibbles(uint32_t w0, uint32_t w1) {
-  return __byte_perm(w0 | (w0 >> 4), w1 | (w1 >> 4), 0x6420);
 }
 
 // 8 guidance bits -> bit 0 of 8 nibbles (shift-or steps written as
@@ -1398,22 +1389,18 @@ __device__ __forceinline__ void report_bad_lane(bool bad, int32_t* status) {
 
 // One block of a guided pass: its codeword-safe multiplier r (0 when the
 // block takes the exact comparisons, whose codes then go to c) and whether
-// it holds a non-finite input.  Uniform grid: `clamp` when a product may
-// reach 7.5 (the block max times r, rounded as the products are, bounds
-// them all), else the conversions may skip their clamp.
-template <int FMT, bool RZ>
+// it holds a non-finite input.
+template <int FMT>
 __device__ __forceinline__ float guided_block_r(const uint32_t (&w)[kE4M3<FMT> ? 8 : 16], uint32_t sc, uint32_t g,
                                                 const GuidedTables& tb, uint32_t (&c)[kE4M3<FMT> ? 2 : 4],
-                                                bool& bad, bool& clamp) {
+                                                bool& bad) {
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int NQ = BE / 8;
-  const uint32_t mb = block_absmax_bits(w);
-  bad = mb >= 0x7F80u;
+  bad = block_absmax_bits(w) >= 0x7F80u;
   float r;
   if constexpr (kE4M3<FMT>) r = tb.rblk[sc];
   else r = (sc >= 1u && sc <= 252u) ? __uint_as_float((254u - sc) << 23) : 0.0f;  // 2^-(sc-127), exact
-  clamp = UG && !(mul<RZ>(__uint_as_float(mb << 16), r) < 7.5f);
   if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
     float S;
     if constexpr (kE4M3<FMT>) S = tb.sblk[sc];
@@ -1478,31 +1465,18 @@ __device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, in
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       uint32_t c[NQ], mm[NQ];
-      bool bad = false, clamp = false;
+      bool bad = false;
       float r = 0.0f;
-      if (ok[u]) r = guided_block_r<FMT, RZ>(w[u], sc[u], g[u], tb, c, bad, clamp);
+      if (ok[u]) r = guided_block_r<FMT>(w[u], sc[u], g[u], tb, c, bad);
       const bool fast = ok[u] && r != 0.0f;
-      if (UG) clamp = __any_sync(0xFFFFFFFFu, clamp);  // one conversion per warp
-#pragma unroll
-      for (int q = 0; q < NQ; ++q) mm[q] = 0u;
-      if (fast) {
-        if (UG && clamp) {
-#pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const uint32_t* wq = &w[u][4 * q];
-            c[q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const uint32_t* wq = &w[u][4 * q];
-            c[q] = nearest_x8<RZ, UG, false>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
-          }
-        }
-      }
       uint32_t any = 0u;
 #pragma unroll
-      for (int q = 0; q < NQ; ++q) any |= mm[q];
+      for (int q = 0; q < NQ; ++q) {
+        const uint32_t* wq = &w[u][4 * q];
+        mm[q] = 0u;
+        if (fast) c[q] = nearest_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g[u] >> (8 * q), mm[q]);
+        any |= mm[q];
+      }
       if (md.note(any != 0u)) {
 #pragma unroll
         for (int q = 0; q < NQ; ++q) {
@@ -1518,27 +1492,15 @@ __device__ __forceinline__ void guided_piece(const GuidedArgs& a, int64_t lo, in
     const int64_t k = j + tid;
     const bool ok = k < n && unit_ok(lo + k, lo, hi, a.nblocks);
     uint32_t w[NW], sc = 0u, g = 0u, c[NQ];
-    bool bad = false, clamp = false;
-    float r = 0.0f;
+    bool bad = false;
     if (ok) {
       guided_load<FMT>(a, lo + k, w, sc, g);
-      r = guided_block_r<FMT, RZ>(w, sc, g, tb, c, bad, clamp);
-    }
-    if (UG) clamp = __any_sync(0xFFFFFFFFu, clamp);  // one conversion per warp
-    if (ok) {
+      const float r = guided_block_r<FMT>(w, sc, g, tb, c, bad);
       if (r != 0.0f) {
-        if (UG && clamp) {
 #pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const uint32_t* wq = &w[4 * q];
-            c[q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g >> (8 * q));
-          }
-        } else {
-#pragma unroll
-          for (int q = 0; q < NQ; ++q) {
-            const uint32_t* wq = &w[4 * q];
-            c[q] = guided_x8<RZ, UG, false>(wq[0], wq[1], wq[2], wq[3], r, g >> (8 * q));
-          }
+        for (int q = 0; q < NQ; ++q) {
+          const uint32_t* wq = &w[4 * q];
+          c[q] = guided_x8<RZ, UG, true>(wq[0], wq[1], wq[2], wq[3], r, g >> (8 * q));
         }
       }
       guided_store<FMT>(a, lo + k, c);
@@ -1610,12 +1572,11 @@ enum { kOutBf16 = 0, kOutF32 = 1, kOutF32V8 = 2 };
 // One oct of the fused pass: scale S of its block, codeword-safe multiplier
 // r (0 when the oct takes the exact comparisons, whose codes then go to c)
 // and whether it holds a non-finite input.
-template <int FMT, bool RZ>
+template <int FMT>
 __device__ __forceinline__ float fq_oct_r(const uint32_t (&w)[4], uint32_t sc, uint32_t g, const GuidedTables& tb,
-                                          float& S, uint32_t& c, bool& bad, bool& clamp) {
+                                          float& S, uint32_t& c, bool& bad) {
   constexpr bool UG = kUni<FMT>;
-  const uint32_t mb = block_absmax_bits(w);
-  bad = mb >= 0x7F80u;
+  bad = block_absmax_bits(w) >= 0x7F80u;
   float r;
   if constexpr (kE4M3<FMT>) {
     S = tb.sblk[sc];
@@ -1624,7 +1585,6 @@ __device__ __forceinline__ float fq_oct_r(const uint32_t (&w)[4], uint32_t sc, u
     S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
     r = (sc >= 1u && sc <= 252u) ? __uint_as_float((254u - sc) << 23) : 0.0f;
   }
-  clamp = UG && !(mul<RZ>(__uint_as_float(mb << 16), r) < 7.5f);
   if (r == 0.0f) {  // no codeword-safe multiplier: exact comparisons per element
     c = 0u;
 #pragma unroll
@@ -1686,13 +1646,9 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
       const uint32_t w[4] = {xv[u].x, xv[u].y, xv[u].z, xv[u].w};
       uint32_t c = 0u, mm = 0u;
       float r = 0.0f, S = 0.0f;
-      bool bad = false, clamp = false;
-      if (ok[u]) r = fq_oct_r<FMT, RZ>(w, sc[u], g[u], tb, S, c, bad, clamp);
-      if (UG) clamp = __any_sync(0xFFFFFFFFu, clamp);  // one conversion per warp
-      if (ok[u] && r != 0.0f) {
-        if (UG && clamp) c = nearest_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u], mm);
-        else c = nearest_x8<RZ, UG, false>(w[0], w[1], w[2], w[3], r, g[u], mm);
-      }
+      bool bad = false;
+      if (ok[u]) r = fq_oct_r<FMT>(w, sc[u], g[u], tb, S, c, bad);
+      if (ok[u] && r != 0.0f) c = nearest_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u], mm);
       if (md.note(mm != 0u) && mm != 0u) c = guided_x8_call<RZ, UG>(w[0], w[1], w[2], w[3], r, g[u]);
       if (ok[u]) fq_store<FMT, OUT>(a, ob + u * kThreads + tid, c, S);
       report_bad_lane(bad, a.status);
@@ -1701,22 +1657,15 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
   for (; ob < o1; ob += kThreads) {
     const int64_t o = ob + tid;
     const bool ok = o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB);
-    bool bad = false, clamp = false;
-    uint32_t w[4] = {0u, 0u, 0u, 0u}, g = 0u, c = 0u;
-    float r = 0.0f, S = 0.0f;
+    bool bad = false;
     if (ok) {
       const uint4 xv = __ldg(a.x + o);
-      const uint32_t sc = __ldg(a.rec_scales + o / OPB);
-      g = __ldg(a.rec_bits + o);
-      w[0] = xv.x; w[1] = xv.y; w[2] = xv.z; w[3] = xv.w;
-      r = fq_oct_r<FMT, RZ>(w, sc, g, tb, S, c, bad, clamp);
-    }
-    if (UG) clamp = __any_sync(0xFFFFFFFFu, clamp);  // one conversion per warp
-    if (ok) {
-      if (r != 0.0f) {
-        if (UG && clamp) c = guided_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g);
-        else c = guided_x8<RZ, UG, false>(w[0], w[1], w[2], w[3], r, g);
-      }
+      const uint32_t sc = __ldg(a.rec_scales + o / OPB), g = __ldg(a.rec_bits + o);
+      const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
+      uint32_t c = 0u;
+      float S = 0.0f;
+      const float r = fq_oct_r<FMT>(w, sc, g, tb, S, c, bad);
+      if (r != 0.0f) c = guided_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g);
       fq_store<FMT, OUT>(a, o, c, S);
     }
     report_bad_lane(bad, a.status);
