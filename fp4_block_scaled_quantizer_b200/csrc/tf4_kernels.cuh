@@ -304,6 +304,35 @@ __device__ __forceinline__ float4 decode4_grid(uint32_t c, float S) {
   else return decode4(c, S);
 }
 
+// Eight nibbles (a code word) -> v0 (elements 0..3), v1 (4..7), as
+// decode4_grid twice; on the uniform grid the nibbles are spread to bytes
+// for all eight at once (byte_perm of the even and odd nibbles).
+template <bool U>
+__device__ __forceinline__ void decode8_grid(uint32_t c, float S, float4& v0, float4& v1) {
+  if constexpr (U) {
+    if (S <= 0x1p100f) {
+      const uint32_t lo = c & 0x0F0F0F0Fu, hi = (c >> 4) & 0x0F0F0F0Fu;  // nibbles 0,2,4,6 / 1,3,5,7
+      uint32_t p[2] = {__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362)};
+      const float S9 = S * 512.0f;  // exact
+      float4 v[2];
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        p[h] = (p[h] & 0x07070707u) | ((p[h] & 0x08080808u) << 4);
+        const __half2_raw h0 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(p[h] & 0xFFFFu), __NV_E4M3);
+        const __half2_raw h1 = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(p[h] >> 16), __NV_E4M3);
+        const float2 f0 = __half22float2(__half2(h0));
+        const float2 f1 = __half22float2(__half2(h1));
+        v[h] = make_float4(__fmul_rn(f0.x, S9), __fmul_rn(f0.y, S9), __fmul_rn(f1.x, S9), __fmul_rn(f1.y, S9));
+      }
+      v0 = v[0];
+      v1 = v[1];
+      return;
+    }
+  }
+  v0 = decode4_grid<U>(c & 0xFFFFu, S);
+  v1 = decode4_grid<U>(c >> 16, S);
+}
+
 // One 32-byte store (sm_100 256-bit vector store); p must be 32-B aligned.
 __device__ __forceinline__ void st_v8(float* p, const float4& a, const float4& b) {
   asm volatile("st.global.v8.f32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "f"(a.x), "f"(a.y), "f"(a.z),
@@ -772,14 +801,15 @@ __device__ __forceinline__ uint32_t cvt_uni_words(uint32_t w0, uint32_t w1, uint
   cvt_e2m3x8(mul<RZ>(bf_lo(w0), r8), mul<RZ>(bf_hi(w0), r8), mul<RZ>(bf_lo(w1), r8), mul<RZ>(bf_hi(w1), r8),
              mul<RZ>(bf_lo(w2), r8), mul<RZ>(bf_hi(w2), r8), mul<RZ>(bf_lo(w3), r8), mul<RZ>(bf_hi(w3), r8), b[0],
              b[1]);
+  if (CLAMP && ((b[0] | b[1]) & 0x18181818u)) {  // some magnitude >= 8 (rare unless train values leave the grid)
 #pragma unroll
-  for (int h = 0; h < 2; ++h) {
-    if (CLAMP) {
+    for (int h = 0; h < 2; ++h) {
       const uint32_t t = (b[h] | (b[h] >> 1)) & 0x08080808u;  // magnitude >= 8
       b[h] |= t - (t >> 3);                                   // -> low three bits all ones
     }
-    b[h] = ((b[h] >> 2) & 0x08080808u) | (b[h] & 0x07070707u);
   }
+#pragma unroll
+  for (int h = 0; h < 2; ++h) b[h] = ((b[h] >> 2) & 0x08080808u) | (b[h] & 0x07070707u);
   return pack_nibbles(b[0], b[1]);
 }
 
@@ -1259,9 +1289,9 @@ __device__ __forceinline__ void fine_codes(uint32_t w0, uint32_t w1, uint32_t w2
   cvt_e2m3x8(mul<RZ>(bf_lo(w0), rr), mul<RZ>(bf_hi(w0), rr), mul<RZ>(bf_lo(w1), rr), mul<RZ>(bf_hi(w1), rr),
              mul<RZ>(bf_lo(w2), rr), mul<RZ>(bf_hi(w2), rr), mul<RZ>(bf_lo(w3), rr), mul<RZ>(bf_hi(w3), rr), b0, b1);
   if constexpr (U) {
-    if (CLAMP) {
-      const uint32_t t0 = b0 & 0x10101010u, t1 = b1 & 0x10101010u;  // N >= 16
-      b0 |= t0 - (t0 >> 4);                                        // -> low four bits all ones
+    if (CLAMP && ((b0 | b1) & 0x10101010u)) {  // some N >= 16 (rare unless train values leave the grid)
+      const uint32_t t0 = b0 & 0x10101010u, t1 = b1 & 0x10101010u;
+      b0 |= t0 - (t0 >> 4);                    // -> low four bits all ones
       b1 |= t1 - (t1 >> 4);
     }
     b0 = ((b0 << 1) & 0x1E1E1E1Eu) | (b0 & 0x20202020u);
@@ -1603,7 +1633,8 @@ template <int FMT, int OUT>
 __device__ __forceinline__ void fq_store(const GuidedFqArgs& a, int64_t o, uint32_t c, float S) {
   constexpr bool UG = kUni<FMT>;
   if (a.codes) reinterpret_cast<uint32_t*>(a.codes)[o] = c;
-  const float4 v0 = decode4_grid<UG>(c & 0xFFFFu, S), v1 = decode4_grid<UG>(c >> 16, S);
+  float4 v0, v1;
+  decode8_grid<UG>(c, S, v0, v1);
   if constexpr (OUT == kOutBf16) {
     reinterpret_cast<uint4*>(a.out)[o] = make_uint4(bf16x2_bits(v0.x, v0.y), bf16x2_bits(v0.z, v0.w),
                                                     bf16x2_bits(v1.x, v1.y), bf16x2_bits(v1.z, v1.w));
@@ -1950,7 +1981,9 @@ __global__ void __launch_bounds__(kThreads) k_dequant8(DequantArgs a, SEG seg) {
           float S;
           if constexpr (kE4M3<FMT>) S = __fmul_rn(st, e4m3_decode(sc[u]));
           else S = __uint_as_float(sc[u] >= 1u ? sc[u] << 23 : 0x00400000u);
-          st_v8(out + 8 * o, decode4_grid<kUni<FMT>>(cw[u] & 0xFFFFu, S), decode4_grid<kUni<FMT>>(cw[u] >> 16, S));
+          float4 v0, v1;
+          decode8_grid<kUni<FMT>>(cw[u], S, v0, v1);
+          st_v8(out + 8 * o, v0, v1);
         }
       }
     }

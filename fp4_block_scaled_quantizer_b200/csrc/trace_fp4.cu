@@ -210,14 +210,6 @@ constexpr int64_t kFusedMaxElems = int64_t(1) << 25;
 // its amax phase over 64 MiB takes about 10 us.
 constexpr uint64_t kFusedWaitNs = 100000000ull;
 
-int64_t fused_max_elems() {
-  static const int64_t v = [] {
-    const char* e = getenv("TF4_FUSED_MAX_ELEMS");
-    return e ? (int64_t)atoll(e) : kFusedMaxElems;
-  }();
-  return v;
-}
-
 // Resident CTAs per SM of `kernel` with `smem` bytes of dynamic shared
 // memory on the current device (not cached).
 int occupancy_smem(const void* kernel, size_t smem) {
@@ -308,7 +300,7 @@ tf4_status quantize_impl(const tf4_desc* d, const void* x, uint64_t seed, const 
       if constexpr (tf4::kE4M3<FMT>) {
         const int64_t grid = nvfp4_grid<FMT, MODE>(sh);
         if constexpr (MODE != tf4::kSR) {
-          if (!amax_in && !multi(sh) && sh.n <= fused_max_elems()) {
+          if (!amax_in && !multi(sh) && sh.n <= kFusedMaxElems) {
             e = launch_fused<FMT, MODE>(sh, a, static_cast<uint32_t*>(ws), pk, st);
             return;
           }
