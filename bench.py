@@ -177,10 +177,15 @@ def hbm_peak():
 
 
 def kernel_source_hash():
+    """Hash of the kernel sources' code: line comments and blank lines are
+    left out, so that a comment edit does not void committed counters."""
     h = hashlib.sha256()
     for rel in ("fp4_block_scaled_quantizer_b200/csrc/tf4_kernels.cuh", "fp4_block_scaled_quantizer_b200/csrc/trace_fp4.cu"):
-        with open(os.path.join(ROOT, rel), "rb") as f:
-            h.update(f.read())
+        with open(os.path.join(ROOT, rel), encoding="utf-8") as f:
+            for line in f:
+                code = line.split("//", 1)[0].rstrip()
+                if code:
+                    h.update(code.encode() + b"\n")
     return h.hexdigest()[:16]
 
 

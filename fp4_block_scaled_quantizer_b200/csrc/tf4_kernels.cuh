@@ -1251,8 +1251,9 @@ __global__ void __launch_bounds__(kThreads) k_quant_fused(QuantArgs a, uint32_t*
 // bits, 3 mantissa bits, subnormals 0..7/8) for the E2M1 grid -- an E2M1
 // value with code m3 is the E2M3 value with code m3 << 2 -- and the
 // half-integers for the uniform grid.  Let N be the fine code of y
-// (hardware RNE; for the uniform grid 2^22 + |y| is rounded once to a
-// multiple of 1/2), f = N >> 2 its codeword part and l = N & 3 the rest:
+// (hardware RNE; for the uniform grid the E2M3 rounding of y/4, whose
+// spacing below 2 is 1/8, i.e. y to a multiple of 1/2), f = N >> 2 its
+// codeword part and l = N & 3 the rest (uniform grid: N = 2f + l, l = N & 1):
 //  * l != 0: N lies strictly between two codewords, and so does y (a tie
 //    between N and a codeword goes to the codeword, whose code is even):
 //    the answer is f + ((f ^ g) & 1), capped at 7;
