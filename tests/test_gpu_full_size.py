@@ -171,3 +171,20 @@ def test_moe_dispatch_every_row(pool, fmt):
 def test_kv_cache_k_every_row(pool, fmt):
     w = W.kv_cache(DEV)
     check_all(pool, fmt, w["k"], w["k_train"])
+
+
+@pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4, O.MXFP4])
+def test_guided_phases_mixed_within_ranges(pool, fmt):
+    """A 16384x4096 train copy perturbed (rel 5e-2) on every fourth band of 8
+    rows and equal to the rollout tensor elsewhere.  Each CTA's range spans
+    several iterations, some clean and some with mismatches, so warps run the
+    nearest phase with and without fine-rounding calls and switch to the
+    fine phase at different points of their ranges; every element of the
+    guided codes, the fused pass and the counts equals the oracle's."""
+    x = W.layer_stack_layer(27, DEV, rows=16384)
+    hot = W.perturb(x, 1027, rel=5e-2)
+    band = (torch.arange(x.shape[0], device=DEV) // 8) % 4 == 0
+    xt = torch.where(band[:, None], hot, x)
+    del hot
+    counts = check_all(pool, fmt, x, xt)
+    assert 0.002 * x.numel() < counts[0] < 0.03 * x.numel()
