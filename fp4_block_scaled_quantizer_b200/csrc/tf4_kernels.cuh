@@ -1374,10 +1374,11 @@ __device__ __forceinline__ uint32_t nearest_x8(uint32_t w0, uint32_t w1, uint32_
 
 // Per warp, guided rounding starts with nearest rounding plus the fine
 // rounding for the (warp-uniform) iterations where some lane's nearest code
-// has the wrong bit.  A score (one register) gains 4 on such an iteration
-// and loses 1 on a clean one, kept within [-16, 0]; once it passes 0 (at
-// least 3 such iterations in a row from the start, or about one in four
-// later on) the warp takes the fine rounding for the rest of its range.
+// has the wrong bit.  A score (one register, starting at -8) gains 4 on
+// such an iteration and loses 1 on a clean one, never going below -16; once
+// it passes 0 (three such iterations in a row from the start, or a run in
+// which more than one iteration in five has one) the warp takes the fine
+// rounding for the rest of its range.
 struct GuidedMode {
   int score = -8;
   __device__ __forceinline__ bool fine() const { return score > 0; }
