@@ -1278,17 +1278,19 @@ struct GuidedArgs {
   int32_t* status;
 };
 
-// Fine codes of eight elements (bf16 pairs w0..w3) times r, four per word
-// as above.  Uniform grid: N = RN(2 min(|y|, 7.5)), from RNE of y/4 to
-// E2M3 (as in cvt_uni_words, at half the step: magnitude bits = N, clamped
-// to 15 when CLAMP), placed as s << 5 | N << 1 = s << 5 | f << 2 |
+// Fine codes of eight elements (bf16 pairs w0..w3) times r, one byte each
+// as above: b0 holds the even elements (element 2j in byte j), b1 the odd
+// ones (element 2j + 1 in byte j), so that one shift-and-merge puts both
+// into nibble order.  Uniform grid: N = RN(2 min(|y|, 7.5)), from RNE of
+// y/4 to E2M3 (as in cvt_uni_words, at half the step: magnitude bits = N,
+// clamped to 15 when CLAMP), placed as s << 5 | N << 1 = s << 5 | f << 2 |
 // (N & 1) << 1.
 template <bool RZ, bool U, bool CLAMP>
 __device__ __forceinline__ void fine_codes(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
                                            uint32_t& b0, uint32_t& b1) {
   const float rr = U ? r * 0.25f : r;
-  cvt_e2m3x8(mul<RZ>(bf_lo(w0), rr), mul<RZ>(bf_hi(w0), rr), mul<RZ>(bf_lo(w1), rr), mul<RZ>(bf_hi(w1), rr),
-             mul<RZ>(bf_lo(w2), rr), mul<RZ>(bf_hi(w2), rr), mul<RZ>(bf_lo(w3), rr), mul<RZ>(bf_hi(w3), rr), b0, b1);
+  cvt_e2m3x8(mul<RZ>(bf_lo(w0), rr), mul<RZ>(bf_lo(w1), rr), mul<RZ>(bf_lo(w2), rr), mul<RZ>(bf_lo(w3), rr),
+             mul<RZ>(bf_hi(w0), rr), mul<RZ>(bf_hi(w1), rr), mul<RZ>(bf_hi(w2), rr), mul<RZ>(bf_hi(w3), rr), b0, b1);
   if constexpr (U) {
     if (CLAMP && ((b0 | b1) & 0x10101010u)) {  // some N >= 16 (rare unless train values leave the grid)
       const uint32_t t0 = b0 & 0x10101010u, t1 = b1 & 0x10101010u;
@@ -1342,13 +1344,14 @@ __device__ __noinline__ uint32_t guided_sides(uint32_t c, uint32_t P, uint32_t f
 template <bool RZ, bool U, bool CLAMP>
 __device__ __forceinline__ uint32_t guided_x8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
                                               uint32_t g8) {
-  uint32_t b0, b1;
-  fine_codes<RZ, U, CLAMP>(w0, w1, w2, w3, r, b0, b1);
-  const uint32_t P = pack_nibbles((b0 >> 2) & 0x0F0F0F0Fu, (b1 >> 2) & 0x0F0F0F0Fu);
-  const uint32_t A = (P ^ spread_bits(g8)) & 0x11111111u;       // f's bit != g
-  const uint32_t F7 = P & (P >> 1) & (P >> 2) & 0x11111111u;    // f == 7
+  uint32_t be, bo;  // fine codes of the even / odd elements
+  fine_codes<RZ, U, CLAMP>(w0, w1, w2, w3, r, be, bo);
+  const uint32_t P = ((be >> 2) & 0x0F0F0F0Fu) | ((bo << 2) & 0xF0F0F0F0u);  // s << 3 | f, nibble k = element k
+  const uint32_t A = (P ^ spread_bits(g8)) & 0x11111111u;                   // f's bit != g
+  const uint32_t F7 = P & (P >> 1) & (P >> 2) & 0x11111111u;                // f == 7
   const uint32_t c = P + (A & ~F7);
-  const uint32_t fl = A & ~pack_nibbles((b0 | (b0 >> 1)) & 0x01010101u, (b1 | (b1 >> 1)) & 0x01010101u);
+  const uint32_t L = ((be | (be >> 1)) & 0x01010101u) | (((bo | (bo >> 1)) << 4) & 0x10101010u);  // l != 0
+  const uint32_t fl = A & ~L;
   return fl ? guided_sides<RZ, U>(c, P, fl, w0, w1, w2, w3, r) : c;
 }
 
