@@ -228,11 +228,6 @@ __device__ __forceinline__ void cvt_e2m3x8(float v0, float v1, float v2, float v
       : "f"(v0), "f"(v1), "f"(v2), "f"(v3), "f"(v4), "f"(v5), "f"(v6), "f"(v7));
 }
 
-// Four bytes holding values < 16 in each of two words -> eight nibbles
-// (byte k of w0 -> nibble k, byte k of w1 -> nibble 4 + k).
-__device__ __forceinline__ uint32_t pack_nibbles(uint32_t w0, uint32_t w1) {
-  return __byte_perm(w0 | (w0 >> 4), w1 | (w1 >> 4), 0x6420);
-}
 
 // Eight fp32 values -> eight uniform-grid nibbles: round |v| to the nearest
 // integer, ties to even (adding 2^23 does exactly that: the sum is rounded
@@ -797,9 +792,9 @@ __device__ __forceinline__ float block_rho(float rho_c, uint32_t e_b) {
 template <bool RZ, bool CLAMP>
 __device__ __forceinline__ uint32_t cvt_uni_words(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r) {
   const float r8 = r * 0.125f;
-  uint32_t b[2];
-  cvt_e2m3x8(mul<RZ>(bf_lo(w0), r8), mul<RZ>(bf_hi(w0), r8), mul<RZ>(bf_lo(w1), r8), mul<RZ>(bf_hi(w1), r8),
-             mul<RZ>(bf_lo(w2), r8), mul<RZ>(bf_hi(w2), r8), mul<RZ>(bf_lo(w3), r8), mul<RZ>(bf_hi(w3), r8), b[0],
+  uint32_t b[2];  // E2M3 bytes of the even / odd elements (element 2j, 2j + 1 in byte j)
+  cvt_e2m3x8(mul<RZ>(bf_lo(w0), r8), mul<RZ>(bf_lo(w1), r8), mul<RZ>(bf_lo(w2), r8), mul<RZ>(bf_lo(w3), r8),
+             mul<RZ>(bf_hi(w0), r8), mul<RZ>(bf_hi(w1), r8), mul<RZ>(bf_hi(w2), r8), mul<RZ>(bf_hi(w3), r8), b[0],
              b[1]);
   if (CLAMP && ((b[0] | b[1]) & 0x18181818u)) {  // some magnitude >= 8 (rare unless train values leave the grid)
 #pragma unroll
@@ -808,9 +803,9 @@ __device__ __forceinline__ uint32_t cvt_uni_words(uint32_t w0, uint32_t w1, uint
       b[h] |= t - (t >> 3);                                   // -> low three bits all ones
     }
   }
-#pragma unroll
-  for (int h = 0; h < 2; ++h) b[h] = ((b[h] >> 2) & 0x08080808u) | (b[h] & 0x07070707u);
-  return pack_nibbles(b[0], b[1]);
+  // even element -> low nibble of byte j, odd -> high nibble: s << 3 | k
+  return ((b[0] >> 2) & 0x08080808u) | (b[0] & 0x07070707u) | ((b[1] << 2) & 0x80808080u) |
+         ((b[1] << 4) & 0x70707070u);
 }
 
 // Eight bf16 (four words) times rho -> eight grid nibbles (signed, RNE).
@@ -1282,9 +1277,8 @@ struct GuidedArgs {
 // as above: b0 holds the even elements (element 2j in byte j), b1 the odd
 // ones (element 2j + 1 in byte j), so that one shift-and-merge puts both
 // into nibble order.  Uniform grid: N = RN(2 min(|y|, 7.5)), from RNE of
-// y/4 to E2M3 (as in cvt_uni_words, at half the step: magnitude bits = N,
-// clamped to 15 when CLAMP), placed as s << 5 | N << 1 = s << 5 | f << 2 |
-// (N & 1) << 1.
+// y/4 to E2M3 (as in cvt_uni_words, at half the step): byte s << 5 | N,
+// N clamped to 15 when CLAMP.
 template <bool RZ, bool U, bool CLAMP>
 __device__ __forceinline__ void fine_codes(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
                                            uint32_t& b0, uint32_t& b1) {
@@ -1297,8 +1291,6 @@ __device__ __forceinline__ void fine_codes(uint32_t w0, uint32_t w1, uint32_t w2
       b0 |= t0 - (t0 >> 4);                    // -> low four bits all ones
       b1 |= t1 - (t1 >> 4);
     }
-    b0 = ((b0 << 1) & 0x1E1E1E1Eu) | (b0 & 0x20202020u);
-    b1 = ((b1 << 1) & 0x1E1E1E1Eu) | (b1 & 0x20202020u);
   }
 }
 
@@ -1346,11 +1338,18 @@ __device__ __forceinline__ uint32_t guided_x8(uint32_t w0, uint32_t w1, uint32_t
                                               uint32_t g8) {
   uint32_t be, bo;  // fine codes of the even / odd elements
   fine_codes<RZ, U, CLAMP>(w0, w1, w2, w3, r, be, bo);
-  const uint32_t P = ((be >> 2) & 0x0F0F0F0Fu) | ((bo << 2) & 0xF0F0F0F0u);  // s << 3 | f, nibble k = element k
-  const uint32_t A = (P ^ spread_bits(g8)) & 0x11111111u;                   // f's bit != g
-  const uint32_t F7 = P & (P >> 1) & (P >> 2) & 0x11111111u;                // f == 7
+  uint32_t P, L;    // s << 3 | f and (bit 0) l != 0, nibble k = element k
+  if constexpr (U) {  // byte s << 5 | N, N = 2f + l
+    P = ((be >> 2) & 0x08080808u) | ((be >> 1) & 0x07070707u) | ((bo << 2) & 0x80808080u) |
+        ((bo << 3) & 0x70707070u);
+    L = (be & 0x01010101u) | ((bo << 4) & 0x10101010u);
+  } else {            // byte s << 5 | f << 2 | l
+    P = ((be >> 2) & 0x0F0F0F0Fu) | ((bo << 2) & 0xF0F0F0F0u);
+    L = ((be | (be >> 1)) & 0x01010101u) | (((bo | (bo >> 1)) << 4) & 0x10101010u);
+  }
+  const uint32_t A = (P ^ spread_bits(g8)) & 0x11111111u;       // f's bit != g
+  const uint32_t F7 = P & (P >> 1) & (P >> 2) & 0x11111111u;    // f == 7
   const uint32_t c = P + (A & ~F7);
-  const uint32_t L = ((be | (be >> 1)) & 0x01010101u) | (((bo | (bo >> 1)) << 4) & 0x10101010u);  // l != 0
   const uint32_t fl = A & ~L;
   return fl ? guided_sides<RZ, U>(c, P, fl, w0, w1, w2, w3, r) : c;
 }
