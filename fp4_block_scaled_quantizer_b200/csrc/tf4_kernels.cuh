@@ -1659,20 +1659,23 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
                                                 const GuidedTables& tb, GuidedMode& md) {
   constexpr bool UG = kUni<FMT>;
   constexpr int OPB = kE4M3<FMT> ? 2 : 4;  // octs per block
+  constexpr int OPB_LOG = kE4M3<FMT> ? 1 : 2;
   const int tid = threadIdx.x;
   const int64_t o0 = lo * OPB, o1 = hi * OPB;
-  int64_t ob = o0;
-  for (; ob < o1 && !md.fine(); ob += 2 * kThreads) {
+  const int n = (int)(o1 - o0);  // one CTA's share of a segment: far below 2^31 octs
+  int kb = 0;
+  for (; kb < n && !md.fine(); kb += 2 * kThreads) {
     uint4 xv[2];
     uint32_t sc[2], g[2];
     bool ok[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int64_t o = ob + u * kThreads + tid;
-      ok[u] = o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB);
+      const int k = kb + u * kThreads + tid;
+      const int64_t o = o0 + k;
+      ok[u] = k < n && unit_ok(o, o0, o1, a.nblocks * OPB);
       if (ok[u]) {
         xv[u] = __ldg(a.x + o);
-        sc[u] = __ldg(a.rec_scales + o / OPB);
+        sc[u] = __ldg(a.rec_scales + (o >> OPB_LOG));
         g[u] = __ldg(a.rec_bits + o);
       }
     }
@@ -1685,17 +1688,18 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
       if (ok[u]) r = fq_oct_r<FMT>(w, sc[u], g[u], tb, S, c, bad);
       if (ok[u] && r != 0.0f) c = nearest_x8<RZ, UG, true>(w[0], w[1], w[2], w[3], r, g[u], mm);
       if (md.note(mm != 0u) && mm != 0u) c = guided_x8_call<RZ, UG>(w[0], w[1], w[2], w[3], r, g[u]);
-      if (ok[u]) fq_store<FMT, OUT>(a, ob + u * kThreads + tid, c, S);
+      if (ok[u]) fq_store<FMT, OUT>(a, o0 + kb + u * kThreads + tid, c, S);
       report_bad_lane(bad, a.status);
     }
   }
-  for (; ob < o1; ob += kThreads) {
-    const int64_t o = ob + tid;
-    const bool ok = o < o1 && unit_ok(o, o0, o1, a.nblocks * OPB);
+  for (; kb < n; kb += kThreads) {
+    const int k = kb + tid;
+    const int64_t o = o0 + k;
+    const bool ok = k < n && unit_ok(o, o0, o1, a.nblocks * OPB);
     bool bad = false;
     if (ok) {
       const uint4 xv = __ldg(a.x + o);
-      const uint32_t sc = __ldg(a.rec_scales + o / OPB), g = __ldg(a.rec_bits + o);
+      const uint32_t sc = __ldg(a.rec_scales + (o >> OPB_LOG)), g = __ldg(a.rec_bits + o);
       const uint32_t w[4] = {xv.x, xv.y, xv.z, xv.w};
       uint32_t c = 0u;
       float S = 0.0f;
