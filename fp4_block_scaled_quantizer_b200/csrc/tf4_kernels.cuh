@@ -1662,15 +1662,19 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
   constexpr int OPB_LOG = kE4M3<FMT> ? 1 : 2;
   const int tid = threadIdx.x;
   const int64_t o0 = lo * OPB, o1 = hi * OPB;
-  const int n = (int)(o1 - o0);  // one CTA's share of a segment: far below 2^31 octs
-  int kb = 0;
+  // oct counters within the piece (one CTA's share of a segment: far below
+  // 2^31 octs); 32-bit ones measured faster except for NVFP4's fp32 output,
+  // where they cost registers
+  using Idx = std::conditional_t<kE4M3<FMT> && !kUni<FMT> && OUT != kOutBf16, int64_t, int>;
+  const Idx n = (Idx)(o1 - o0);
+  Idx kb = 0;
   for (; kb < n && !md.fine(); kb += 2 * kThreads) {
     uint4 xv[2];
     uint32_t sc[2], g[2];
     bool ok[2];
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
-      const int k = kb + u * kThreads + tid;
+      const Idx k = kb + u * kThreads + tid;
       const int64_t o = o0 + k;
       ok[u] = k < n && unit_ok(o, o0, o1, a.nblocks * OPB);
       if (ok[u]) {
@@ -1693,7 +1697,7 @@ __device__ __forceinline__ void guided_fq_piece(const GuidedFqArgs& a, int64_t l
     }
   }
   for (; kb < n; kb += kThreads) {
-    const int k = kb + tid;
+    const Idx k = kb + tid;
     const int64_t o = o0 + k;
     const bool ok = k < n && unit_ok(o, o0, o1, a.nblocks * OPB);
     bool bad = false;
