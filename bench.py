@@ -73,6 +73,9 @@ def parse():
                    help="time every call of the path on every workload (a table, not the bench line)")
     p.add_argument("--only", action="append",
                    help="with --suite: run only rows matching workload-prefix[:format[:call]] (repeatable)")
+    p.add_argument("--mismatch-by-layer", action="store_true",
+                   help="per layer of the stack: the diagnostics' counts of the train copy against the layer's "
+                        "capture, the corrections split by direction (a table, not the bench line)")
     return p.parse_args()
 
 
@@ -581,6 +584,32 @@ CALL_BYTES = {
 CALL_BYTES.update({("ufp4", c): v for (f, c), v in list(CALL_BYTES.items()) if f == "nvfp4"})
 
 
+def run_mismatch_by_layer(args):
+    """For every layer of the stack: NVFP4 capture of the layer, its train
+    copy drawn as the benchmark draws it (seed 1000 + layer, --train-rel),
+    and the diagnostics' counts -- nearest-rounding mismatches, adjacent or
+    farther, after guidance, and the corrections guidance makes toward the
+    smaller and toward the larger codeword."""
+    from fp4_block_scaled_quantizer_b200 import binding as B
+    from fp4_block_scaled_quantizer_b200 import build as libbuild
+    from fp4_block_scaled_quantizer_b200 import workloads as W
+
+    libbuild.build()
+    dev = torch.device("cuda", 0)
+    out = []
+    cnt = torch.zeros(B.MISMATCH_COUNTS, dtype=torch.int64, device=dev)
+    for layer in range(args.layers):
+        x = W.layer_stack_layer(layer, dev, rows=args.rows, cols=args.cols)
+        q = B.tf4_quantize_capture(x)
+        xt = W.perturb(x, 1000 + layer, rel=args.train_rel)
+        c = [int(v) for v in B.tf4_mismatch_stats(xt, q, counts=cnt.zero_()).tolist()]
+        out.append(dict(layer=layer, elements=x.numel(), mismatch=c[0], adjacent=c[1], far=c[2], after_guidance=c[3],
+                        toward_smaller=c[4], toward_larger=c[5]))
+        del x, q, xt
+    return dict(workload=f"layer_stack: {args.layers} layers x {args.rows}x{args.cols} bf16, NVFP4 capture, "
+                         f"train copy x (1 + {args.train_rel:g} N(0,1))", rows=out)
+
+
 def run_suite(args):
     """Every call of the path on every workload, CUDA-event timed (3 warm-up
     calls, then the mean of 10); GB/s from the algorithmic bytes above."""
@@ -861,6 +890,9 @@ def main():
     args = parse()
     if args.suite:
         print(json.dumps(run_suite(args)), flush=True)
+        return
+    if args.mismatch_by_layer:
+        print(json.dumps(run_mismatch_by_layer(args)), flush=True)
         return
     if args.impl == "reference":
         world = int(os.environ.get("WORLD_SIZE", "1"))
