@@ -612,7 +612,9 @@ def run_mismatch_by_layer(args):
 
 def run_suite(args):
     """Every call of the path on every workload, CUDA-event timed (3 warm-up
-    calls, then the mean of 10); GB/s from the algorithmic bytes above."""
+    calls, then the mean of 10 back-to-back calls, and the median and minimum
+    of 20 calls timed one by one); GB/s from the algorithmic bytes above and
+    the mean."""
     from fp4_block_scaled_quantizer_b200 import binding as B
     from fp4_block_scaled_quantizer_b200 import build as libbuild
     from fp4_block_scaled_quantizer_b200 import workloads as W
@@ -633,6 +635,20 @@ def run_suite(args):
         b.record()
         torch.cuda.synchronize()
         return a.elapsed_time(b) / reps * 1e3  # us
+
+    def per_call(fn, reps=20, flush=None):
+        """Median and minimum of reps calls, each between its own pair of
+        events (optionally after `flush`, outside the events)."""
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        for a, b in ev:
+            if flush is not None:
+                flush()
+            a.record()
+            fn()
+            b.record()
+        torch.cuda.synchronize()
+        t = sorted(a.elapsed_time(b) * 1e3 for a, b in ev)
+        return dict(us_median=round(0.5 * (t[(reps - 1) // 2] + t[reps // 2]), 2), us_min=round(t[0], 2))
 
     only = [tuple(f.split(":")) + ("", "", "") for f in (args.only or [])]
 
@@ -686,16 +702,18 @@ def run_suite(args):
     def run(workload, fmt, call, n, fn, cold=False, **extra):
         if not sel(workload, fmt, call):
             return
+        flush = lambda: flush_buf[0].zero_()  # noqa: E731 (timed_cold allocates flush_buf first)
         if cold:
-            record(workload, fmt, call, n, timed(fn), l2="warm", **extra)
+            record(workload, fmt, call, n, timed(fn), l2="warm", **per_call(fn), **extra)
             record(workload, fmt, call, n, timed_graph(fn), l2="warm, CUDA graph", **extra)
-            record(workload, fmt, call, n, timed_cold(fn), l2="cold", **extra)
+            record(workload, fmt, call, n, timed_cold(fn), l2="cold", **per_call(fn, flush=flush), **extra)
         elif CALL_BYTES[(fmt, call)] * n < 2 * L2_BYTES:
             # a working set that back-to-back calls would find in L2: flush before each call so that
             # the figure is an HBM one
-            record(workload, fmt, call, n, timed_cold(fn), l2="cold (flushed: working set < 2 x L2)", **extra)
+            record(workload, fmt, call, n, timed_cold(fn), l2="cold (flushed: working set < 2 x L2)",
+                   **per_call(fn, flush=flush), **extra)
         else:
-            record(workload, fmt, call, n, timed(fn), **extra)
+            record(workload, fmt, call, n, timed(fn), **per_call(fn), **extra)
 
     def record(workload, fmt, call, n, us, l2=None, **extra):
         gbs = CALL_BYTES[(fmt, call)] * n / (us * 1e-6) / 1e9
