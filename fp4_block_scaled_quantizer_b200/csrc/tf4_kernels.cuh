@@ -1799,13 +1799,17 @@ __device__ __forceinline__ void count_diffs(uint32_t cx, uint32_t co, uint32_t (
 // no verified multiplier exists; the code words are then compared with the
 // rollout's nibble-wise, and only differing nibbles are classified.
 template <int FMT, class SEG>
-__global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) {
+__global__ void __launch_bounds__(kThreads, (kE4M3<FMT> && std::is_same<SEG, Seg1>::value) ? 6 : 1)
+    k_mismatch(MismatchArgs a, SEG seg) {
   pdl_enter();
   constexpr bool UG = kUni<FMT>;
   constexpr int BE = kE4M3<FMT> ? 16 : 32;
   constexpr int NW = BE / 2;
   constexpr int NQ = BE / 8;
   __shared__ SegTables tmid, tcw;
+  // per recorded scale byte: the multipliers of the two tables (0: exact
+  // comparisons) and the block scale, one shared-memory load each per block
+  __shared__ float rm_of[256], rc_of[256], s_of[256];
   const int64_t b0 = cta_begin(blockIdx.x, gridDim.x, a.nblocks);
   const int64_t b1 = cta_begin(blockIdx.x + 1, gridDim.x, a.nblocks);
   uint32_t cnt[kMismatchCounts] = {0u, 0u, 0u, 0u, 0u, 0u};
@@ -1817,7 +1821,18 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
     const float st = kE4M3<FMT> ? a.rec_s_t[s] : 0.0f;
     if constexpr (kE4M3<FMT>) {
       build_tables<UG, true, false>(st, tmid);
-      build_tables<UG, false>(st, tcw);
+      build_tables<UG, false>(st, tcw);  // ends with a barrier: tmid and tcw are complete
+      static_assert(kThreads == 256, "one table entry per thread");
+      const uint32_t sc = threadIdx.x;
+      float rm = 0.0f, rc = 0.0f;
+      if ((sc >> 3) >= 1u && sc < 0x7Fu) {
+        if (tmid.fast && tmid.rho[sc & 7u] != 0.0f) rm = block_rho(tmid.rho[sc & 7u], sc >> 3);
+        if (tcw.fast && tcw.rho[sc & 7u] != 0.0f) rc = block_rho(tcw.rho[sc & 7u], sc >> 3);
+      }
+      rm_of[sc] = rm;
+      rc_of[sc] = rc;
+      s_of[sc] = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
+      __syncthreads();
     }
     for (int64_t blk = lo + threadIdx.x; blk < hi; blk += kThreads) {
       if (!unit_ok(blk, lo, hi, a.nblocks)) continue;
@@ -1838,17 +1853,11 @@ __global__ void __launch_bounds__(kThreads) k_mismatch(MismatchArgs a, SEG seg) 
       float S, rm = 0.0f, rc = 0.0f;
       bool rzm = false, rzc = false;
       if constexpr (kE4M3<FMT>) {
-        S = st > 0.0f ? __fmul_rn(st, e4m3_decode(sc)) : 0.0f;
-        if ((sc >> 3) >= 1u && sc < 0x7Fu) {
-          if (tmid.fast && tmid.rho[sc & 7u] != 0.0f) {
-            rm = block_rho(tmid.rho[sc & 7u], sc >> 3);
-            rzm = tmid.rz;
-          }
-          if (tcw.fast && tcw.rho[sc & 7u] != 0.0f) {
-            rc = block_rho(tcw.rho[sc & 7u], sc >> 3);
-            rzc = tcw.rz;
-          }
-        }
+        S = s_of[sc];
+        rm = rm_of[sc];
+        rc = rc_of[sc];
+        rzm = tmid.rz;
+        rzc = tcw.rz;
       } else {
         S = __uint_as_float(sc >= 1u ? sc << 23 : 0x00400000u);
         if (sc >= 1u && sc <= 252u) rm = rc = __uint_as_float((254u - sc) << 23);  // 2^-(sc-127), exact
