@@ -468,6 +468,28 @@ def test_mismatch_stats_parity(fmt, seg, rel):
         assert want[0] == want[1] + want[2]
 
 
+def test_bench_mismatch_by_layer_counts():
+    """The bench's per-layer diagnostics mode (a few small layers of the
+    stack) reports, for every layer, the oracle's counts of that layer's
+    train copy against its capture."""
+    import argparse
+
+    import bench
+
+    args = argparse.Namespace(layers=3, rows=512, cols=1024, train_rel=0.05)
+    out = bench.run_mismatch_by_layer(args)
+    assert [r["layer"] for r in out["rows"]] == [0, 1, 2]
+    for r in out["rows"]:
+        x = W.layer_stack_layer(r["layer"], DEV, rows=512, cols=1024)
+        xs = W.bf16_bits(x)
+        rec = O.quantize(xs, O.NVFP4, O.RTN, bits=True)
+        xt = W.bf16_bits(W.perturb(x, 1000 + r["layer"], rel=0.05))
+        want = O.mismatch_stats(xt, rec["scales"], rec["codes"], O.NVFP4, rec_s_t=rec["s_t"])
+        got = [r[k] for k in ("mismatch", "adjacent", "far", "after_guidance", "toward_smaller", "toward_larger")]
+        assert got == want.tolist(), (r["layer"], got, want.tolist())
+        assert r["elements"] == x.numel()
+
+
 @pytest.mark.parametrize("fmt", [O.NVFP4, O.UFP4])
 def test_mismatch_stats_near_ties(fmt):
     """Train values on and around the recorded grid's midpoints and codewords:
