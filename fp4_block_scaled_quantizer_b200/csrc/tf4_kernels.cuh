@@ -1342,14 +1342,14 @@ __device__ __noinline__ uint32_t guided_sides(uint32_t c, uint32_t P, uint32_t f
   return c;
 }
 
-// Guided rounding of eight elements (bf16 pairs w0..w3; recorded bits g8,
-// element k in bit k) on the codeword-safe multiplier r -> eight nibbles.
-// In nibble form (P: s << 3 | f per element) the answer is f + ((f ^ g) & 1)
-// with f = 7 left as it is; elements with l = 0 whose f's bit differs from
-// g take the side test.
+// Guided rounding of eight elements (bf16 pairs w0..w3; recorded bits gs,
+// element k's bit at bit 4k) on the codeword-safe multiplier r -> eight
+// nibbles.  In nibble form (P: s << 3 | f per element) the answer is
+// f + ((f ^ g) & 1) with f = 7 left as it is; elements with l = 0 whose f's
+// bit differs from g take the side test.
 template <bool RZ, bool U, bool CLAMP>
-__device__ __forceinline__ uint32_t guided_x8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
-                                              uint32_t g8) {
+__device__ __forceinline__ uint32_t guided_x8_spread(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
+                                                     uint32_t gs) {
   uint32_t be, bo;  // fine codes of the even / odd elements
   fine_codes<RZ, U, CLAMP>(w0, w1, w2, w3, r, be, bo);
   uint32_t P, L;    // s << 3 | f and (bit 0) l != 0, nibble k = element k
@@ -1361,11 +1361,18 @@ __device__ __forceinline__ uint32_t guided_x8(uint32_t w0, uint32_t w1, uint32_t
     P = ((be >> 2) & 0x0F0F0F0Fu) | ((bo << 2) & 0xF0F0F0F0u);
     L = ((be | (be >> 1)) & 0x01010101u) | (((bo | (bo >> 1)) << 4) & 0x10101010u);
   }
-  const uint32_t A = (P ^ spread_bits(g8)) & 0x11111111u;       // f's bit != g
+  const uint32_t A = (P ^ gs) & 0x11111111u;                     // f's bit != g
   const uint32_t F7 = P & (P >> 1) & (P >> 2) & 0x11111111u;    // f == 7
   const uint32_t c = P + (A & ~F7);
   const uint32_t fl = A & ~L;
   return fl ? guided_sides<RZ, U>(c, P, fl, w0, w1, w2, w3, r) : c;
+}
+
+// The same with the recorded bits g8 packed (element k in bit k).
+template <bool RZ, bool U, bool CLAMP>
+__device__ __forceinline__ uint32_t guided_x8(uint32_t w0, uint32_t w1, uint32_t w2, uint32_t w3, float r,
+                                              uint32_t g8) {
+  return guided_x8_spread<RZ, U, CLAMP>(w0, w1, w2, w3, r, spread_bits(g8));
 }
 
 // The same as a call: the nearest-rounding loops recompute a word with it
@@ -1900,9 +1907,9 @@ __global__ void __launch_bounds__(kThreads, (kE4M3<FMT> && std::is_same<SEG, Seg
         // nibble can add to any count.
         if (cr == co) continue;
         if (rc != 0.0f) {
-          const uint32_t go = nibble_lsbs(co);  // the rollout codes' bits
-          cg = rzc ? guided_x8<true, UG, true>(wq[0], wq[1], wq[2], wq[3], rc, go)
-                   : guided_x8<false, UG, true>(wq[0], wq[1], wq[2], wq[3], rc, go);
+          const uint32_t gs = co & 0x11111111u;  // the rollout codes' bits, in place
+          cg = rzc ? guided_x8_spread<true, UG, true>(wq[0], wq[1], wq[2], wq[3], rc, gs)
+                   : guided_x8_spread<false, UG, true>(wq[0], wq[1], wq[2], wq[3], rc, gs);
         } else {
 #pragma unroll
           for (int e = 0; e < 8; ++e) {
